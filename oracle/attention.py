@@ -1,0 +1,270 @@
+"""Float64 CPU oracle: exact causal softmax attention with RoPE and packing mask.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  The product path never
+imports this module.
+
+What it computes, step by step, and where each step comes from:
+
+1. RoPE frequencies  w_i = theta ** (-2 i / D),  i = 0 .. D/2-1.
+   LWM research note, section "模型架构" (model architecture): "standard RoPE";
+   the RoFormer entry of the paper card's reference list fixes the form.
+   theta is the per-stage value of the note's section "训练方法" (32K: 1e6,
+   128K: 1e7, 256K: 1e7, 512K: 2.5e7, 1M: 5e7).
+2. Rotation of query and key vectors by angle p * w_i on the interleaved
+   pairs (x[2i], x[2i+1]), p = position of the token in its row.
+3. Scores  s_ij = scale * <q~_i, k~_j>.
+4. Mask  allowed(i, j) = seg_i == seg_j  and  seg_i >= 0  and  (j <= i if
+   causal).  Research note, section "训练方法", Masked Sequence Packing: each
+   packed sample attends only to itself.
+5. Exact softmax (paper card, Summary: "without approximation"):
+   LSE_i = ln sum_{allowed j} exp(s_ij),  P_ij = exp(s_ij - LSE_i) on allowed
+   pairs and 0 elsewhere,  O_i = sum_j P_ij v_j.
+6. Backward (the gradients that training through this layer needs; the
+   FlashAttention entry of the reference list recomputes P from LSE, which is
+   the same arithmetic):  dP_ij = <dO_i, v_j>,  D_i = sum_j P_ij dP_ij,
+   dS_ij = P_ij (dP_ij - D_i),  dq~_i = scale sum_j dS_ij k~_j,
+   dk~_j = scale sum_i dS_ij q~_i,  dv_j = sum_i P_ij dO_i,
+   dq = R(p)^T dq~,  dk = R(p)^T dk~.
+
+Scores are materialised one block of query rows at a time so memory stays
+bounded; there is no other blocking, fusion or reordering.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# Readings of points the pages leave open.  Each one is also listed in the
+# design notes of the repository.
+READINGS = {
+    "rope_pairing": "interleaved pairs (x[2i], x[2i+1]) as in the RoFormer formulation",
+    "rope_frequency": "w_i = theta ** (-2 i / D)",
+    "rope_positions": "p = index of the token in its row, continuing across packed segments "
+                      "(attention output and gradients are unchanged by a per-segment restart, "
+                      "since rotary scores depend only on i - j)",
+    "rope_disabled": "theta <= 0 disables the rotation",
+    "scale": "1/sqrt(D) unless given",
+    "padding": "segment id < 0 marks padding: O = 0, LSE = -inf, all gradients 0",
+    "lse_base": "natural log of the scaled scores",
+    "grad_wrt": "dq, dk are gradients with respect to the un-rotated inputs",
+}
+
+
+def rope_frequencies(head_dim: int, theta: float) -> np.ndarray:
+    """w_i = theta ** (-2 i / D) for i < D/2 (RoFormer form; LWM note, "模型架构")."""
+    if head_dim % 2:
+        raise ValueError("head_dim must be even for rotary pairs")
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(np.float64(theta), -2.0 * i / head_dim)
+
+
+def rope_angles(positions, head_dim: int, theta: float) -> np.ndarray:
+    """Angles p * w_i in float64, shape [len(positions), D/2]."""
+    p = np.asarray(positions, dtype=np.float64)
+    return np.multiply.outer(p, rope_frequencies(head_dim, theta))
+
+
+def rope_apply(x, theta: float, inverse: bool = False, position_offset: int = 0) -> np.ndarray:
+    """Rotate x of shape [B, S, H, D] by R(p), or by R(p)^T when ``inverse``.
+
+    Position p of token t is ``t + position_offset``.  Interleaved pairs
+    (x[2i], x[2i+1]) turn by angle p * w_i:
+        y[2i]   = x[2i] cos - x[2i+1] sin
+        y[2i+1] = x[2i] sin + x[2i+1] cos
+    theta <= 0 returns x unchanged (as float64).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if theta is None or theta <= 0:
+        return x.copy()
+    B, S, H, D = x.shape
+    ang = rope_angles(np.arange(S) + position_offset, D, theta)  # [S, D/2]
+    c = np.cos(ang)[None, :, None, :]
+    s = np.sin(ang)[None, :, None, :]
+    if inverse:
+        s = -s
+    xe = x[..., 0::2]
+    xo = x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = xe * c - xo * s
+    y[..., 1::2] = xe * s + xo * c
+    return y
+
+
+def allowed_mask(seg_row, q_idx, k_idx, causal: bool) -> np.ndarray:
+    """Boolean [len(q_idx), len(k_idx)]: same segment, not padding, causal order."""
+    seg_row = np.asarray(seg_row)
+    sq = seg_row[np.asarray(q_idx)][:, None]
+    sk = seg_row[np.asarray(k_idx)][None, :]
+    m = (sq == sk) & (sq >= 0)
+    if causal:
+        m &= np.asarray(k_idx)[None, :] <= np.asarray(q_idx)[:, None]
+    return m
+
+
+def _seg_or_default(seg, B, S):
+    if seg is None:
+        return np.zeros((B, S), dtype=np.int64)
+    seg = np.asarray(seg).astype(np.int64)
+    if seg.shape != (B, S):
+        raise ValueError(f"segment ids must be [B, S] = {(B, S)}, got {seg.shape}")
+    return seg
+
+
+def _scale(scale, D):
+    return 1.0 / np.sqrt(D) if (scale is None or scale <= 0) else float(scale)
+
+
+def _softmax_rows(s, allowed):
+    """LSE per row and P, exact in float64; rows with nothing allowed give LSE=-inf, P=0."""
+    sm = np.where(allowed, s, -np.inf)
+    m = np.max(sm, axis=1, initial=-np.inf)
+    has = np.isfinite(m)
+    m_safe = np.where(has, m, 0.0)
+    e = np.where(allowed, np.exp(s - m_safe[:, None]), 0.0)
+    tot = e.sum(axis=1)
+    lse = np.where(has, m_safe + np.log(np.where(has, tot, 1.0)), -np.inf)
+    p = np.where(allowed, np.exp(s - np.where(has, lse, 0.0)[:, None]), 0.0)
+    return lse, p
+
+
+def _rows_per_block(S):
+    return int(min(512, max(1, (1 << 24) // max(S, 1))))
+
+
+def attention_forward(q, k, v, seg=None, causal=True, theta=1e4, scale=None,
+                      position_offset=0):
+    """O [B,S,H,D] and LSE [B,H,S] in float64 (steps 1-5 of the module docstring)."""
+    out = attention_backward(q, k, v, None, seg=seg, causal=causal, theta=theta,
+                             scale=scale, position_offset=position_offset)
+    return out["o"], out["lse"]
+
+
+def attention_backward(q, k, v, d_o, seg=None, causal=True, theta=1e4, scale=None,
+                       row_start=0, position_offset=0):
+    """Forward plus (when ``d_o`` is given) backward, in float64.
+
+    Query rows ``[row_start, S)`` of every (batch, head) are processed.  The
+    returned ``o``, ``lse`` and ``dq`` are exact for those rows (other rows are
+    left at 0 / -inf).  ``dk`` and ``dv`` hold the contributions of those rows
+    only; with a causal mask that is the exact gradient of every key at
+    position >= row_start, which is how long inputs are checked on their last
+    rows without the full quadratic cost.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, S, H, D = q.shape
+    seg = _seg_or_default(seg, B, S)
+    sc = _scale(scale, D)
+    qt = rope_apply(q, theta, position_offset=position_offset)
+    kt = rope_apply(k, theta, position_offset=position_offset)
+    want_bwd = d_o is not None
+    if want_bwd:
+        d_o = np.asarray(d_o, dtype=np.float64)
+
+    o = np.zeros((B, S, H, D))
+    lse = np.full((B, H, S), -np.inf)
+    dqt = np.zeros((B, S, H, D)) if want_bwd else None
+    dkt = np.zeros((B, S, H, D)) if want_bwd else None
+    dv = np.zeros((B, S, H, D)) if want_bwd else None
+    blk = _rows_per_block(S)
+
+    for b in range(B):
+        for h in range(H):
+            Q, K, V = qt[b, :, h, :], kt[b, :, h, :], v[b, :, h, :]
+            for r0 in range(row_start, S, blk):
+                r1 = min(S, r0 + blk)
+                kend = r1 if causal else S
+                rows = np.arange(r0, r1)
+                keys = np.arange(kend)
+                s = sc * (Q[r0:r1] @ K[:kend].T)
+                allowed = allowed_mask(seg[b], rows, keys, causal)
+                l, P = _softmax_rows(s, allowed)
+                lse[b, h, r0:r1] = l
+                o[b, r0:r1, h, :] = P @ V[:kend]
+                if want_bwd:
+                    dO = d_o[b, r0:r1, h, :]
+                    dP = dO @ V[:kend].T
+                    Di = np.sum(P * dP, axis=1)
+                    dS = P * (dP - Di[:, None])
+                    dqt[b, r0:r1, h, :] = sc * (dS @ K[:kend])
+                    dkt[b, :kend, h, :] += sc * (dS.T @ Q[r0:r1])
+                    dv[b, :kend, h, :] += P.T @ dO
+
+    res = {"o": o, "lse": lse}
+    if want_bwd:
+        res["dq"] = rope_apply(dqt, theta, inverse=True, position_offset=position_offset)
+        res["dk"] = rope_apply(dkt, theta, inverse=True, position_offset=position_offset)
+        res["dv"] = dv
+    return res
+
+
+def attention_rows(q, k, v, d_o, samples, seg=None, causal=True, theta=1e4, scale=None):
+    """Exact O row, LSE and dq row for sampled query rows.
+
+    ``samples`` is a sequence of (b, h, i).  Each row needs only its own keys,
+    so this scales to any sequence length.  ``d_o`` may be None (no dq).
+    Returns dict of arrays: o [n, D], lse [n], dq [n, D] (when d_o given).
+    """
+    q = np.asarray(q)
+    B, S, H, D = q.shape
+    seg = _seg_or_default(seg, B, S)
+    sc = _scale(scale, D)
+    n = len(samples)
+    o = np.zeros((n, D))
+    lse = np.full(n, -np.inf)
+    dq = np.zeros((n, D)) if d_o is not None else None
+    use_rope = theta is not None and theta > 0
+    for r, (b, h, i) in enumerate(samples):
+        b, h, i = int(b), int(h), int(i)
+        kend = i + 1 if causal else S
+        keys = np.arange(kend)
+        qi = np.asarray(q[b, i, h, :], dtype=np.float64)
+        K = np.asarray(k[b, :kend, h, :], dtype=np.float64)
+        V = np.asarray(v[b, :kend, h, :], dtype=np.float64)
+        if use_rope:
+            qi = rope_apply(qi.reshape(1, 1, 1, D), theta, position_offset=i).reshape(D)
+            K = rope_apply(K.reshape(1, kend, 1, D), theta).reshape(kend, D)
+        s = sc * (K @ qi)
+        allowed = allowed_mask(seg[b], np.array([i]), keys, causal)
+        l, P = _softmax_rows(s[None, :], allowed)
+        lse[r] = l[0]
+        o[r] = P[0] @ V
+        if d_o is not None:
+            dOi = np.asarray(d_o[b, i, h, :], dtype=np.float64)
+            dP = V @ dOi
+            Di = np.sum(P[0] * dP)
+            dS = P[0] * (dP - Di)
+            dqt = sc * (dS @ K)
+            if use_rope:
+                dqt = rope_apply(dqt.reshape(1, 1, 1, D), theta, inverse=True,
+                                 position_offset=i).reshape(D)
+            dq[r] = dqt
+    res = {"o": o, "lse": lse}
+    if dq is not None:
+        res["dq"] = dq
+    return res
+
+
+def kept_pairs(seg, causal=True) -> int:
+    """Number of allowed (i, j) pairs summed over rows: sum over segments of
+    L(L+1)/2 when causal, L^2 otherwise (each id's tokens counted together)."""
+    seg = np.asarray(seg)
+    total = 0
+    for row in seg.reshape(-1, seg.shape[-1]):
+        ids, counts = np.unique(row[row >= 0], return_counts=True)
+        if causal:
+            # causal within a segment counts pairs j <= i that share the id
+            total += int(sum(c * (c + 1) // 2 for c in counts))
+        else:
+            total += int(sum(c * c for c in counts))
+    return total
+
+
+def attention_flops(seg, heads: int, head_dim: int, causal=True) -> dict:
+    """Algorithmic FLOPs: forward 4 D H Pi (two matmuls, 2 flops per MAC),
+    backward 2.5x forward (five matmuls), as stated for blockwise exact
+    attention with recomputation (FlashAttention entry of the reference list)."""
+    pi = kept_pairs(seg, causal)
+    fwd = 4.0 * head_dim * heads * pi
+    return {"pairs": pi, "fwd": fwd, "bwd": 2.5 * fwd, "fwd_bwd": 3.5 * fwd}
