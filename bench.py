@@ -1,0 +1,353 @@
+"""Benchmark: causal attention fwd+bwd TFLOP/s at 32 heads x 128, bf16, on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload long_128k]
+    python bench.py --impl reference ...     (the float64 CPU oracle, timed)
+
+One step = lwm_attn_fwd + lwm_attn_bwd over one batch of the workload (all of
+the hot path: segment prepass, RoPE, forward, dot(dO, O), backward).  The
+default workload is 128K tokens, one segment, theta 1e7, B1 H32 D128 bf16.
+Work is counted algorithmically: forward 4*D*H*Pi flops, backward 2.5x that,
+Pi = allowed (i, j) pairs (causal within segments; skipped tiles and masked
+elements are not counted).
+
+Under torchrun each rank runs an independent problem of the same size
+(different seed): weak scaling, no collective on the data path.  Timing is
+on the device (CUDA events) with a barrier and a synchronize on both sides;
+rank 0 prints one JSON line with the max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, segment_ids  # noqa: E402
+
+METRIC = "causal attn fwd+bwd TFLOP/s (32x128 heads, bf16) and % of B200 BF16 peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
+    total = 0
+    for row in seg:
+        _, counts = np.unique(row[row >= 0], return_counts=True)
+        c = counts.astype(np.int64)
+        total += int((c * (c + 1) // 2).sum()) if causal else int((c * c).sum())
+    return total
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def time_oracle_sample(w, seg, rows: int, seed: int):
+    """Oracle fwd+bwd on the last `rows` query rows of head 0 of batch row 0.
+
+    Returns (seconds, algorithmic flops of the sample, threads used)."""
+    import torch
+    import oracle
+    from workloads import make_tensors
+    small = w.with_(batch=1, heads=1)
+    t = make_tensors(small, seed=seed, device="cpu", with_grad_out=True)
+    f = lambda x: x.double().numpy()
+    r0 = w.seqlen - rows
+    t0 = time.perf_counter()
+    oracle.attention_backward(f(t["q"]), f(t["k"]), f(t["v"]), f(t["do"]), seg[:1],
+                              causal=w.causal, theta=w.theta, row_start=r0)
+    dt = time.perf_counter() - t0
+    row = seg[0]
+    pairs = 0
+    for i in range(r0, w.seqlen):
+        if row[i] >= 0:
+            keys = row[: i + 1] if w.causal else row
+            pairs += int(np.count_nonzero(keys == row[i]))
+    flops = 3.5 * 4.0 * w.head_dim * pairs
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    return dt, flops, threads
+
+
+def reference_arm(args):
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    seg = segment_ids(w, seed=args.seed)
+    rows = args.oracle_rows
+    for _ in range(args.warmup):
+        time_oracle_sample(w, seg, rows, args.seed)
+    times, flops, threads = [], 0.0, 1
+    for _ in range(args.steps):
+        dt, flops, threads = time_oracle_sample(w, seg, rows, args.seed)
+        times.append(dt)
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    sample = (f"float64 numpy oracle, fwd+bwd of the last {rows} query rows of one head "
+              f"(b=0, h=0) of {w.name}; {flops / 1e9:.2f} GFLOP algorithmic per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "heads": w.heads,
+                   "head_dim": w.head_dim, "theta": w.theta},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import long_context_causal_attention_b200 as lwm
+    from workloads import make_tensors
+
+    ws, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    w = WORKLOADS[args.workload]
+    seed = args.seed + rank
+    seg = segment_ids(w, seed=seed)
+    single = w.segments == "single"
+    seg_d = None if single else torch.as_tensor(seg, dtype=torch.int32, device=dev)
+    t = make_tensors(w, seed=seed, device=dev, with_grad_out=True)
+    q, k, v, do = t["q"], t["k"], t["v"], t["do"]
+    desc = lwm.make_desc(q, seg_d, w.causal, w.theta, w.scale)
+    ws_f = lwm.alloc_workspace(desc, False, dev)
+    ws_b = lwm.alloc_workspace(desc, True, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(w.batch, w.heads, w.seqlen, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lwm.lwm_attn_fwd(q, k, v, seg_d, w.causal, w.theta, w.scale, o=o, lse=lse,
+                         workspace=ws_f, stream=stream)
+        lwm.lwm_attn_bwd(q, k, v, o, lse, do, seg_d, w.causal, w.theta, w.scale, dq=dq, dk=dk,
+                         dv=dv, workspace=ws_b, stream=stream)
+
+    pairs = kept_pairs(seg, w.causal)
+    fwd_flops = 4.0 * w.head_dim * w.heads * pairs
+    step_flops = 3.5 * fwd_flops
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # per-step events around the main kernels (recorded by the library)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for evs in kev:
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    launches0 = lwm.lwm_attn_kernel_launches()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for s in range(args.steps):
+        lwm.lwm_attn_set_timing_events(*kev[s])
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    lwm.lwm_attn_set_timing_events()
+    launches = lwm.lwm_attn_kernel_launches() - launches0
+    clk = clocks.stop()
+    ms = start.elapsed_time(stop)
+    fwd_k = sum(e[0].elapsed_time(e[1]) for e in kev) / args.steps
+    bwd_k = sum(e[2].elapsed_time(e[3]) for e in kev) / args.steps
+    if ws > 1:
+        tt = torch.tensor([ms, fwd_k, bwd_k], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, fwd_k, bwd_k = tt.tolist()
+    ms_step = ms / args.steps
+    value = step_flops * ws / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs in, gradients out
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
+        hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3))
+        n_e2e = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            for hsrc, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
+                dst.copy_(hsrc, non_blocking=True)
+            step()
+            for src, hdst in ((dq, hdq), (dk, hdk), (dv, hdv)):
+                hdst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if ws > 1:
+            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = tt.item()
+        nb = q.numel() * q.element_size()
+        e2e = {"value": step_flops * ws / (ems / n_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 3 * nb, "steps": n_e2e}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    bwd_flops = 2.5 * fwd_flops
+    achieved = bwd_flops / (bwd_k * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "backward main kernel(s)",
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "fwd_kernel_tflops": fwd_flops / (fwd_k * 1e-3) / 1e12,
+                "fwd_kernel_ms": fwd_k, "bwd_kernel_ms": bwd_k}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, fl, threads = time_oracle_sample(w, seg, args.oracle_rows, seed)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"float64 numpy oracle, fwd+bwd of the last {args.oracle_rows} query rows "
+                         f"of one head of {w.name} ({fl / 1e9:.2f} GFLOP in {dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
+                       "heads": w.heads, "head_dim": w.head_dim, "theta": w.theta,
+                       "causal": w.causal, "segments": w.segments,
+                       "parallelism": f"independent problem per GPU x{ws}",
+                       "l2": "inputs larger than L2 (1 GiB per tensor vs 126 MB), no flush",
+                       "algorithmic_fwd_bwd_tflop_per_gpu": step_flops / 1e12,
+                       "tokens_per_s": w.batch * w.seqlen * ws / (ms_step * 1e-3),
+                       "pct_of_bf16_peak": 100.0 * value / ws / peak},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long_128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--oracle-rows", type=int, default=1024)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

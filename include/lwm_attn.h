@@ -1,0 +1,151 @@
+/*
+ * lwm_attn.h -- C ABI of liblwm_attn.so: exact blockwise causal self-attention
+ * with rotary position embedding (RoPE) and a masked-sequence-packing mask,
+ * forward and backward, for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are the pages describing Large World
+ * Model, "LWM"):
+ *
+ *   - LWM research note (zhao9797.github.io), section "模型架构" (model
+ *     architecture): exact blockwise attention (RingAttention + Blockwise
+ *     Parallel Transformer fused with FlashAttention) and "standard RoPE"
+ *     whose theta grows with the context window.
+ *   - Same note, section "训练方法" (training method): the theta schedule
+ *     (32K: 1e6, 128K: 1e7, 256K: 1e7, 512K: 2.5e7, 1M: 5e7) and Masked
+ *     Sequence Packing: samples packed into one sequence attend only to
+ *     themselves, numerically the same as unpacked training with padding.
+ *   - Paper card "World Model on Million-Length Video And Language With
+ *     Blockwise RingAttention" (research.elamur.ai), Summary: the attention is
+ *     computed "without approximation"; its reference list names RoFormer
+ *     (the rotary form) and FlashAttention (blockwise exact softmax).
+ *
+ * Definitions (row i, key j of one (batch, head); D = head_dim):
+ *   w_t      = theta^(-2t/D),  t = 0 .. D/2-1
+ *   R(p)     = rotation of each interleaved pair (x[2t], x[2t+1]) by p*w_t,
+ *              p = index of the token in its row (positions continue across
+ *              packed segments; outputs do not depend on that choice)
+ *   s_ij     = scale * <R(i) q_i, R(j) k_j>
+ *   allowed  = seg_i == seg_j  &&  seg_i >= 0  &&  (!causal || j <= i)
+ *   LSE_i    = ln sum_{allowed j} exp(s_ij)         (-inf if nothing allowed)
+ *   O_i      = sum_{allowed j} exp(s_ij - LSE_i) v_j  (0 if nothing allowed)
+ *   dq, dk, dv = gradients of sum(O * dO) with respect to the UN-rotated q, k
+ *              and v.
+ *
+ * Layout (all tensors): Q, K, V, O, dO, dQ, dK, dV are [B, S, H, D]
+ * contiguous, D fastest (token stride H*D).  LSE is [B, H, S] fp32.
+ * Segment ids are [B, S] int32 on the device.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates no device
+ * memory in any call; it caches only device properties under a mutex.
+ *
+ * Calling convention: every compute call is asynchronous on `stream` (a
+ * cudaStream_t passed as void*; NULL = legacy default stream).  Argument,
+ * alignment and workspace errors are returned synchronously before anything
+ * is launched.  A bounded device-side wait that runs out writes
+ * LWM_ERR_TIMEOUT into the workspace status word; read it with
+ * lwm_attn_read_status after the stream's work.  Launch failures are
+ * returned as LWM_ERR_CUDA.
+ *
+ * Thread safety: calls may come from several host threads; calls that share
+ * a workspace must not overlap on the device.
+ */
+#ifndef LWM_ATTN_H
+#define LWM_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LWM_OK = 0,
+  LWM_ERR_INVALID_ARG = -1,  /* null pointer, bad size, bad enum value */
+  LWM_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. head_dim 96) */
+  LWM_ERR_ALIGNMENT = -3,    /* a tensor pointer is not 16-byte aligned */
+  LWM_ERR_WORKSPACE = -4,    /* workspace null or smaller than required */
+  LWM_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed */
+  LWM_ERR_TIMEOUT = -6       /* a bounded device wait ran out (status word) */
+} lwm_status;
+
+typedef enum { LWM_DTYPE_BF16 = 0, LWM_DTYPE_FP32 = 1 } lwm_dtype;
+
+/* Problem description shared by forward and backward. */
+typedef struct {
+  int64_t batch;              /* B >= 1 */
+  int64_t seqlen;             /* S >= 1 (no upper limit beyond memory; 64-bit offsets) */
+  int64_t heads;              /* H >= 1 */
+  int64_t head_dim;           /* D in {64, 128} */
+  int32_t dtype;              /* lwm_dtype of Q, K, V, O, dO, dQ, dK, dV */
+  int32_t causal;             /* 1: j <= i within a segment; 0: whole segment */
+  double rope_theta;          /* RoPE base; <= 0 disables the rotation */
+  float softmax_scale;        /* <= 0 selects 1/sqrt(head_dim) */
+  const int32_t* segment_ids; /* device [B, S]; NULL = one segment per row;
+                                 id < 0 marks padding (O = 0, LSE = -inf,
+                                 gradients 0).  Any ids are correct; ids that
+                                 form contiguous runs (what packing produces)
+                                 let whole tiles be skipped. */
+} lwm_attn_desc;
+
+/* Bytes of device workspace lwm_attn_fwd (is_bwd = 0) or lwm_attn_bwd
+ * (is_bwd != 0) needs for `desc`; 0 if `desc` is invalid.  The workspace
+ * holds the status word, per-tile segment bounds, the rotated Q and K and,
+ * for the backward, the fp32 dQ accumulator and the per-row dot(dO, O).
+ * The forward's need is never larger than the backward's. */
+size_t lwm_attn_workspace_size(const lwm_attn_desc* desc, int is_bwd);
+
+/* Forward pass (research note, "模型架构": exact blockwise attention with RoPE;
+ * "训练方法": packing mask).  q, k, v: device [B,S,H,D] of desc->dtype,
+ * un-rotated.  o: device [B,S,H,D] output.  lse: device [B,H,S] fp32 output
+ * (natural log of the scaled scores).  ws: device workspace of at least
+ * lwm_attn_workspace_size(desc, 0) bytes, 256-byte aligned.  All tensor
+ * pointers must be 16-byte aligned.  o and lse may not alias the inputs. */
+lwm_status lwm_attn_fwd(const lwm_attn_desc* desc, const void* q, const void* k,
+                        const void* v, void* o, float* lse, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* Backward pass: gradients of sum(O * dO) with respect to the un-rotated q,
+ * k and v (the gradients training needs, research note "训练方法"; P is
+ * recomputed from the saved LSE as in the FlashAttention reference of the
+ * paper card).  o and lse must be the outputs of lwm_attn_fwd for the same
+ * inputs; d_o is [B,S,H,D] of desc->dtype.  dq, dk, dv are written (not
+ * accumulated).  ws: at least lwm_attn_workspace_size(desc, 1) bytes. */
+lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
+                        const void* v, const void* o, const float* lse,
+                        const void* d_o, void* dq, void* dk, void* dv, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* y = R(p) x (inverse = 0) or R(p)^T x (inverse != 0) for x of [B,S,H,D]
+ * (research note, "模型架构": standard RoPE; theta per "训练方法").  Angles
+ * p*w_t are formed and reduced modulo 2*pi in fp64, cos/sin taken in fp32,
+ * the pair rotated in fp32 and rounded to dtype (nearest even).  y may equal
+ * x (in place); otherwise they must not overlap.  theta <= 0 copies. */
+lwm_status lwm_rope_apply(int64_t batch, int64_t seqlen, int64_t heads,
+                          int64_t head_dim, int32_t dtype, double theta,
+                          const void* x, void* y, int inverse, void* stream);
+
+/* Waits for `stream`, then returns the status word the kernels of the last
+ * call on `ws` left (LWM_OK or LWM_ERR_TIMEOUT), or LWM_ERR_CUDA. */
+lwm_status lwm_attn_read_status(const void* ws, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* lwm_status_string(lwm_status status);
+
+/* Instrumentation (no counterpart on the pages; used by the benchmark).
+ * lwm_attn_set_timing_events: cudaEvent_t handles (as void*, any may be
+ * NULL) that the next calls record on their stream immediately before and
+ * after the main attention kernel(s) of lwm_attn_fwd / lwm_attn_bwd, so the
+ * caller can time those kernels alone.  The handles stay in effect until
+ * replaced; pass NULLs to stop.  Process-wide; guarded by a mutex.
+ * lwm_attn_kernel_launches: number of kernels this library has launched
+ * since it was loaded. */
+void lwm_attn_set_timing_events(void* fwd_start, void* fwd_stop, void* bwd_start,
+                                void* bwd_stop);
+uint64_t lwm_attn_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LWM_ATTN_H */

@@ -1,0 +1,225 @@
+"""ctypes binding of liblwm_attn.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it checks that tensors are CUDA tensors of the right
+shape, allocates outputs and workspace with torch (device memory is torch's
+job), passes raw pointers and the current stream, and turns a non-zero
+status into an exception.  If the shared library is missing the import fails
+loudly; there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblwm_attn.so")
+
+LWM_OK = 0
+LWM_DTYPE_BF16 = 0
+LWM_DTYPE_FP32 = 1
+
+STATUS_NAMES = {
+    0: "LWM_OK", -1: "LWM_ERR_INVALID_ARG", -2: "LWM_ERR_UNSUPPORTED", -3: "LWM_ERR_ALIGNMENT",
+    -4: "LWM_ERR_WORKSPACE", -5: "LWM_ERR_CUDA", -6: "LWM_ERR_TIMEOUT",
+}
+
+ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_rope_apply",
+                "lwm_attn_read_status", "lwm_status_string", "lwm_attn_set_timing_events",
+                "lwm_attn_kernel_launches")
+
+
+class LwmAttnDesc(ctypes.Structure):
+    """Mirror of lwm_attn_desc in include/lwm_attn.h."""
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("heads", ctypes.c_int64),
+        ("head_dim", ctypes.c_int64),
+        ("dtype", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("rope_theta", ctypes.c_double),
+        ("softmax_scale", ctypes.c_float),
+        ("segment_ids", ctypes.c_void_p),
+    ]
+
+
+class LwmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({lwm_status_string(status)})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m long_context_causal_attention_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    lib.lwm_attn_workspace_size.argtypes = [ctypes.POINTER(LwmAttnDesc), ctypes.c_int]
+    lib.lwm_attn_workspace_size.restype = ctypes.c_size_t
+    lib.lwm_attn_fwd.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.lwm_attn_fwd.restype = ctypes.c_int
+    lib.lwm_attn_bwd.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P, P, P, P, P,
+                                 ctypes.c_size_t, P]
+    lib.lwm_attn_bwd.restype = ctypes.c_int
+    lib.lwm_rope_apply.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.c_int32, ctypes.c_double, P, P, ctypes.c_int, P]
+    lib.lwm_rope_apply.restype = ctypes.c_int
+    lib.lwm_attn_read_status.argtypes = [P, P]
+    lib.lwm_attn_read_status.restype = ctypes.c_int
+    lib.lwm_status_string.argtypes = [ctypes.c_int]
+    lib.lwm_status_string.restype = ctypes.c_char_p
+    lib.lwm_attn_set_timing_events.argtypes = [P, P, P, P]
+    lib.lwm_attn_set_timing_events.restype = None
+    lib.lwm_attn_kernel_launches.argtypes = []
+    lib.lwm_attn_kernel_launches.restype = ctypes.c_uint64
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def lwm_status_string(status: int) -> str:
+    return _lib.lwm_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LWM_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return LWM_DTYPE_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def make_desc(q: torch.Tensor, segment_ids=None, causal=True, rope_theta=1e4,
+              softmax_scale=0.0) -> LwmAttnDesc:
+    if q.dim() != 4:
+        raise ValueError("q must be [B, S, H, D]")
+    B, S, H, D = q.shape
+    seg_ptr = None
+    if segment_ids is not None:
+        _cuda(segment_ids, "segment_ids")
+        if segment_ids.dtype != torch.int32 or tuple(segment_ids.shape) != (B, S):
+            raise ValueError("segment_ids must be int32 [B, S]")
+        seg_ptr = segment_ids.data_ptr()
+    return LwmAttnDesc(B, S, H, D, _dtype_code(q), 1 if causal else 0, float(rope_theta),
+                       float(softmax_scale), seg_ptr)
+
+
+def lwm_attn_workspace_size(desc: LwmAttnDesc, is_bwd: bool) -> int:
+    return int(_lib.lwm_attn_workspace_size(ctypes.byref(desc), 1 if is_bwd else 0))
+
+
+def alloc_workspace(desc: LwmAttnDesc, is_bwd: bool, device) -> torch.Tensor:
+    n = lwm_attn_workspace_size(desc, is_bwd)
+    if n == 0:
+        raise LwmError(-1, "lwm_attn_workspace_size")
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _check(status: int, what: str):
+    if status != LWM_OK:
+        raise LwmError(status, what)
+
+
+def lwm_attn_fwd(q, k, v, segment_ids=None, causal=True, rope_theta=1e4, softmax_scale=0.0,
+                 o=None, lse=None, workspace=None, stream=None):
+    """O [B,S,H,D] and LSE [B,H,S] fp32 for un-rotated q, k, v (see lwm_attn.h)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, name)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    desc = make_desc(q, segment_ids, causal, rope_theta, softmax_scale)
+    B, S, H, D = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(desc, False, q.device)
+    st = _lib.lwm_attn_fwd(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                           o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                           workspace.numel(), _stream(stream))
+    _check(st, "lwm_attn_fwd")
+    return o, lse
+
+
+def lwm_attn_bwd(q, k, v, o, lse, d_o, segment_ids=None, causal=True, rope_theta=1e4,
+                 softmax_scale=0.0, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dq, dk, dv (gradients w.r.t. the un-rotated inputs) of sum(O * dO)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("d_o", d_o)):
+        _cuda(t, name)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    _cuda(lse, "lse")
+    desc = make_desc(q, segment_ids, causal, rope_theta, softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = alloc_workspace(desc, True, q.device)
+    st = _lib.lwm_attn_bwd(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                           o.data_ptr(), lse.data_ptr(), d_o.data_ptr(), dq.data_ptr(),
+                           dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                           _stream(stream))
+    _check(st, "lwm_attn_bwd")
+    return dq, dk, dv
+
+
+def lwm_rope_apply(x, theta, inverse=False, out=None, stream=None):
+    """y = R(p) x (or R(p)^T x) for x [B,S,H,D]; out may be x (in place)."""
+    _cuda(x, "x")
+    if x.dim() != 4:
+        raise ValueError("x must be [B, S, H, D]")
+    out = torch.empty_like(x) if out is None else out
+    B, S, H, D = x.shape
+    st = _lib.lwm_rope_apply(B, S, H, D, _dtype_code(x), float(theta), x.data_ptr(),
+                             out.data_ptr(), 1 if inverse else 0, _stream(stream))
+    _check(st, "lwm_rope_apply")
+    return out
+
+
+def lwm_attn_read_status(workspace, stream=None) -> int:
+    return int(_lib.lwm_attn_read_status(workspace.data_ptr(), _stream(stream)))
+
+
+def lwm_attn_set_timing_events(fwd_start=None, fwd_stop=None, bwd_start=None, bwd_stop=None):
+    """Have the next calls record these torch.cuda.Event objects around their
+    main attention kernels (None leaves that slot empty)."""
+    def handle(e):
+        if e is None:
+            return None
+        if not e.cuda_event:  # torch creates the CUDA event on first record
+            e.record()
+        return ctypes.c_void_p(e.cuda_event)
+    _lib.lwm_attn_set_timing_events(handle(fwd_start), handle(fwd_stop), handle(bwd_start),
+                                    handle(bwd_stop))
+
+
+def lwm_attn_kernel_launches() -> int:
+    return int(_lib.lwm_attn_kernel_launches())

@@ -1,0 +1,232 @@
+// C ABI of liblwm_attn: argument checks, workspace layout and dispatch.
+// The operations are defined in include/lwm_attn.h.
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace lwm {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_events_mu;
+cudaEvent_t g_events[4] = {nullptr, nullptr, nullptr, nullptr};
+
+void record_event(int which, cudaStream_t st) {
+  std::lock_guard<std::mutex> lk(g_events_mu);
+  if (g_events[which]) cudaEventRecord(g_events[which], st);
+}
+}  // namespace
+
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+Path choose_path(const Problem& p) {
+  static const bool force_simt = [] {
+    const char* e = std::getenv("LWM_ATTN_FORCE_SIMT");
+    return e && e[0] == '1';
+  }();
+  if (force_simt) return Path::kSimt;
+  return Path::kSimt;
+}
+
+size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
+  char* b = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    off = align_up(off, 1024);
+    void* r = b ? b + off : nullptr;
+    off += bytes;
+    return r;
+  };
+  Workspace w{};
+  w.status = static_cast<DeviceStatus*>(take(sizeof(DeviceStatus)));
+  const size_t tiles = (size_t)p.B * (size_t)p.n_tiles * sizeof(int32_t);
+  w.tile_min = static_cast<int32_t*>(take(tiles));
+  w.tile_max = static_cast<int32_t*>(take(tiles));
+  w.q_lo = static_cast<int32_t*>(take(tiles));
+  w.k_hi = static_cast<int32_t*>(take(tiles));
+  const size_t nel = (size_t)p.B * p.S * p.H * p.D;
+  if (p.theta > 0.0) {
+    w.q_rot = take(nel * p.elt);
+    w.k_rot = take(nel * p.elt);
+  }
+  if (bwd) {
+    w.delta = static_cast<float*>(take((size_t)p.B * p.H * p.S * sizeof(float)));
+    if (choose_path(p) == Path::kSm100) w.dq_acc = static_cast<float*>(take(nel * sizeof(float)));
+  }
+  w.bytes = align_up(off, 1024);
+  if (ws) *ws = w;
+  return w.bytes;
+}
+
+namespace {
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+lwm_status make_problem(const lwm_attn_desc* d, Problem* p) {
+  if (!d) return LWM_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->seqlen < 0 || d->heads < 1 || d->head_dim < 1) return LWM_ERR_INVALID_ARG;
+  if (d->dtype != LWM_DTYPE_BF16 && d->dtype != LWM_DTYPE_FP32) return LWM_ERR_INVALID_ARG;
+  if (d->causal != 0 && d->causal != 1) return LWM_ERR_INVALID_ARG;
+  if (!std::isfinite(d->rope_theta) || !std::isfinite(d->softmax_scale)) return LWM_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return LWM_ERR_UNSUPPORTED;
+  if (d->heads > 65535 || d->batch > 65535) return LWM_ERR_UNSUPPORTED;
+  if (d->seqlen > ((int64_t)1 << 33)) return LWM_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(d->segment_ids) & 3u) return LWM_ERR_ALIGNMENT;
+  p->B = d->batch;
+  p->S = d->seqlen;
+  p->H = d->heads;
+  p->D = d->head_dim;
+  p->dtype = d->dtype;
+  p->causal = d->causal;
+  p->theta = d->rope_theta;
+  p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / std::sqrt((double)d->head_dim));
+  p->seg = d->segment_ids;
+  p->n_tiles = (d->seqlen + kTile - 1) / kTile;
+  p->elt = d->dtype == LWM_DTYPE_BF16 ? 2 : 4;
+  return LWM_OK;
+}
+
+lwm_status check_ws(const Problem& p, bool bwd, void* ws, size_t ws_bytes, Workspace* w) {
+  const size_t need = layout_workspace(p, bwd, nullptr, nullptr);
+  if (!ws || ws_bytes < need) return LWM_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return LWM_ERR_ALIGNMENT;
+  layout_workspace(p, bwd, ws, w);
+  return LWM_OK;
+}
+
+lwm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LWM_OK : LWM_ERR_CUDA; }
+
+// Shared front half of forward and backward: status word, segment bounds,
+// rotated q and k.
+cudaError_t prologue(const Problem& p, Workspace& w, const void* q, const void* k, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
+  if (e != cudaSuccess) return e;
+  e = launch_segment_bounds(p, w, st);
+  if (e != cudaSuccess) return e;
+  if (p.theta > 0.0) {
+    e = launch_rope(p.B, p.S, p.H, p.D, p.dtype, p.theta, q, w.q_rot, 0, st);
+    if (e != cudaSuccess) return e;
+    e = launch_rope(p.B, p.S, p.H, p.D, p.dtype, p.theta, k, w.k_rot, 0, st);
+  } else {
+    w.q_rot = const_cast<void*>(q);
+    w.k_rot = const_cast<void*>(k);
+  }
+  return e;
+}
+
+}  // namespace
+}  // namespace lwm
+
+using namespace lwm;
+
+extern "C" {
+
+size_t lwm_attn_workspace_size(const lwm_attn_desc* desc, int is_bwd) {
+  Problem p{};
+  if (make_problem(desc, &p) != LWM_OK) return 0;
+  return layout_workspace(p, is_bwd != 0, nullptr, nullptr);
+}
+
+lwm_status lwm_attn_fwd(const lwm_attn_desc* desc, const void* q, const void* k, const void* v,
+                        void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Problem p{};
+  lwm_status s = make_problem(desc, &p);
+  if (s != LWM_OK) return s;
+  if (p.B * p.S == 0) return LWM_OK;
+  if (!q || !k || !v || !o || !lse) return LWM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return LWM_ERR_ALIGNMENT;
+  Workspace w{};
+  s = check_ws(p, false, ws, ws_bytes, &w);
+  if (s != LWM_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = prologue(p, w, q, k, st);
+  if (e != cudaSuccess) return LWM_ERR_CUDA;
+  record_event(0, st);
+  e = launch_simt_fwd(p, w, v, o, lse, st);
+  record_event(1, st);
+  return cuda_status(e);
+}
+
+lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* d_o, void* dq, void* dk,
+                        void* dv, void* ws, size_t ws_bytes, void* stream) {
+  Problem p{};
+  lwm_status s = make_problem(desc, &p);
+  if (s != LWM_OK) return s;
+  if (p.B * p.S == 0) return LWM_OK;
+  if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv) return LWM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(d_o) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return LWM_ERR_ALIGNMENT;
+  Workspace w{};
+  s = check_ws(p, true, ws, ws_bytes, &w);
+  if (s != LWM_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = prologue(p, w, q, k, st);
+  if (e != cudaSuccess) return LWM_ERR_CUDA;
+  e = launch_delta(p, o, d_o, w.delta, st);
+  if (e != cudaSuccess) return LWM_ERR_CUDA;
+  record_event(2, st);
+  e = launch_simt_bwd(p, w, v, lse, d_o, dq, dk, dv, st);
+  record_event(3, st);
+  return cuda_status(e);
+}
+
+lwm_status lwm_rope_apply(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
+                          int32_t dtype, double theta, const void* x, void* y, int inverse,
+                          void* stream) {
+  if (batch < 0 || seqlen < 0 || heads < 1 || head_dim < 2 || (head_dim & 1)) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32) return LWM_ERR_INVALID_ARG;
+  if (!std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  const int vec = dtype == LWM_DTYPE_BF16 ? 8 : 4;
+  if (head_dim % vec != 0 || head_dim > 512) return LWM_ERR_UNSUPPORTED;
+  if (batch * seqlen == 0) return LWM_OK;
+  if (!x || !y) return LWM_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return LWM_ERR_ALIGNMENT;
+  return cuda_status(launch_rope(batch, seqlen, heads, head_dim, dtype, theta, x, y, inverse,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+lwm_status lwm_attn_read_status(const void* ws, void* stream) {
+  if (!ws) return LWM_ERR_INVALID_ARG;
+  int32_t code = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return LWM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LWM_ERR_CUDA;
+  return code == 0 ? LWM_OK : static_cast<lwm_status>(code);
+}
+
+const char* lwm_status_string(lwm_status status) {
+  switch (status) {
+    case LWM_OK: return "LWM_OK";
+    case LWM_ERR_INVALID_ARG: return "LWM_ERR_INVALID_ARG: invalid argument";
+    case LWM_ERR_UNSUPPORTED: return "LWM_ERR_UNSUPPORTED: unsupported configuration";
+    case LWM_ERR_ALIGNMENT: return "LWM_ERR_ALIGNMENT: pointer not 16-byte aligned (workspace: 256)";
+    case LWM_ERR_WORKSPACE: return "LWM_ERR_WORKSPACE: workspace missing or too small";
+    case LWM_ERR_CUDA: return "LWM_ERR_CUDA: CUDA runtime error";
+    case LWM_ERR_TIMEOUT: return "LWM_ERR_TIMEOUT: a bounded device wait ran out";
+  }
+  return "unknown lwm_status";
+}
+
+void lwm_attn_set_timing_events(void* fwd_start, void* fwd_stop, void* bwd_start,
+                                void* bwd_stop) {
+  std::lock_guard<std::mutex> lk(g_events_mu);
+  g_events[0] = static_cast<cudaEvent_t>(fwd_start);
+  g_events[1] = static_cast<cudaEvent_t>(fwd_stop);
+  g_events[2] = static_cast<cudaEvent_t>(bwd_start);
+  g_events[3] = static_cast<cudaEvent_t>(bwd_stop);
+}
+
+uint64_t lwm_attn_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

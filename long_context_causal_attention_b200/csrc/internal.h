@@ -1,0 +1,61 @@
+// Host-side internals shared by the translation units of liblwm_attn.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lwm_attn.h"
+
+namespace lwm {
+
+struct DeviceStatus;
+
+// Validated problem, in the form the launchers take.
+struct Problem {
+  int64_t B, S, H, D;
+  int dtype;          // lwm_dtype
+  int causal;
+  double theta;       // <= 0: no rotation
+  float scale;        // resolved softmax scale (> 0)
+  const int32_t* seg; // may be null
+  int64_t n_tiles;    // ceil(S / 128)
+  size_t elt;         // bytes per element of dtype
+};
+
+// Carved-up workspace.  Every region is 1024-byte aligned.
+struct Workspace {
+  DeviceStatus* status;
+  int32_t* tile_min;   // [B, n_tiles] smallest non-negative id in the tile (INT32_MAX if none)
+  int32_t* tile_max;   // [B, n_tiles] largest id in the tile (-1 if none)
+  int32_t* q_lo;       // [B, n_tiles] first key tile a query tile may need
+  int32_t* k_hi;       // [B, n_tiles] last query tile a key tile may feed
+  void* q_rot;         // [B, S, H, D] rotated q (dtype)
+  void* k_rot;         // [B, S, H, D] rotated k (dtype)
+  float* dq_acc;       // [B, S, H, D] fp32 (backward, tensor-core path)
+  float* delta;        // [B, H, S] fp32 dot(dO, O) per row (backward)
+  size_t bytes;        // total bytes the layout needs
+};
+
+enum class Path { kSimt = 0, kSm100 = 1 };
+
+Path choose_path(const Problem& p);
+
+// Instrumentation: kernels launched so far (process-wide).
+void note_launches(int n);
+size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws);
+
+// Launchers (return the first CUDA error, or cudaSuccess).
+cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, double theta,
+                        const void* x, void* y, int inverse, cudaStream_t st);
+cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st);
+cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float* delta,
+                         cudaStream_t st);
+
+cudaError_t launch_simt_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
+                            float* lse, cudaStream_t st);
+cudaError_t launch_simt_bwd(const Problem& p, const Workspace& ws, const void* v,
+                            const float* lse, const void* d_o, void* dq, void* dk, void* dv,
+                            cudaStream_t st);
+
+}  // namespace lwm

@@ -1,0 +1,133 @@
+// RoPE application (HBM-bound elementwise kernel) and the per-row dot(dO, O).
+//
+// Rotation as the LWM research note describes it ("模型架构": standard RoPE,
+// theta scaled with the context per "训练方法"): pair (x[2t], x[2t+1]) of the
+// token at position p turns by p * theta^(-2t/D).
+#include "common.cuh"
+#include "internal.h"
+
+namespace lwm {
+namespace {
+
+// 16-byte vectors: 8 bf16 or 4 fp32 elements (4 or 2 rotary pairs).
+template <typename T> struct Vec;
+template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };
+template <> struct Vec<float> { static constexpr int N = 4; };
+
+// One CTA walks tokens with a grid stride.  Thread layout inside a token:
+// lane c = tid % (D / N) picks the pair group (fixed for the thread, so its
+// frequencies are computed once), hg = tid / (D / N) the head it starts at.
+template <typename T>
+__global__ void __launch_bounds__(128) rope_kernel(const T* __restrict__ x, T* __restrict__ y,
+                                                   int64_t n_tok, int64_t S, int H, int D,
+                                                   double log2_theta, int inverse) {
+  constexpr int N = Vec<T>::N;
+  constexpr int P = N / 2;
+  const int per_head = D / N;
+  const int c = threadIdx.x % per_head;
+  const int hg = threadIdx.x / per_head;
+  const int heads_per_pass = blockDim.x / per_head;
+  if (hg >= heads_per_pass) return;
+  double w[P];
+#pragma unroll
+  for (int u = 0; u < P; ++u) w[u] = rope_freq(c * P + u, D, log2_theta);
+  const float sgn = inverse ? -1.0f : 1.0f;
+  for (int64_t tok = blockIdx.x; tok < n_tok; tok += gridDim.x) {
+    const int64_t pos = tok % S;
+    float cs[P], sn[P];
+#pragma unroll
+    for (int u = 0; u < P; ++u) {
+      rope_cos_sin_w(pos, w[u], &cs[u], &sn[u]);
+      sn[u] *= sgn;
+    }
+    const size_t base = (size_t)tok * H * D;
+    for (int h = hg; h < H; h += heads_per_pass) {
+      const size_t off = base + (size_t)h * D + (size_t)c * N;
+      uint4 raw = *reinterpret_cast<const uint4*>(x + off);
+      T* e = reinterpret_cast<T*>(&raw);
+      uint4 outv;
+      T* f = reinterpret_cast<T*>(&outv);
+#pragma unroll
+      for (int u = 0; u < P; ++u) {
+        const float a = to_f32(e[2 * u]), b = to_f32(e[2 * u + 1]);
+        f[2 * u] = from_f32<T>(a * cs[u] - b * sn[u]);
+        f[2 * u + 1] = from_f32<T>(a * sn[u] + b * cs[u]);
+      }
+      *reinterpret_cast<uint4*>(y + off) = outv;
+    }
+  }
+}
+
+// delta[b, h, i] = sum_d dO[b, i, h, d] * O[b, i, h, d]; one warp per (token, head).
+template <typename T>
+__global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, const T* __restrict__ d_o,
+                                                    float* __restrict__ delta, int64_t n_rows,
+                                                    int64_t S, int H, int D) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= n_rows) return;  // row = (b * S + i) * H + h
+  const T* a = o + (size_t)row * D;
+  const T* g = d_o + (size_t)row * D;
+  float acc = 0.f;
+  for (int d = lane; d < D; d += 32) acc += to_f32(a[d]) * to_f32(g[d]);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) {
+    const int64_t h = row % H, tok = row / H;
+    const int64_t b = tok / S, i = tok % S;
+    delta[((size_t)b * H + h) * S + i] = acc;
+  }
+}
+
+int grid_for(int64_t n) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t g = (int64_t)sms * 16;
+  return (int)(n < g ? (n > 0 ? n : 1) : g);
+}
+
+}  // namespace
+
+cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, double theta,
+                        const void* x, void* y, int inverse, cudaStream_t st) {
+  const int64_t n_tok = B * S;
+  if (n_tok == 0) return cudaSuccess;
+  const size_t bytes = (size_t)n_tok * H * D * (dtype == LWM_DTYPE_BF16 ? 2 : 4);
+  if (!(theta > 0.0)) {
+    if (x == y) return cudaSuccess;
+    return cudaMemcpyAsync(y, x, bytes, cudaMemcpyDeviceToDevice, st);
+  }
+  const double l2t = log2(theta);
+  const int grid = grid_for(n_tok);
+  if (dtype == LWM_DTYPE_BF16) {
+    rope_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), n_tok, S, (int)H,
+        (int)D, l2t, inverse);
+  } else {
+    rope_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(x), static_cast<float*>(y),
+                                             n_tok, S, (int)H, (int)D, l2t, inverse);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float* delta,
+                         cudaStream_t st) {
+  const int64_t rows = p.B * p.S * p.H;
+  if (rows == 0) return cudaSuccess;
+  const int64_t grid = (rows + 7) / 8;
+  if (p.dtype == LWM_DTYPE_BF16) {
+    delta_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), delta, rows,
+        p.S, (int)p.H, (int)p.D);
+  } else {
+    delta_kernel<float><<<(unsigned)grid, 256, 0, st>>>(static_cast<const float*>(o),
+                                                       static_cast<const float*>(d_o), delta, rows,
+                                                       p.S, (int)p.H, (int)p.D);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace lwm

@@ -215,31 +215,38 @@ def attention_rows(q, k, v, d_o, samples, seg=None, causal=True, theta=1e4, scal
     lse = np.full(n, -np.inf)
     dq = np.zeros((n, D)) if d_o is not None else None
     use_rope = theta is not None and theta > 0
+    # group the samples by (b, h) so each head's keys are rotated once
+    groups = {}
     for r, (b, h, i) in enumerate(samples):
-        b, h, i = int(b), int(h), int(i)
-        kend = i + 1 if causal else S
-        keys = np.arange(kend)
-        qi = np.asarray(q[b, i, h, :], dtype=np.float64)
-        K = np.asarray(k[b, :kend, h, :], dtype=np.float64)
-        V = np.asarray(v[b, :kend, h, :], dtype=np.float64)
+        groups.setdefault((int(b), int(h)), []).append((r, int(i)))
+    for (b, h), items in groups.items():
+        kmax = max(i for _, i in items) + 1 if causal else S
+        Kall = np.asarray(k[b, :kmax, h, :], dtype=np.float64)
         if use_rope:
-            qi = rope_apply(qi.reshape(1, 1, 1, D), theta, position_offset=i).reshape(D)
-            K = rope_apply(K.reshape(1, kend, 1, D), theta).reshape(kend, D)
-        s = sc * (K @ qi)
-        allowed = allowed_mask(seg[b], np.array([i]), keys, causal)
-        l, P = _softmax_rows(s[None, :], allowed)
-        lse[r] = l[0]
-        o[r] = P[0] @ V
-        if d_o is not None:
-            dOi = np.asarray(d_o[b, i, h, :], dtype=np.float64)
-            dP = V @ dOi
-            Di = np.sum(P[0] * dP)
-            dS = P[0] * (dP - Di)
-            dqt = sc * (dS @ K)
+            Kall = rope_apply(Kall.reshape(1, kmax, 1, D), theta).reshape(kmax, D)
+        Vall = np.asarray(v[b, :kmax, h, :], dtype=np.float64)
+        for r, i in items:
+            kend = i + 1 if causal else S
+            keys = np.arange(kend)
+            K, V = Kall[:kend], Vall[:kend]
+            qi = np.asarray(q[b, i, h, :], dtype=np.float64)
             if use_rope:
-                dqt = rope_apply(dqt.reshape(1, 1, 1, D), theta, inverse=True,
-                                 position_offset=i).reshape(D)
-            dq[r] = dqt
+                qi = rope_apply(qi.reshape(1, 1, 1, D), theta, position_offset=i).reshape(D)
+            s = sc * (K @ qi)
+            allowed = allowed_mask(seg[b], np.array([i]), keys, causal)
+            l, P = _softmax_rows(s[None, :], allowed)
+            lse[r] = l[0]
+            o[r] = P[0] @ V
+            if d_o is not None:
+                dOi = np.asarray(d_o[b, i, h, :], dtype=np.float64)
+                dP = V @ dOi
+                Di = np.sum(P[0] * dP)
+                dS = P[0] * (dP - Di)
+                dqt = sc * (dS @ K)
+                if use_rope:
+                    dqt = rope_apply(dqt.reshape(1, 1, 1, D), theta, inverse=True,
+                                     position_offset=i).reshape(D)
+                dq[r] = dqt
     res = {"o": o, "lse": lse}
     if dq is not None:
         res["dq"] = dq

@@ -1,0 +1,43 @@
+"""Helpers for GPU-vs-oracle parity tests.
+
+Tolerances (max-abs and mean-abs over the compared elements):
+  bf16 tensors (O, dQ, dK, dV): max-abs <= 2e-2, mean-abs <= 2e-3
+  fp32 tensors:                 max-abs <= 1e-4
+  LSE (fp32 output in both cases, but computed from bf16 operands when the
+  inputs are bf16): bf16 inputs 2e-2 / 2e-3, fp32 inputs 1e-4.
+The bf16 bound is the one stated for this method's parity; the LSE bound
+follows from it: rotated q and k are rounded to bf16 (relative 2^-9), which
+moves a score of size |s| by about |s| 2^-8, well under 2e-2 for the score
+scales of these workloads.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+TOL = {"bf16": (2e-2, 2e-3), "fp32": (1e-4, 1e-4)}
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def err_stats(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    fin = np.isfinite(want)
+    if not np.array_equal(np.isfinite(got), fin):
+        return {"max_abs": float("inf"), "mean_abs": float("inf"), "nonfinite_mismatch": True}
+    if not fin.any():
+        return {"max_abs": 0.0, "mean_abs": 0.0}
+    d = np.abs(got[fin] - want[fin])
+    return {"max_abs": float(d.max()), "mean_abs": float(d.mean())}
+
+
+def assert_close(name, got, want, dtype: str, report=None):
+    mx, mean = TOL[dtype]
+    st = err_stats(got, want)
+    if report is not None:
+        report[name] = st
+    assert st["max_abs"] <= mx and st["mean_abs"] <= mean, f"{name}: {st} (tol {mx}, {mean})"
+    return st

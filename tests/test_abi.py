@@ -1,0 +1,106 @@
+"""The C ABI library: it loads, exports every declared entry point, sizes its
+workspace, and rejects bad arguments before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lwm_attn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lwm_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lwm():
+    from long_context_causal_attention_b200 import build
+    build.build()
+    import long_context_causal_attention_b200 as m
+    return m
+
+
+def test_library_exports_every_declared_symbol(lwm):
+    declared = _declared_functions()
+    assert set(declared) >= {"lwm_attn_fwd", "lwm_attn_bwd", "lwm_rope_apply",
+                             "lwm_attn_workspace_size", "lwm_attn_read_status",
+                             "lwm_status_string"}
+    lib = ctypes.CDLL(lwm.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) <= set(lwm.ENTRY_POINTS)
+
+
+def test_desc_struct_matches_header_layout(lwm):
+    d = lwm.LwmAttnDesc
+    assert ctypes.sizeof(d) == 64
+    assert d.rope_theta.offset == 40 and d.softmax_scale.offset == 48
+    assert d.segment_ids.offset == 56
+
+
+def _desc(lwm, **kw):
+    base = dict(batch=2, seqlen=300, heads=4, head_dim=128, dtype=0, causal=1,
+                rope_theta=1e6, softmax_scale=0.0, segment_ids=None)
+    base.update(kw)
+    return lwm.LwmAttnDesc(**base)
+
+
+def test_workspace_size(lwm):
+    d = _desc(lwm)
+    f = lwm.lwm_attn_workspace_size(d, False)
+    b = lwm.lwm_attn_workspace_size(d, True)
+    nel = 2 * 300 * 4 * 128
+    assert f >= 2 * nel * 2 and b >= f
+    assert f % 1024 == 0 and b % 1024 == 0
+    # no rotation: the rotated copies are not needed
+    assert lwm.lwm_attn_workspace_size(_desc(lwm, rope_theta=0.0), False) < f
+    assert lwm.lwm_attn_workspace_size(_desc(lwm, head_dim=96), False) == 0
+    assert lwm.lwm_attn_workspace_size(_desc(lwm, dtype=7), True) == 0
+
+
+def test_status_strings(lwm):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lwm.lwm_status_string(code).startswith("LWM_")
+    assert "unknown" in lwm.lwm_status_string(42)
+
+
+def test_argument_errors_return_before_any_launch(lwm):
+    lib = lwm._lib.lib()
+    P = 0x10000  # fake, aligned, never dereferenced: every check below fails first
+    big = 1 << 40
+    d = _desc(lwm)
+    args = lambda desc, ws=P, wsb=big, q=P: (ctypes.byref(desc), q, P, P, P, P, ws, wsb, None)
+    assert lib.lwm_attn_fwd(None, P, P, P, P, P, P, big, None) == -1
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, head_dim=96))) == -2
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, dtype=3))) == -1
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, causal=2))) == -1
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, rope_theta=float("nan")))) == -1
+    assert lib.lwm_attn_fwd(*args(d, q=None)) == -1
+    assert lib.lwm_attn_fwd(*args(d, q=P + 8)) == -3
+    assert lib.lwm_attn_fwd(*args(d, ws=None)) == -4
+    assert lib.lwm_attn_fwd(*args(d, wsb=1024)) == -4
+    assert lib.lwm_attn_fwd(*args(d, ws=P + 16)) == -3
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, heads=0))) == -1
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, segment_ids=P + 2))) == -3
+    # empty problems are a successful no-op
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, seqlen=0))) == 0
+    assert lib.lwm_attn_fwd(*args(_desc(lwm, batch=0))) == 0
+    bw = lambda desc, ws=P, wsb=big: (ctypes.byref(desc), P, P, P, P, P, P, P, P, P, ws, wsb, None)
+    assert lib.lwm_attn_bwd(*bw(d, wsb=lwm.lwm_attn_workspace_size(d, False) - 1)) == -4
+    assert lib.lwm_attn_bwd(*bw(_desc(lwm, head_dim=32))) == -2
+    assert lib.lwm_rope_apply(1, 8, 2, 7, 0, 1e4, P, P, 0, None) == -1
+    assert lib.lwm_rope_apply(1, 8, 2, 12, 0, 1e4, P, P, 0, None) == -2
+    assert lib.lwm_rope_apply(1, 8, 2, 64, 0, 1e4, P + 4, P, 0, None) == -3
+    assert lib.lwm_rope_apply(0, 8, 2, 64, 0, 1e4, None, None, 0, None) == 0
+    assert lib.lwm_attn_read_status(None, None) == -1
+
+
+def test_python_binding_requires_cuda_tensors(lwm):
+    import torch
+    q = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError):
+        lwm.lwm_attn_fwd(q, q, q)

@@ -1,0 +1,202 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small inputs are compared element by element on every output (O, LSE, dQ,
+dK, dV); they span several 128-row tiles with ragged tails, packed segments,
+padding, both mask modes, both dtypes, both head sizes and theta from 0 to
+5e7.  The named workloads are compared in the launch configuration the bench
+uses: in full where the oracle finishes in seconds, otherwise on sampled
+query rows (exact O/LSE/dQ per row) and on the last rows of sampled heads
+(exact dK/dV for the keys there).
+"""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity_util import assert_close, to64
+from workloads import WORKLOADS, Workload, make_tensors, random_segments, segment_ids
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lwm():
+    import long_context_causal_attention_b200 as m
+    return m
+
+
+def run(lwm, t, seg, w: Workload, backward=True):
+    dev = "cuda"
+    seg_d = torch.as_tensor(seg, dtype=torch.int32, device=dev) if seg is not None else None
+    o, lse = lwm.lwm_attn_fwd(t["q"], t["k"], t["v"], seg_d, causal=w.causal,
+                              rope_theta=w.theta, softmax_scale=w.scale)
+    out = {"o": o, "lse": lse}
+    if backward:
+        dq, dk, dv = lwm.lwm_attn_bwd(t["q"], t["k"], t["v"], o, lse, t["do"], seg_d,
+                                      causal=w.causal, rope_theta=w.theta,
+                                      softmax_scale=w.scale)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    return out
+
+
+def full_oracle(t, seg, w, backward=True):
+    q, k, v = (to64(t[n]) for n in ("q", "k", "v"))
+    do = to64(t["do"]) if backward else None
+    return oracle.attention_backward(q, k, v, do, seg, causal=w.causal, theta=w.theta,
+                                     scale=w.scale if w.scale > 0 else None)
+
+
+SMALL = [
+    # name, B, S, H, D, dtype, theta, causal, sigma, segments
+    ("s1", 1, 1, 2, 128, "bf16", 1e4, True, 0.5, "single"),
+    ("ragged127_pad", 2, 127, 2, 128, "bf16", 1e6, True, 0.5, "random_pad"),
+    ("tiles129_sharp", 1, 129, 3, 128, "bf16", 1e7, True, 2.0, "single"),
+    ("noncausal300", 2, 300, 2, 128, "bf16", 1e4, False, 1.0, "random"),
+    ("packed640_theta5e7", 1, 640, 2, 128, "bf16", 5e7, True, 2.0, "random_pad"),
+    ("d64_bf16", 2, 257, 2, 64, "bf16", 1e6, True, 1.0, "random"),
+    ("fp32_d128", 1, 200, 2, 128, "fp32", 1e4, True, 1.0, "random"),
+    ("fp32_noncausal_d64", 1, 190, 2, 64, "fp32", 1e6, False, 1.0, "random_pad"),
+    ("no_rope", 1, 384, 2, 128, "bf16", 0.0, True, 1.0, "single"),
+    ("long_segments_1000", 1, 1000, 2, 128, "bf16", 1e6, True, 1.0, "random_long"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_cases_full(lwm, case):
+    name, B, S, H, D, dt, theta, causal, sigma, segkind = case
+    w = Workload(name, B, S, H, D, dt, theta, causal=causal, sigma=sigma)
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    if segkind == "single":
+        seg = np.zeros((B, S), np.int32)
+    elif segkind == "random":
+        seg = random_segments(rng, B, S, 1, 150)
+    elif segkind == "random_long":
+        seg = random_segments(rng, B, S, 100, 700)
+    else:
+        seg = random_segments(rng, B, S, 1, 150, pad_tail=min(5, S - 1))
+        seg[:, :3] = -1
+    t = make_tensors(w, seed=7, device="cuda", with_grad_out=True)
+    got = run(lwm, t, seg, w)
+    ref = full_oracle(t, seg, w)
+    for key in ("o", "lse", "dq", "dk", "dv"):
+        assert_close(key, to64(got[key]), ref[key], dt)
+
+
+def test_tiny_packed_fp32_workload(lwm):
+    """B1 H1 D64 fp32, S=256 as segments 100 + 156, theta 1e4, causal."""
+    w = WORKLOADS["tiny_packed_fp32"]
+    seg = segment_ids(w)
+    t = make_tensors(w, seed=0, device="cuda", with_grad_out=True)
+    got = run(lwm, t, seg, w, backward=True)
+    ref = full_oracle(t, seg, w, backward=True)
+    for key in ("o", "lse", "dq", "dk", "dv"):
+        assert_close(key, to64(got[key]), ref[key], "fp32")
+
+
+def _sampled_rows(rng, B, S, H, n):
+    return [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(S))) for _ in range(n)]
+
+
+def check_rows(t, got, seg, w, samples, backward):
+    q, k, v = t["q"], t["k"], t["v"]
+    do = t.get("do") if backward else None
+    # oracle per (b, h): copy only that head to the host
+    by_head = {}
+    for s in samples:
+        by_head.setdefault((s[0], s[1]), []).append(s[2])
+    for (b, h), rows in by_head.items():
+        sl = lambda x: to64(x[b:b + 1, :, h:h + 1, :])
+        ref = oracle.attention_rows(sl(q), sl(k), sl(v), sl(do) if do is not None else None,
+                                    [(0, 0, i) for i in rows], seg[b:b + 1], causal=w.causal,
+                                    theta=w.theta)
+        assert_close(f"o[{b},{h}]", to64(got["o"][b, rows, h]), ref["o"], w.dtype)
+        assert_close(f"lse[{b},{h}]", to64(got["lse"][b, h, rows]), ref["lse"], w.dtype)
+        if backward:
+            assert_close(f"dq[{b},{h}]", to64(got["dq"][b, rows, h]), ref["dq"], w.dtype)
+
+
+def check_tail(t, got, seg, w, b, h, rows):
+    """Exact dK/dV (and O/LSE/dQ) for the last `rows` positions of head (b, h)."""
+    S = t["q"].shape[1]
+    r0 = S - rows
+    sl = lambda x: to64(x[b:b + 1, :, h:h + 1, :])
+    ref = oracle.attention_backward(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["do"]),
+                                    seg[b:b + 1], causal=w.causal, theta=w.theta, row_start=r0)
+    for key in ("dk", "dv", "dq", "o"):
+        assert_close(f"{key} tail[{b},{h}]", to64(got[key][b, r0:, h]), ref[key][0, r0:, 0], w.dtype)
+
+
+def test_fwd_32k_workload_sampled(lwm):
+    """B1 H32 D128 bf16, S=32768, one segment, theta 1e6, forward."""
+    w = WORKLOADS["fwd_32k"]
+    seg = segment_ids(w)
+    t = make_tensors(w, seed=0, device="cuda")
+    got = run(lwm, t, seg, w, backward=False)
+    rng = np.random.default_rng(1)
+    samples = _sampled_rows(rng, w.batch, w.seqlen, w.heads, 64)
+    samples += [(0, 5, w.seqlen - 1), (0, 31, 0), (0, 0, 127), (0, 0, 128)]
+    check_rows(t, got, seg, w, samples, backward=False)
+
+
+def test_packed_8k_workload(lwm):
+    """B4 H32 D128 bf16, S=8192 packed video/text segments, theta 1e6, fwd+bwd.
+
+    Two heads in full against the oracle, sampled rows on the rest, and the
+    per-segment gradient sums on every head."""
+    w = WORKLOADS["packed_8k"]
+    seg = segment_ids(w, seed=0)
+    t = make_tensors(w, seed=0, device="cuda")
+    got = run(lwm, t, seg, w, backward=True)
+    for b, h in ((0, 0), (3, 31)):
+        sl = lambda x: to64(x[b:b + 1, :, h:h + 1, :])
+        ref = oracle.attention_backward(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["do"]),
+                                        seg[b:b + 1], causal=True, theta=w.theta)
+        for key in ("o", "dq", "dk", "dv"):
+            assert_close(f"{key}[{b},{h}]", to64(got[key][b:b + 1, :, h:h + 1]), ref[key], "bf16")
+        assert_close(f"lse[{b},{h}]", to64(got["lse"][b, h]), ref["lse"][0, 0], "bf16")
+    rng = np.random.default_rng(2)
+    check_rows(t, got, seg, w, _sampled_rows(rng, w.batch, w.seqlen, w.heads, 64), True)
+    # per segment: sum_j dv_j == sum_i dO_i (softmax rows sum to one)
+    dv = got["dv"].double()
+    do = t["do"].double()
+    for b in range(w.batch):
+        ids = torch.as_tensor(seg[b], device="cuda", dtype=torch.int64)
+        n = int(ids.max()) + 1
+        sdv = torch.zeros(n, w.heads, w.head_dim, device="cuda", dtype=torch.float64)
+        sdo = torch.zeros_like(sdv)
+        sdv.index_add_(0, ids, dv[b]); sdo.index_add_(0, ids, do[b])
+        cnt = torch.bincount(ids).double()[:, None, None]
+        err = (sdv - sdo).abs() / cnt.sqrt()
+        assert float(err.max()) < 2e-2, float(err.max())
+
+
+@pytest.mark.parametrize("name", ["long_128k", "million_1m"])
+def test_long_workloads_sampled(lwm, name):
+    """128K and 1M tokens, one segment, fwd+bwd: 64 random query rows and the
+    last 256 rows of two heads against the oracle."""
+    w = WORKLOADS[name]
+    if name == "million_1m" and torch.cuda.get_device_properties(0).total_memory < 150e9:
+        pytest.skip("needs a 180 GB device")
+    seg = segment_ids(w)
+    t = make_tensors(w, seed=0, device="cuda")
+    got = run(lwm, t, seg, w, backward=True)
+    rng = np.random.default_rng(3)
+    samples = _sampled_rows(rng, w.batch, w.seqlen, w.heads, 64)
+    check_rows(t, got, seg, w, samples, backward=True)
+    for b, h in ((0, 0), (0, 17)):
+        check_tail(t, got, seg, w, b, h, rows=256)
+    # sum over all keys of dv equals sum over all rows of dO, per head
+    err = (chunked_sum(got["dv"]) - chunked_sum(t["do"])).abs().max()
+    assert float(err) < 2e-2 * math.sqrt(w.seqlen)
+
+
+def chunked_sum(x, chunk=65536):
+    """Sum over the sequence axis in float64 without a full-size float64 copy."""
+    acc = torch.zeros(x.shape[0], x.shape[2], x.shape[3], dtype=torch.float64, device=x.device)
+    for s0 in range(0, x.shape[1], chunk):
+        acc += x[:, s0:s0 + chunk].double().sum(1)
+    return acc
