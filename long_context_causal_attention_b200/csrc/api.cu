@@ -26,12 +26,27 @@ void record_event(int which, cudaStream_t st) {
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
-Path choose_path(const Problem& p) {
-  static const bool force_simt = [] {
+bool tensor_core_shape(const Problem& p) {
+  return p.dtype == LWM_DTYPE_BF16 && p.D == 128 && p.S < ((int64_t)1 << 31);
+}
+
+// LWM_ATTN_FORCE_SIMT=1 routes every call to the CUDA-core kernels (used to
+// cross-check the two kernel families against each other).
+static bool force_simt() {
+  static const bool v = [] {
     const char* e = std::getenv("LWM_ATTN_FORCE_SIMT");
     return e && e[0] == '1';
   }();
-  if (force_simt) return Path::kSimt;
+  return v;
+}
+
+Path choose_fwd_path(const Problem& p) {
+  if (force_simt() || !tensor_core_shape(p) || !sm100_available()) return Path::kSimt;
+  return Path::kSm100;
+}
+
+Path choose_bwd_path(const Problem& p) {
+  (void)p;
   return Path::kSimt;
 }
 
@@ -58,7 +73,7 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
   }
   if (bwd) {
     w.delta = static_cast<float*>(take((size_t)p.B * p.H * p.S * sizeof(float)));
-    if (choose_path(p) == Path::kSm100) w.dq_acc = static_cast<float*>(take(nel * sizeof(float)));
+    if (tensor_core_shape(p)) w.dq_acc = static_cast<float*>(take(nel * sizeof(float)));
   }
   w.bytes = align_up(off, 1024);
   if (ws) *ws = w;
@@ -150,7 +165,10 @@ lwm_status lwm_attn_fwd(const lwm_attn_desc* desc, const void* q, const void* k,
   cudaError_t e = prologue(p, w, q, k, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   record_event(0, st);
-  e = launch_simt_fwd(p, w, v, o, lse, st);
+  if (choose_fwd_path(p) == Path::kSm100)
+    e = launch_sm100_fwd(p, w, v, o, lse, st);
+  else
+    e = launch_simt_fwd(p, w, v, o, lse, st);
   record_event(1, st);
   return cuda_status(e);
 }

@@ -1,0 +1,615 @@
+// Forward attention on the 5th-generation tensor cores (sm_100a), bf16, D=128.
+//
+// What it computes: exact causal softmax attention with a packing mask
+// (LWM research note, "模型架构": exact blockwise attention; "训练方法":
+// Masked Sequence Packing), over q and k that the RoPE pre-pass has already
+// rotated.  Output O (bf16) and LSE = ln sum exp(s) per row (fp32).
+//
+// Design (one persistent CTA per SM, 384 threads):
+//   warp 0      TMA producer: Q tile pair once per work item, then K_j and V_j
+//               for every key tile j the pair needs, through 2-stage rings
+//               (K runs one tile ahead of V).
+//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
+//               with tcgen05.mma, fp32 accumulators in tensor memory.
+//   warp 2      allocates / frees the 512 tensor-memory columns.
+//   warps 4-7   softmax for query tile t=0 (one row per thread),
+//   warps 8-11  softmax for query tile t=1: read S from TMEM, mask partial
+//               tiles, online max/sum in log2 units, write P (bf16) back
+//               into the S columns for the PV MMA, rescale O when the
+//               running max grows by more than 2^8, then normalise and
+//               store O and LSE.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
+// P_t is packed bf16 in the first 64 columns of S_t.
+// The MMA issue order ping-pongs the two tiles so one softmax warpgroup
+// works while the tensor core runs the other tile's MMAs:
+//   S_0(j) S_1(j) | PV_0(j) S_0(j+1) | PV_1(j) S_1(j+1) | ...
+// Work items (b, h, pair of 128-row query tiles) go to CTAs round-robin in
+// head-major order with the costliest pair of each head first, so CTAs that
+// run at the same time share one head's K/V through L2.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace lwm {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = 128 * kD * 2;  // one 128 x 128 bf16 tile = two 16 KB boxes
+constexpr uint32_t kBoxBytes = kTileBytes / 2;
+constexpr float kRescaleLog2 = 8.0f;  // keep a stale max until the true one is 2^8 larger
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr uint32_t OFF_Q = 0;                          // Q_0, Q_1
+constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;     // K ring, 2 stages
+constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;     // V ring, 2 stages
+constexpr uint32_t OFF_BAR = OFF_V + 2 * kTileBytes;   // mbarriers
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;           // TMEM base, abort flag
+constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;  // + alignment slack
+
+// barrier slots (8 bytes each)
+enum : uint32_t {
+  B_Q_FULL = 0, B_Q_EMPTY = 1,
+  B_K_FULL = 2,   // 2 stages
+  B_K_EMPTY = 4,  // 2
+  B_V_FULL = 6,   // 2
+  B_V_EMPTY = 8,  // 2
+  B_S_FULL = 10,  // per tile
+  B_P_FULL = 12,  // per tile
+  B_O_FULL = 14,  // per tile
+  B_O_EMPTY = 16, // per tile
+  B_FIN = 18,
+  B_COUNT = 19
+};
+
+struct FwdParams {
+  const int32_t* seg;    // [B, S] or null
+  const int32_t* tmin;   // [B, nT] (valid when seg != null)
+  const int32_t* tmax;
+  const int32_t* q_lo;
+  __nv_bfloat16* o;
+  float* lse;
+  DeviceStatus* status;
+  int64_t S;
+  int H, B, n_tiles, n_pairs;
+  float scale_log2;
+  int causal;
+};
+
+struct Item {
+  int b, h;
+  int qt[2];       // query tile index, -1 when past the end
+  int lo[2], hi[2];
+  int32_t qmin[2], qmax[2];
+};
+
+__device__ __forceinline__ bool meet(int32_t a0, int32_t a1, int32_t b0, int32_t b1) {
+  return a1 >= 0 && b1 >= 0 && a0 <= b1 && b0 <= a1;
+}
+
+__device__ __forceinline__ Item decode(const FwdParams& p, int idx) {
+  Item it;
+  const int bh = idx / p.n_pairs;
+  const int pr = p.n_pairs - 1 - (idx % p.n_pairs);
+  it.b = bh / p.H;
+  it.h = bh % p.H;
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * pr + t;
+    it.qt[t] = qt < p.n_tiles ? qt : -1;
+    it.lo[t] = 0;
+    it.hi[t] = -1;
+    it.qmin[t] = 0;
+    it.qmax[t] = 0;
+    if (it.qt[t] < 0) continue;
+    const size_t ti = (size_t)it.b * p.n_tiles + qt;
+    it.hi[t] = p.causal ? qt : p.n_tiles - 1;
+    if (p.seg) {
+      it.lo[t] = p.q_lo[ti];
+      it.qmin[t] = p.tmin[ti];
+      it.qmax[t] = p.tmax[ti];
+    }
+  }
+  return it;
+}
+
+__device__ __forceinline__ bool rel(const FwdParams& p, const Item& it, int t, int j) {
+  if (it.qt[t] < 0 || j < it.lo[t] || j > it.hi[t]) return false;
+  if (!p.seg) return true;
+  const size_t kj = (size_t)it.b * p.n_tiles + j;
+  return meet(it.qmin[t], it.qmax[t], p.tmin[kj], p.tmax[kj]);
+}
+
+__device__ __forceinline__ bool rel_any(const FwdParams& p, const Item& it, int j) {
+  return rel(p, it, 0, j) || rel(p, it, 1, j);
+}
+
+__device__ __forceinline__ int next_any(const FwdParams& p, const Item& it, int j, int jend) {
+  for (++j; j <= jend; ++j)
+    if (rel_any(p, it, j)) return j;
+  return -1;
+}
+
+__device__ __forceinline__ void union_range(const Item& it, int* jlo, int* jhi) {
+  int lo = 1 << 30, hi = -1;
+  for (int t = 0; t < 2; ++t) {
+    if (it.qt[t] < 0 || it.lo[t] > it.hi[t]) continue;
+    lo = min(lo, it.lo[t]);
+    hi = max(hi, it.hi[t]);
+  }
+  *jlo = lo;
+  *jhi = hi;
+}
+
+// A wait that ignores the abort flag: used only while draining.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t bar0 = base + OFF_BAR;
+  auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  const Abort ab{abort_flag, p.status};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = p.B * p.H * p.n_pairs;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(B_Q_FULL), 1);
+    mbar_init(bar(B_Q_EMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_K_FULL + s), 1);
+      mbar_init(bar(B_K_EMPTY + s), 1);
+      mbar_init(bar(B_V_FULL + s), 1);
+      mbar_init(bar(B_V_EMPTY + s), 1);
+      mbar_init(bar(B_S_FULL + s), 1);
+      mbar_init(bar(B_P_FULL + s), 128);
+      mbar_init(bar(B_O_FULL + s), 1);
+      mbar_init(bar(B_O_EMPTY + s), 128);
+    }
+    mbar_init(bar(B_FIN), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // per-stage state the producer keeps for draining after an abort
+  uint32_t k_issued = 0, v_issued = 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      uint32_t k_it = 0, v_it = 0;
+      int items = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+        const Item it = decode(p, idx);
+        if (items > 0 && !mbar_wait(bar(B_Q_EMPTY), (items - 1) & 1, ab, 1)) { ok = false; break; }
+        const int nq = (it.qt[0] >= 0) + (it.qt[1] >= 0);
+        mbar_expect_tx(bar(B_Q_FULL), nq * kTileBytes);
+        for (int t = 0; t < 2; ++t) {
+          if (it.qt[t] < 0) continue;
+          const uint32_t dst = base + OFF_Q + t * kTileBytes;
+          tma_load_4d(dst, &tm_q, bar(B_Q_FULL), 0, it.h, it.qt[t] * 128, it.b);
+          tma_load_4d(dst + kBoxBytes, &tm_q, bar(B_Q_FULL), 64, it.h, it.qt[t] * 128, it.b);
+        }
+        int jlo, jhi;
+        union_range(it, &jlo, &jhi);
+        int j = (jlo <= jhi && rel_any(p, it, jlo)) ? jlo : next_any(p, it, jlo, jhi);
+        auto load_k = [&](int jj) -> bool {
+          const uint32_t s = k_it & 1;
+          if (!mbar_wait(bar(B_K_EMPTY + s), ((k_it >> 1) & 1) ^ 1, ab, 2)) return false;
+          mbar_expect_tx(bar(B_K_FULL + s), kTileBytes);
+          const uint32_t dst = base + OFF_K + s * kTileBytes;
+          tma_load_4d(dst, &tm_k, bar(B_K_FULL + s), 0, it.h, jj * 128, it.b);
+          tma_load_4d(dst + kBoxBytes, &tm_k, bar(B_K_FULL + s), 64, it.h, jj * 128, it.b);
+          ++k_it;
+          k_issued = k_it;
+          return true;
+        };
+        auto load_v = [&](int jj) -> bool {
+          const uint32_t s = v_it & 1;
+          if (!mbar_wait(bar(B_V_EMPTY + s), ((v_it >> 1) & 1) ^ 1, ab, 3)) return false;
+          mbar_expect_tx(bar(B_V_FULL + s), kTileBytes);
+          const uint32_t dst = base + OFF_V + s * kTileBytes;
+          tma_load_4d(dst, &tm_v, bar(B_V_FULL + s), 0, it.h, jj * 128, it.b);
+          tma_load_4d(dst + kBoxBytes, &tm_v, bar(B_V_FULL + s), 64, it.h, jj * 128, it.b);
+          ++v_it;
+          v_issued = v_it;
+          return true;
+        };
+        if (j >= 0 && !load_k(j)) { ok = false; break; }
+        while (j >= 0) {
+          const int jn = next_any(p, it, j, jhi);
+          if (jn >= 0 && !load_k(jn)) { ok = false; break; }
+          if (!load_v(j)) { ok = false; break; }
+          j = jn;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
+      constexpr uint32_t kIdPV = idesc_bf16(128, 128, 0, 1); // P (TMEM) x V (MN-major)
+      uint32_t k_it = 0, v_it = 0, p_cnt[2] = {0, 0}, act[2] = {0, 0};
+      int items = 0;
+      bool ok = true;
+      const uint32_t sq0 = base + OFF_Q;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+        const Item it = decode(p, idx);
+        if (!mbar_wait(bar(B_Q_FULL), items & 1, ab, 4)) { ok = false; break; }
+        tc_fence_after();
+        int jlo, jhi;
+        union_range(it, &jlo, &jhi);
+        int jc = (jlo <= jhi && rel_any(p, it, jlo)) ? jlo : next_any(p, it, jlo, jhi);
+        bool first_pv[2] = {true, true}, active[2] = {false, false};
+
+        auto issue_s = [&](int t) {
+          const uint32_t ks = base + OFF_K + (k_it & 1) * kTileBytes;
+          const uint32_t qs = sq0 + t * kTileBytes;
+          const uint32_t d = tmem + (uint32_t)(t * 128);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+            mma_ss(d, smem_desc_sw128(qs + off, 16, 1024), smem_desc_sw128(ks + off, 16, 1024),
+                   kIdS, kk > 0);
+          }
+          mma_commit(bar(B_S_FULL + t));
+        };
+        auto issue_pv = [&](int t) {
+          const uint32_t vs = base + OFF_V + (v_it & 1) * kTileBytes;
+          const uint32_t d = tmem + 256u + (uint32_t)(t * 128);
+          const uint32_t a = tmem + (uint32_t)(t * 128);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            mma_ts(d, a + kk * 8, smem_desc_sw128(vs + kk * 2048, kBoxBytes, 1024), kIdPV,
+                   (kk > 0 || !first_pv[t]) ? 1u : 0u);
+          }
+          first_pv[t] = false;
+        };
+
+        if (jc >= 0) {
+          if (!mbar_wait(bar(B_K_FULL + (k_it & 1)), (k_it >> 1) & 1, ab, 5)) { ok = false; break; }
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if (rel(p, it, t, jc)) issue_s(t);
+          mma_commit(bar(B_K_EMPTY + (k_it & 1)));
+          ++k_it;
+        }
+        while (jc >= 0 && ok) {
+          const int jn = next_any(p, it, jc, jhi);
+          bool v_ready = false, k_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (rel(p, it, t, jc)) {
+              if (!v_ready) {
+                if (!mbar_wait(bar(B_V_FULL + (v_it & 1)), (v_it >> 1) & 1, ab, 6)) { ok = false; break; }
+                v_ready = true;
+              }
+              if (first_pv[t] && act[t] > 0) {
+                if (!mbar_wait(bar(B_O_EMPTY + t), (act[t] - 1) & 1, ab, 7)) { ok = false; break; }
+              }
+              if (!mbar_wait(bar(B_P_FULL + t), p_cnt[t] & 1, ab, 8)) { ok = false; break; }
+              ++p_cnt[t];
+              tc_fence_after();
+              issue_pv(t);
+              active[t] = true;
+            }
+            if (jn >= 0 && rel(p, it, t, jn)) {
+              if (!k_ready) {
+                if (!mbar_wait(bar(B_K_FULL + (k_it & 1)), (k_it >> 1) & 1, ab, 9)) { ok = false; break; }
+                tc_fence_after();
+                k_ready = true;
+              }
+              issue_s(t);
+            }
+          }
+          if (!ok) break;
+          if (k_ready) {
+            mma_commit(bar(B_K_EMPTY + (k_it & 1)));
+            ++k_it;
+          }
+          mma_commit(bar(B_V_EMPTY + (v_it & 1)));
+          ++v_it;
+          jc = jn;
+        }
+        if (!ok) break;
+        for (int t = 0; t < 2; ++t) {
+          if (active[t]) {
+            mma_commit(bar(B_O_FULL + t));
+            ++act[t];
+          }
+        }
+        mma_commit(bar(B_Q_EMPTY));
+      }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- softmax
+    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
+    const int tid = threadIdx.x - 128 - 128 * t;  // 0..127 = TMEM lane = row in tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (uint32_t)(t * 128);
+    const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(t * 128);
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const Item it = decode(p, idx);
+      if (it.qt[t] < 0) continue;
+      const int64_t row = (int64_t)it.qt[t] * 128 + tid;
+      const bool row_ok = row < p.S;
+      int32_t seg_row = row_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + row] : 0) : -1;
+      const size_t tok = (size_t)it.b * p.S + (size_t)(row_ok ? row : 0);
+      float m = -INFINITY, l = 0.f;
+      int ntiles = 0;
+      for (int j = it.lo[t]; j <= it.hi[t]; ++j) {
+        if (!rel(p, it, t, j)) continue;
+        // tile needs element masking?
+        bool partial = (p.causal && j == it.qt[t]) || ((int64_t)(j + 1) * 128 > p.S);
+        if (p.seg) {
+          const size_t kj = (size_t)it.b * p.n_tiles + j;
+          const int32_t a0 = p.tmin[kj], a1 = p.tmax[kj];
+          partial |= !(it.qmin[t] >= 0 && it.qmin[t] == it.qmax[t] && a0 == it.qmin[t] &&
+                       a1 == it.qmin[t]);
+        }
+        // every thread of the warp must agree before the .sync.aligned TMEM ops
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + t), s_cnt & 1, ab, 10 + t))) {
+          ok = false;
+          break;
+        }
+        ++s_cnt;
+        tc_fence_after();
+        // S row in registers (raw scores); masked entries become -inf.
+        uint32_t r[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+        tmem_wait_ld();
+        if (partial) {
+          // keys c <= lim are inside the row's causal window and the sequence
+          const int64_t d = row - (int64_t)j * 128;
+          const int64_t kvalid = p.S - (int64_t)j * 128;
+          int lim = p.causal ? (int)(d < -1 ? -1 : (d > 127 ? 127 : d)) : 127;
+          if (kvalid - 1 < lim) lim = (int)(kvalid - 1);
+          if (seg_row < 0) lim = -1;
+          // 128-bit keep mask, built without touching the score registers
+          const int32_t* ks = p.seg ? p.seg + (size_t)it.b * p.S + (size_t)j * 128 : nullptr;
+          uint32_t mw[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t bits = 0;
+#pragma unroll 4
+            for (int c = 0; c < 32; ++c) {
+              const int kc = w * 32 + c;
+              const bool okk = kc <= lim && (ks == nullptr || __ldg(ks + kc) == seg_row);
+              bits |= (uint32_t)okk << c;
+            }
+            mw[w] = bits;
+          }
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            r[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? r[c] : 0xff800000u;
+        }
+        float mxr = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mxr = fmaxf(mxr, __uint_as_float(r[c]));
+        const float mx = mxr * p.scale_log2;  // scale > 0 keeps the order
+        float fscale = 1.f;  // factor for O when the running max moves
+        if (mx != -INFINITY) {
+          if (m == -INFINITY) {
+            m = mx;
+          } else if (mx > m + kRescaleLog2) {
+            fscale = fast_exp2(m - mx);
+            l *= fscale;
+            m = mx;
+          }
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        float sum = 0.f;
+        // p = 2^(s * scale * log2e - m), packed two bf16 per column in place
+#pragma unroll
+        for (int u = 0; u < 64; ++u) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(r[2 * u]), p.scale_log2, neg_m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(r[2 * u + 1]), p.scale_log2, neg_m));
+          sum += p0 + p1;
+          r[u] = pack_bf16(p0, p1);
+        }
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        if (__any_sync(0xffffffffu, fscale != 1.f)) {  // warp-uniform: TMEM ops are .sync.aligned
+          // the previous PV of this tile has completed (it was issued before
+          // the S MMA whose completion this thread waited for)
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * fscale);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        l += sum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_P_FULL + t));
+        ++ntiles;
+      }
+      if (!ok) break;
+      __nv_bfloat16* orow = p.o + (tok * p.H + it.h) * kD;
+      if (ntiles == 0) {
+        if (row_ok) {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+          p.lse[((size_t)it.b * p.H + it.h) * p.S + row] = -INFINITY;
+        }
+        continue;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL + t), o_cnt & 1, ab, 12 + t))) {
+        ok = false;
+        break;
+      }
+      ++o_cnt;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + c * 32, r);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            pk[u] = pack_bf16(__uint_as_float(r[2 * u]) * inv, __uint_as_float(r[2 * u + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+      if (row_ok)
+        p.lse[((size_t)it.b * p.H + it.h) * p.S + row] =
+            l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(bar(B_O_EMPTY + t));
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 1 && lane == 0) {
+      mma_commit(bar(B_FIN));
+      drain_wait(bar(B_FIN), 0);
+    }
+    if (warp == 0 && lane == 0) {
+      // at most one load in flight per ring stage: the latest one issued
+      for (uint32_t n = (k_issued > 2 ? k_issued - 2 : 0); n < k_issued; ++n)
+        drain_wait(bar(B_K_FULL + (n & 1)), (n >> 1) & 1);
+      for (uint32_t n = (v_issued > 2 ? v_issued - 2 : 0); n < v_issued; ++n)
+        drain_wait(bar(B_V_FULL + (n & 1)), (n >> 1) & 1);
+    }
+  }
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+}  // namespace
+
+// [B, S, H, D] bf16 as a 4-D tensor map {D, H, S, B}, 64 x 1 x 128 x 1 boxes,
+// 128-byte swizzle (the canonical K-major / MN-major SW128 operand layout).
+bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2), (cuuint64_t)(S * H * D * 2)};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+bool sm100_available() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  return major == 10 && minor == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void* v, void* o,
+                             float* lse, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D))
+    return cudaErrorInvalidValue;
+  FwdParams p{};
+  p.seg = pb.seg;
+  p.tmin = ws.tile_min;
+  p.tmax = ws.tile_max;
+  p.q_lo = ws.q_lo;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = ws.status;
+  p.S = pb.S;
+  p.H = (int)pb.H;
+  p.B = (int)pb.B;
+  p.n_tiles = (int)pb.n_tiles;
+  p.n_pairs = (int)((pb.n_tiles + 1) / 2);
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.causal = pb.causal;
+  const int64_t n_items = pb.B * pb.H * p.n_pairs;
+  if (n_items == 0) return cudaSuccess;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
+  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace lwm

@@ -39,7 +39,12 @@ struct Workspace {
 
 enum class Path { kSimt = 0, kSm100 = 1 };
 
-Path choose_path(const Problem& p);
+// Which kernels serve the forward / backward of this problem on this device.
+Path choose_fwd_path(const Problem& p);
+Path choose_bwd_path(const Problem& p);
+// bf16, head_dim 128: the shape the tensor-core kernels are built for.
+bool tensor_core_shape(const Problem& p);
+bool sm100_available();
 
 // Instrumentation: kernels launched so far (process-wide).
 void note_launches(int n);
@@ -51,6 +56,9 @@ cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, d
 cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st);
 cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float* delta,
                          cudaStream_t st);
+
+cudaError_t launch_sm100_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
+                             float* lse, cudaStream_t st);
 
 cudaError_t launch_simt_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                             float* lse, cudaStream_t st);

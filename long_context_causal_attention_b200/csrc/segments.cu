@@ -2,9 +2,12 @@
 //
 // LWM research note, section "训练方法", Masked Sequence Packing: samples
 // packed into one row attend only to themselves.  Per 128-token tile this
-// records the smallest and largest non-negative segment id; two tiles can
-// only share an allowed pair when their id ranges intersect, so every other
-// tile pair is skipped without being loaded.  From the bounds it also derives,
+// records the smallest and largest non-negative segment id (tile_min is set
+// to -1 instead when the tile holds any padding token, id < 0; tile_max is
+// -1 when the tile holds no valid token).  Two tiles can only share an
+// allowed pair when their id ranges intersect, so every other tile pair is
+// skipped without being loaded, and a tile pair is free of masking inside
+// when all four bounds are the same non-negative id.  From the bounds it also derives,
 // per query tile, the first key tile it may need (q_lo) and, per key tile, the
 // last query tile it may feed (k_hi).  Both are sound for any ids; for ids in
 // contiguous runs (what packing produces) they are tight.
@@ -24,20 +27,23 @@ __global__ void tile_bounds_kernel(const int32_t* __restrict__ seg, int64_t B, i
   const int64_t b = idx / n_tiles, t = idx % n_tiles;
   const int64_t i0 = t * kTile, i1 = min(S, i0 + kTile);
   int32_t lo = INT_MAX, hi = -1;
+  bool pad = false;
   const int32_t* row = seg + b * S;
   for (int64_t i = i0; i < i1; ++i) {
     const int32_t s = row[i];
     if (s >= 0) {
       lo = min(lo, s);
       hi = max(hi, s);
+    } else {
+      pad = true;
     }
   }
-  tmin[idx] = lo;
+  tmin[idx] = (pad || hi < 0) ? -1 : lo;
   tmax[idx] = hi;
 }
 
 __device__ __forceinline__ bool meet(int32_t a0, int32_t a1, int32_t b0, int32_t b1) {
-  return a0 <= a1 && b0 <= b1 && a0 <= b1 && b0 <= a1;
+  return a1 >= 0 && b1 >= 0 && a0 <= b1 && b0 <= a1;
 }
 
 __global__ void tile_ranges_kernel(const int32_t* __restrict__ tmin, const int32_t* __restrict__ tmax,

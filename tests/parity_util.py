@@ -9,13 +9,22 @@ The bf16 bound is the one stated for this method's parity; the LSE bound
 follows from it: rotated q and k are rounded to bf16 (relative 2^-9), which
 moves a score of size |s| by about |s| 2^-8, well under 2e-2 for the score
 scales of these workloads.
+
+"bf16_sharp" is for stress inputs with q, k ~ N(0, 4) (score std ~4, far
+sharper than any named workload): the tensor cores take the rotated q and k
+as bf16, so each rotated element is rounded once more (relative 2^-9) than
+in the oracle, which rotates the exact inputs in float64.  A score of size
+16 then moves by ~0.06.  tests/test_tolerance_model.py runs the oracle on
+exactly that rounding and finds up to ~0.10 max / ~0.0045 mean on O, dQ, dK
+at sigma 2; adding the final bf16 rounding of outputs up to |16| (half an
+ulp = 0.03) gives the sharp bound: 0.2 max, 8e-3 mean.
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-TOL = {"bf16": (2e-2, 2e-3), "fp32": (1e-4, 1e-4)}
+TOL = {"bf16": (2e-2, 2e-3), "fp32": (1e-4, 1e-4), "bf16_sharp": (2e-1, 8e-3)}
 
 
 def to64(t: torch.Tensor) -> np.ndarray:

@@ -54,9 +54,11 @@ SMALL = [
     # name, B, S, H, D, dtype, theta, causal, sigma, segments
     ("s1", 1, 1, 2, 128, "bf16", 1e4, True, 0.5, "single"),
     ("ragged127_pad", 2, 127, 2, 128, "bf16", 1e6, True, 0.5, "random_pad"),
+    ("tiles129", 1, 129, 3, 128, "bf16", 1e7, True, 1.0, "single"),
     ("tiles129_sharp", 1, 129, 3, 128, "bf16", 1e7, True, 2.0, "single"),
     ("noncausal300", 2, 300, 2, 128, "bf16", 1e4, False, 1.0, "random"),
-    ("packed640_theta5e7", 1, 640, 2, 128, "bf16", 5e7, True, 2.0, "random_pad"),
+    ("packed640_theta5e7", 1, 640, 2, 128, "bf16", 5e7, True, 1.0, "random_pad"),
+    ("packed640_sharp", 1, 640, 2, 128, "bf16", 5e7, True, 2.0, "random_pad"),
     ("d64_bf16", 2, 257, 2, 64, "bf16", 1e6, True, 1.0, "random"),
     ("fp32_d128", 1, 200, 2, 128, "fp32", 1e4, True, 1.0, "random"),
     ("fp32_noncausal_d64", 1, 190, 2, 64, "fp32", 1e6, False, 1.0, "random_pad"),
@@ -82,8 +84,9 @@ def test_small_cases_full(lwm, case):
     t = make_tensors(w, seed=7, device="cuda", with_grad_out=True)
     got = run(lwm, t, seg, w)
     ref = full_oracle(t, seg, w)
+    tol = "bf16_sharp" if (dt == "bf16" and sigma > 1.0) else dt
     for key in ("o", "lse", "dq", "dk", "dv"):
-        assert_close(key, to64(got[key]), ref[key], dt)
+        assert_close(key, to64(got[key]), ref[key], tol)
 
 
 def test_tiny_packed_fp32_workload(lwm):
