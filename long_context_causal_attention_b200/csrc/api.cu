@@ -46,8 +46,8 @@ Path choose_fwd_path(const Problem& p) {
 }
 
 Path choose_bwd_path(const Problem& p) {
-  (void)p;
-  return Path::kSimt;
+  if (force_simt() || !tensor_core_shape(p) || !sm100_available()) return Path::kSimt;
+  return Path::kSm100;
 }
 
 size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
@@ -73,7 +73,12 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
   }
   if (bwd) {
     w.delta = static_cast<float*>(take((size_t)p.B * p.H * p.S * sizeof(float)));
-    if (tensor_core_shape(p)) w.dq_acc = static_cast<float*>(take(nel * sizeof(float)));
+    if (tensor_core_shape(p)) {
+      const size_t padded = (size_t)p.B * p.H * (size_t)p.n_tiles * kTile * sizeof(float);
+      w.lse2_pad = static_cast<float*>(take(padded));
+      w.delta_pad = static_cast<float*>(take(padded));
+      w.dq_acc = static_cast<float*>(take(nel * sizeof(float)));
+    }
   }
   w.bytes = align_up(off, 1024);
   if (ws) *ws = w;
@@ -190,6 +195,19 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = prologue(p, w, q, k, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
+  if (choose_bwd_path(p) == Path::kSm100) {
+    const size_t nel = (size_t)p.B * p.S * p.H * p.D;
+    e = cudaMemsetAsync(w.dq_acc, 0, nel * sizeof(float), st);
+    if (e != cudaSuccess) return LWM_ERR_CUDA;
+    e = launch_bwd_prep(p, o, d_o, lse, w, st);
+    if (e != cudaSuccess) return LWM_ERR_CUDA;
+    record_event(2, st);
+    e = launch_sm100_bwd(p, w, v, d_o, dk, dv, st);
+    record_event(3, st);
+    if (e != cudaSuccess) return LWM_ERR_CUDA;
+    e = launch_dq_post(p, w, dq, st);
+    return cuda_status(e);
+  }
   e = launch_delta(p, o, d_o, w.delta, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   record_event(2, st);

@@ -1,0 +1,565 @@
+// Backward attention on the 5th-generation tensor cores (sm_100a), bf16, D=128.
+//
+// Gradients of sum(O * dO) for exact causal attention with a packing mask
+// (LWM research note, "训练方法": training through the layer, Masked Sequence
+// Packing).  P is recomputed from the saved LSE, as in the FlashAttention
+// entry of the paper card's references; the backward is FlashAttention's
+// five products per (query tile i, key tile j):
+//   S^T  = K~_j Q~_i^T            P^T  = exp(S^T * scale - LSE_i)
+//   dP^T = V_j dO_i^T             dS^T = P^T o (dP^T - D_i),  D_i = dO_i . O_i
+//   dV_j += P^T dO_i              dK~_j += dS^T Q~_i      dQ~_i += dS K~_j
+//
+// One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
+// walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
+// tensor memory for the whole walk, dQ partials are added into an fp32
+// buffer with vector reductions.  Roles (384 threads):
+//   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i per step
+//               through a 2-stage ring.
+//   warp 1      MMA issuer (one thread).
+//   warp 2      tensor-memory allocation.
+//   warps 4-7   element-wise work on query columns 0-63, warps 8-11 on
+//               columns 64-127: P^T into TMEM (bf16, over S^T), dS^T into
+//               shared memory (bf16, 128-byte swizzle), the dQ drain, and
+//               the dK/dV epilogue (scale, inverse RoPE, bf16).
+// TMEM columns: S^T/P^T [0,128), dP^T then dQ [128,256), dV [256,384),
+// dK [384,512).  MMA issue order per step:
+//   S(i) | dP(i) after drain(i-1) | dV(i) after P(i) | dK(i) dQ(i) after dS(i) | S(i+1)
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace lwm {
+
+bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
+int sm_count();
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = 128 * kD * 2;
+constexpr uint32_t kBoxBytes = kTileBytes / 2;
+
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = OFF_K + kTileBytes;
+constexpr uint32_t OFF_Q = OFF_V + kTileBytes;       // 2 stages
+constexpr uint32_t OFF_DO = OFF_Q + 2 * kTileBytes;  // 2 stages
+constexpr uint32_t OFF_DS = OFF_DO + 2 * kTileBytes;
+constexpr uint32_t OFF_BAR = OFF_DS + kTileBytes;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
+
+enum : uint32_t {
+  B_KV_FULL = 0, B_KV_EMPTY = 1,
+  B_QD_FULL = 2,   // 2 stages
+  B_QD_EMPTY = 4,  // 2 stages
+  B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_DS_FULL = 9, B_DQ_FULL = 10, B_DRAIN = 11,
+  B_DKV_FULL = 12, B_DKV_EMPTY = 13, B_FIN = 14
+};
+
+struct BwdParams {
+  const int32_t* seg;
+  const int32_t* tmin;
+  const int32_t* tmax;
+  const int32_t* k_hi;
+  const float* lse2;   // [B, H, nT*128]: LSE * log2(e), +inf where the row has no keys
+  const float* dpad;   // [B, H, nT*128]: dot(dO, O), 0 past the end
+  float* dq_acc;       // [B, S, H, D]
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  DeviceStatus* status;
+  int64_t S;
+  int H, B, n_tiles;
+  float scale, scale_log2;
+  int causal, rotate;
+  double log2_theta;
+};
+
+struct Item {
+  int b, h, j;
+  int lo, hi;          // query tile range
+  int32_t kmin, kmax;  // key tile id range
+};
+
+__device__ __forceinline__ bool meet(int32_t a0, int32_t a1, int32_t b0, int32_t b1) {
+  return a1 >= 0 && b1 >= 0 && a0 <= b1 && b0 <= a1;
+}
+
+__device__ __forceinline__ Item decode(const BwdParams& p, int idx) {
+  Item it;
+  const int bh = idx / p.n_tiles;
+  it.j = idx % p.n_tiles;  // ascending key tile = most query tiles first (causal)
+  it.b = bh / p.H;
+  it.h = bh % p.H;
+  it.lo = p.causal ? it.j : 0;
+  it.hi = p.n_tiles - 1;
+  it.kmin = 0;
+  it.kmax = 0;
+  if (p.seg) {
+    const size_t kj = (size_t)it.b * p.n_tiles + it.j;
+    it.hi = p.k_hi[kj];
+    it.kmin = p.tmin[kj];
+    it.kmax = p.tmax[kj];
+  }
+  return it;
+}
+
+__device__ __forceinline__ bool rel(const BwdParams& p, const Item& it, int i) {
+  if (i < it.lo || i > it.hi) return false;
+  if (!p.seg) return true;
+  const size_t qi = (size_t)it.b * p.n_tiles + i;
+  return meet(it.kmin, it.kmax, p.tmin[qi], p.tmax[qi]);
+}
+
+__device__ __forceinline__ int next_rel(const BwdParams& p, const Item& it, int i) {
+  for (++i; i <= it.hi; ++i)
+    if (rel(p, it, i)) return i;
+  return -1;
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return;
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t bar0 = base + OFF_BAR;
+  auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  const Abort ab{abort_flag, p.status};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = p.B * p.H * p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(B_KV_FULL), 1);
+    mbar_init(bar(B_KV_EMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_QD_FULL + s), 1);
+      mbar_init(bar(B_QD_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_S_FULL), 1);
+    mbar_init(bar(B_DP_FULL), 1);
+    mbar_init(bar(B_P_FULL), 256);
+    mbar_init(bar(B_DS_FULL), 256);
+    mbar_init(bar(B_DQ_FULL), 1);
+    mbar_init(bar(B_DRAIN), 256);
+    mbar_init(bar(B_DKV_FULL), 1);
+    mbar_init(bar(B_DKV_EMPTY), 256);
+    mbar_init(bar(B_FIN), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  uint32_t q_issued = 0, kv_issued = 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      uint32_t q_it = 0;
+      int items = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+        const Item it = decode(p, idx);
+        if (items > 0 && !mbar_wait(bar(B_KV_EMPTY), (items - 1) & 1, ab, 21)) { ok = false; break; }
+        mbar_expect_tx(bar(B_KV_FULL), 2 * kTileBytes);
+        tma_load_4d(base + OFF_K, &tm_k, bar(B_KV_FULL), 0, it.h, it.j * 128, it.b);
+        tma_load_4d(base + OFF_K + kBoxBytes, &tm_k, bar(B_KV_FULL), 64, it.h, it.j * 128, it.b);
+        tma_load_4d(base + OFF_V, &tm_v, bar(B_KV_FULL), 0, it.h, it.j * 128, it.b);
+        tma_load_4d(base + OFF_V + kBoxBytes, &tm_v, bar(B_KV_FULL), 64, it.h, it.j * 128, it.b);
+        kv_issued = items + 1;
+        int i = rel(p, it, it.lo) ? it.lo : next_rel(p, it, it.lo);
+        while (i >= 0) {
+          const uint32_t s = q_it & 1;
+          if (!mbar_wait(bar(B_QD_EMPTY + s), ((q_it >> 1) & 1) ^ 1, ab, 22)) { ok = false; break; }
+          mbar_expect_tx(bar(B_QD_FULL + s), 2 * kTileBytes);
+          const uint32_t dq = base + OFF_Q + s * kTileBytes, dd = base + OFF_DO + s * kTileBytes;
+          tma_load_4d(dq, &tm_q, bar(B_QD_FULL + s), 0, it.h, i * 128, it.b);
+          tma_load_4d(dq + kBoxBytes, &tm_q, bar(B_QD_FULL + s), 64, it.h, i * 128, it.b);
+          tma_load_4d(dd, &tm_do, bar(B_QD_FULL + s), 0, it.h, i * 128, it.b);
+          tma_load_4d(dd + kBoxBytes, &tm_do, bar(B_QD_FULL + s), 64, it.h, i * 128, it.b);
+          ++q_it;
+          q_issued = q_it;
+          i = next_rel(p, it, i);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);   // K-major x K-major
+      constexpr uint32_t kIdKM = idesc_bf16(128, 128, 0, 1);   // K-major (or TMEM) x MN-major
+      constexpr uint32_t kIdMM = idesc_bf16(128, 128, 1, 1);   // MN-major x MN-major
+      const uint32_t sK = base + OFF_K, sV = base + OFF_V, sDS = base + OFF_DS;
+      const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+      uint32_t q_it = 0, steps = 0, dkv = 0;
+      int items = 0;
+      bool ok = true;
+      // A, B both K-major SW128 128x128 tiles: k-step kk walks 32 bytes inside a
+      // 128-byte row, then jumps to the second 64-column box.
+      auto kdesc = [](uint32_t t, int kk) {
+        return smem_desc_sw128(t + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+      };
+      // MN-major SW128 tile (rows = K, 64-wide boxes along MN): k-step = 16 rows.
+      auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+        const Item it = decode(p, idx);
+        if (!mbar_wait(bar(B_KV_FULL), items & 1, ab, 23)) { ok = false; break; }
+        tc_fence_after();
+        int i = rel(p, it, it.lo) ? it.lo : next_rel(p, it, it.lo);
+        bool first = true;
+        auto issue_s = [&]() {
+          const uint32_t sq = base + OFF_Q + (q_it & 1) * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) mma_ss(tS, kdesc(sK, kk), kdesc(sq, kk), kIdKK, kk > 0);
+          mma_commit(bar(B_S_FULL));
+        };
+        if (i >= 0) {
+          if (!mbar_wait(bar(B_QD_FULL + (q_it & 1)), (q_it >> 1) & 1, ab, 24)) { ok = false; break; }
+          tc_fence_after();
+          issue_s();
+        }
+        while (i >= 0) {
+          const uint32_t sq = base + OFF_Q + (q_it & 1) * kTileBytes;
+          const uint32_t sdo = base + OFF_DO + (q_it & 1) * kTileBytes;
+          if (steps > 0 && !mbar_wait(bar(B_DRAIN), (steps - 1) & 1, ab, 25)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, kdesc(sV, kk), kdesc(sdo, kk), kIdKK, kk > 0);
+          mma_commit(bar(B_DP_FULL));
+          if (first && dkv > 0 && !mbar_wait(bar(B_DKV_EMPTY), (dkv - 1) & 1, ab, 26)) { ok = false; break; }
+          if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 27)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tDV, tS + kk * 8, mdesc(sdo, kk), kIdKM, (kk > 0 || !first) ? 1u : 0u);
+          if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 28)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDK, kdesc(sDS, kk), mdesc(sq, kk), kIdKM, (kk > 0 || !first) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, mdesc(sDS, kk), mdesc(sK, kk), kIdMM, kk > 0);
+          mma_commit(bar(B_DQ_FULL));
+          mma_commit(bar(B_QD_EMPTY + (q_it & 1)));
+          ++q_it;
+          ++steps;
+          first = false;
+          i = next_rel(p, it, i);
+          if (i >= 0) {
+            if (!mbar_wait(bar(B_QD_FULL + (q_it & 1)), (q_it >> 1) & 1, ab, 29)) { ok = false; break; }
+            tc_fence_after();
+            issue_s();
+          }
+        }
+        if (!ok) break;
+        if (!first) {
+          mma_commit(bar(B_DKV_FULL));
+          ++dkv;
+        }
+        mma_commit(bar(B_KV_EMPTY));
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------- element-wise work
+    const int w = (warp - 4) >> 2;                // column half
+    const int row = ((warp & 3) << 5) + lane;     // TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tDP = tmem + lane_base + 128u;
+    const uint32_t tDV = tmem + lane_base + 256u;
+    const uint32_t tDK = tmem + lane_base + 384u;
+    const uint32_t sDS = base + OFF_DS + (uint32_t)w * kBoxBytes + (uint32_t)(row >> 3) * 1024u +
+                         (uint32_t)(row & 7) * 128u;
+    uint32_t steps = 0, dkv = 0;
+    bool ok = true;
+    const size_t hstride = (size_t)p.n_tiles * 128;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const Item it = decode(p, idx);
+      const int64_t key = (int64_t)it.j * 128 + row;
+      const bool key_ok = key < p.S;
+      const int32_t seg_k = key_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + key] : 0) : -1;
+      const float* lse2 = p.lse2 + ((size_t)it.b * p.H + it.h) * hstride;
+      const float* dpad = p.dpad + ((size_t)it.b * p.H + it.h) * hstride;
+      int n = 0;
+      for (int i = it.lo; i <= it.hi; ++i) {
+        if (!rel(p, it, i)) continue;
+        const int64_t q0 = (int64_t)i * 128 + 64 * w;  // first query column of this half
+        bool partial = (p.causal && i == it.j) || ((int64_t)(i + 1) * 128 > p.S) ||
+                       ((int64_t)(it.j + 1) * 128 > p.S);
+        if (p.seg) {
+          const size_t qi = (size_t)it.b * p.n_tiles + i;
+          const int32_t a0 = p.tmin[qi], a1 = p.tmax[qi];
+          partial |= !(it.kmin >= 0 && it.kmin == it.kmax && a0 == it.kmin && a1 == it.kmin);
+        }
+        uint32_t mw0 = 0xffffffffu, mw1 = 0xffffffffu;
+        if (partial) {
+          // keep query q = q0 + c iff q < S, same segment, and q >= key when causal
+          int lo = 0;
+          if (p.causal) {
+            const int64_t d = key - q0;
+            lo = d < 0 ? 0 : (d > 64 ? 64 : (int)d);
+          }
+          const int64_t qv = p.S - q0;
+          const int hi = qv > 64 ? 64 : (int)qv;  // exclusive
+          const int32_t* qs = p.seg ? p.seg + (size_t)it.b * p.S + q0 : nullptr;
+          uint32_t m[2] = {0, 0};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t bits = 0;
+#pragma unroll 4
+            for (int c = 0; c < 32; ++c) {
+              const int cc = h2 * 32 + c;
+              const bool keep = seg_k >= 0 && cc >= lo && cc < hi &&
+                                (qs == nullptr || __ldg(qs + cc) == seg_k);
+              bits |= (uint32_t)keep << c;
+            }
+            m[h2] = bits;
+          }
+          mw0 = m[0];
+          mw1 = m[1];
+        }
+        // ---- P^T = exp2(S^T * scale*log2e - LSE2[q]) ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 30 + w))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(tS + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tS + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        float pr[64];
+        const float4* l4 = reinterpret_cast<const float4*>(lse2 + q0);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float4 L = __ldg(l4 + u);
+          const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * u + e;
+            const uint32_t mword = c < 32 ? mw0 : mw1;
+            const bool keep = (mword >> (c & 31)) & 1u;
+            pr[c] = keep ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -Ls[e])) : 0.f;
+          }
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
+          tmem_st32(tS + 32 * w, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_P_FULL));
+        // ---- dS^T = P^T o (dP^T - D[q]) -> shared memory ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 32 + w))) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        const float4* d4 = reinterpret_cast<const float4*>(dpad + q0);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float4 Dv = __ldg(d4 + u);
+          const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * u + e;
+            pr[c] = pr[c] * (__uint_as_float(r[c]) - Ds[e]);
+          }
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          const int c = c16 * 8;
+          st_shared_v4(sDS + (uint32_t)((c16 ^ (row & 7)) << 4), pack_bf16(pr[c], pr[c + 1]),
+                       pack_bf16(pr[c + 2], pr[c + 3]), pack_bf16(pr[c + 4], pr[c + 5]),
+                       pack_bf16(pr[c + 6], pr[c + 7]));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_DS_FULL));
+        // ---- drain dQ partial (row = query) into the fp32 accumulator ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), steps & 1, ab, 34 + w))) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_DRAIN));
+        const int64_t q = (int64_t)i * 128 + row;
+        if (q < p.S) {
+          float* dst = p.dq_acc + (((size_t)it.b * p.S + q) * p.H + it.h) * kD + 64 * w;
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            red_add_v4(dst + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                       __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+        }
+        ++steps;
+        ++n;
+      }
+      if (!ok) break;
+      // ---- dK, dV epilogue for this key tile ----
+      __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
+      __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
+      if (n == 0) {
+        if (key_ok) {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            reinterpret_cast<uint4*>(dkrow)[c] = z;
+            reinterpret_cast<uint4*>(dvrow)[c] = z;
+          }
+        }
+        continue;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DKV_FULL), dkv & 1, ab, 36 + w))) { ok = false; break; }
+      ++dkv;
+      tc_fence_after();
+      uint32_t r[64];
+      tmem_ld32(tDK + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(tDK + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_wait_ld();
+      uint32_t out[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
+        if (p.rotate) {
+          float c, s;
+          rope_cos_sin_w(key, rope_freq(32 * w + u, kD, p.log2_theta), &c, &s);
+          const float a2 = a * c + b * s, b2 = b * c - a * s;
+          a = a2;
+          b = b2;
+        }
+        out[u] = pack_bf16(a, b);
+      }
+      if (key_ok) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          reinterpret_cast<uint4*>(dkrow)[c] =
+              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+      }
+      tmem_ld32(tDV + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(tDV + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_DKV_EMPTY));
+      if (key_ok) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          reinterpret_cast<uint4*>(dvrow)[c] = make_uint4(
+              pack_bf16(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+              pack_bf16(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+              pack_bf16(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+              pack_bf16(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 1 && lane == 0) {
+      mma_commit(bar(B_FIN));
+      drain_wait(bar(B_FIN), 0);
+    }
+    if (warp == 0 && lane == 0) {
+      if (kv_issued > 0) drain_wait(bar(B_KV_FULL), (kv_issued - 1) & 1);
+      for (uint32_t n = (q_issued > 2 ? q_issued - 2 : 0); n < q_issued; ++n)
+        drain_wait(bar(B_QD_FULL + (n & 1)), (n >> 1) & 1);
+    }
+  }
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sm100_bwd(const Problem& pb, const Workspace& ws, const void* v,
+                             const void* d_o, void* dk, void* dv, cudaStream_t st) {
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
+    return cudaErrorInvalidValue;
+  BwdParams p{};
+  p.seg = pb.seg;
+  p.tmin = ws.tile_min;
+  p.tmax = ws.tile_max;
+  p.k_hi = ws.k_hi;
+  p.lse2 = ws.lse2_pad;
+  p.dpad = ws.delta_pad;
+  p.dq_acc = ws.dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = ws.status;
+  p.S = pb.S;
+  p.H = (int)pb.H;
+  p.B = (int)pb.B;
+  p.n_tiles = (int)pb.n_tiles;
+  p.scale = pb.scale;
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.causal = pb.causal;
+  p.rotate = pb.theta > 0.0;
+  p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
+  const int64_t n_items = pb.B * pb.H * pb.n_tiles;
+  if (n_items == 0) return cudaSuccess;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
+  attn_bwd_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace lwm
