@@ -148,8 +148,11 @@ def _check(status: int, what: str):
 
 
 def lwm_attn_fwd(q, k, v, segment_ids=None, causal=True, rope_theta=1e4, softmax_scale=0.0,
-                 o=None, lse=None, workspace=None, stream=None):
-    """O [B,S,H,D] and LSE [B,H,S] fp32 for un-rotated q, k, v (see lwm_attn.h)."""
+                 o=None, lse=None, workspace=None, stream=None, check_status=False):
+    """O [B,S,H,D] and LSE [B,H,S] fp32 for un-rotated q, k, v (see lwm_attn.h).
+
+    check_status: wait for the stream and raise if a kernel reported a
+    device-side error (a bounded wait that ran out) in the status word."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         _cuda(t, name)
         if t.shape != q.shape or t.dtype != q.dtype:
@@ -166,11 +169,14 @@ def lwm_attn_fwd(q, k, v, segment_ids=None, causal=True, rope_theta=1e4, softmax
                            o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
                            workspace.numel(), _stream(stream))
     _check(st, "lwm_attn_fwd")
+    if check_status:
+        _check(lwm_attn_read_status(workspace, stream), "lwm_attn_fwd (device status)")
     return o, lse
 
 
 def lwm_attn_bwd(q, k, v, o, lse, d_o, segment_ids=None, causal=True, rope_theta=1e4,
-                 softmax_scale=0.0, dq=None, dk=None, dv=None, workspace=None, stream=None):
+                 softmax_scale=0.0, dq=None, dk=None, dv=None, workspace=None, stream=None,
+                 check_status=False):
     """dq, dk, dv (gradients w.r.t. the un-rotated inputs) of sum(O * dO)."""
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("d_o", d_o)):
         _cuda(t, name)
@@ -188,6 +194,8 @@ def lwm_attn_bwd(q, k, v, o, lse, d_o, segment_ids=None, causal=True, rope_theta
                            dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
                            _stream(stream))
     _check(st, "lwm_attn_bwd")
+    if check_status:
+        _check(lwm_attn_read_status(workspace, stream), "lwm_attn_bwd (device status)")
     return dq, dk, dv
 
 

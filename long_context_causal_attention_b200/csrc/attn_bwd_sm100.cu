@@ -21,7 +21,9 @@
 //               columns 64-127: P^T into TMEM (bf16, over S^T), dS^T into
 //               shared memory (bf16, 128-byte swizzle), the dQ drain, and
 //               the dK/dV epilogue (scale, inverse RoPE, bf16).
-// TMEM columns: S^T/P^T [0,128), dP^T then dQ [128,256), dV [256,384),
+// TMEM columns: S^T [0,128) with P^T over it (queries 0-63 packed into
+// columns 0-31, queries 64-127 into 64-95, so each warpgroup overwrites only
+// S^T columns it read itself), dP^T then dQ [128,256), dV [256,384),
 // dK [384,512).  MMA issue order per step:
 //   S(i) | dP(i) after drain(i-1) | dV(i) after P(i) | dK(i) dQ(i) after dS(i) | S(i+1)
 #include <cuda.h>
@@ -274,8 +276,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 27)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDV, tS + kk * 8, mdesc(sdo, kk), kIdKM, (kk > 0 || !first) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)  // P^T: queries 0-63 at cols 0-31, 64-127 at 64-95
+            mma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, mdesc(sdo, kk), kIdKM,
+                   (kk > 0 || !first) ? 1u : 0u);
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 28)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -365,29 +368,34 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---- P^T = exp2(S^T * scale*log2e - LSE2[q]) ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 30 + w))) { ok = false; break; }
         tc_fence_after();
-        uint32_t r[64];
-        tmem_ld32(tS + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tS + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_wait_ld();
         float pr[64];
-        const float4* l4 = reinterpret_cast<const float4*>(lse2 + q0);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float4 L = __ldg(l4 + u);
-          const float Ls[4] = {L.x, L.y, L.z, L.w};
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[32];
+          tmem_ld32(tS + 64 * w + 32 * h2, r);
+          tmem_wait_ld();
+          const uint32_t mword = h2 == 0 ? mw0 : mw1;
+          const float4* l4 = reinterpret_cast<const float4*>(lse2 + q0 + 32 * h2);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * u + e;
-            const uint32_t mword = c < 32 ? mw0 : mw1;
-            const bool keep = (mword >> (c & 31)) & 1u;
-            pr[c] = keep ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -Ls[e])) : 0.f;
+          for (int u = 0; u < 8; ++u) {
+            const float4 L = __ldg(l4 + u);
+            const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * u + e;
+              const bool keep = (mword >> c) & 1u;
+              pr[32 * h2 + c] =
+                  keep ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -Ls[e])) : 0.f;
+            }
           }
         }
         {
           uint32_t pk[32];
 #pragma unroll
           for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
-          tmem_st32(tS + 32 * w, pk);
+          // P^T for this half goes into the first 32 columns of the half's own
+          // S^T range, which no other warpgroup reads.
+          tmem_st32(tS + 64 * w, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -395,18 +403,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---- dS^T = P^T o (dP^T - D[q]) -> shared memory ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 32 + w))) { ok = false; break; }
         tc_fence_after();
-        tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_wait_ld();
-        const float4* d4 = reinterpret_cast<const float4*>(dpad + q0);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float4 Dv = __ldg(d4 + u);
-          const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[32];
+          tmem_ld32(tDP + 64 * w + 32 * h2, r);
+          tmem_wait_ld();
+          const float4* d4 = reinterpret_cast<const float4*>(dpad + q0 + 32 * h2);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * u + e;
-            pr[c] = pr[c] * (__uint_as_float(r[c]) - Ds[e]);
+          for (int u = 0; u < 8; ++u) {
+            const float4 Dv = __ldg(d4 + u);
+            const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 32 * h2 + 4 * u + e;
+              pr[c] = pr[c] * (__uint_as_float(r[4 * u + e]) - Ds[e]);
+            }
           }
         }
 #pragma unroll
@@ -422,18 +433,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---- drain dQ partial (row = query) into the fp32 accumulator ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), steps & 1, ab, 34 + w))) { ok = false; break; }
         tc_fence_after();
-        tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_DRAIN));
-        const int64_t q = (int64_t)i * 128 + row;
-        if (q < p.S) {
-          float* dst = p.dq_acc + (((size_t)it.b * p.S + q) * p.H + it.h) * kD + 64 * w;
+        {
+          const int64_t q = (int64_t)i * 128 + row;
+          float* dst = p.dq_acc + (((size_t)it.b * p.S + (q < p.S ? q : 0)) * p.H + it.h) * kD + 64 * w;
+          uint32_t r[64];
+          tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(B_DRAIN));
+          if (q < p.S) {
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
-            red_add_v4(dst + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                       __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+            for (int u = 0; u < 16; ++u)
+              red_add_v4(dst + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                         __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+          }
         }
         ++steps;
         ++n;
@@ -466,7 +480,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
         if (p.rotate) {
           float c, s;
-          rope_cos_sin_w(key, rope_freq(32 * w + u, kD, p.log2_theta), &c, &s);
+          rope_cos_sin_fast(key, rope_freq(32 * w + u, kD, p.log2_theta), &c, &s);
           const float a2 = a * c + b * s, b2 = b * c - a * s;
           a = a2;
           b = b2;

@@ -64,6 +64,17 @@ __device__ __forceinline__ void rope_cos_sin_w(int64_t pos, double w, float* c, 
   sincosf((float)r, s, c);
 }
 
+// Same angle, cos/sin from the fast hardware approximation.  The argument is
+// already reduced to [-pi, pi], where its absolute error is below 1e-6; used
+// where the result is rounded to bf16 right after (relative 2^-9).
+__device__ __forceinline__ void rope_cos_sin_fast(int64_t pos, double w, float* c, float* s) {
+  const double a = (double)pos * w;
+  const double k = rint(a * kInvTwoPi);
+  double r = fma(-k, kTwoPiHi, a);
+  r = fma(-k, kTwoPiLo, r);
+  __sincosf((float)r, s, c);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }

@@ -32,15 +32,16 @@ def run(lwm, t, seg, w: Workload, backward=True):
     dev = "cuda"
     seg_d = torch.as_tensor(seg, dtype=torch.int32, device=dev) if seg is not None else None
     o, lse = lwm.lwm_attn_fwd(t["q"], t["k"], t["v"], seg_d, causal=w.causal,
-                              rope_theta=w.theta, softmax_scale=w.scale)
+                              rope_theta=w.theta, softmax_scale=w.scale, check_status=True)
     out = {"o": o, "lse": lse}
     if backward:
         dq, dk, dv = lwm.lwm_attn_bwd(t["q"], t["k"], t["v"], o, lse, t["do"], seg_d,
                                       causal=w.causal, rope_theta=w.theta,
-                                      softmax_scale=w.scale)
+                                      softmax_scale=w.scale, check_status=True)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     return out
+
 
 
 def full_oracle(t, seg, w, backward=True):
