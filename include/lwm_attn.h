@@ -116,6 +116,34 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
                         const void* d_o, void* dq, void* dk, void* dv, void* ws,
                         size_t ws_bytes, void* stream);
 
+/* lwm_attn_fwd without a workspace argument: the forward pass takes its
+ * scratch memory (status word, per-tile segment bounds, rotated q and k)
+ * from a fixed 40 MiB device array inside the library instead of from the
+ * caller.  The pages have no counterpart; this is for callers that cannot
+ * call cudaMalloc where they run the forward pass, for example code running
+ * under an allocator or memory planner that forbids new device allocations
+ * after start-up, or a host that must not risk the implicit synchronisation
+ * or out-of-memory failure an allocation can bring at that point.  The
+ * caller still passes q, k, v, o and lse (same meaning as lwm_attn_fwd).
+ *   - Scratch limit: 40 MiB, enough for about 10M bf16 elements per tensor
+ *     (e.g. 2,048 tokens x 32 heads x 128).  A problem whose workspace
+ *     (lwm_attn_workspace_size(desc, 0)) is larger returns
+ *     LWM_ERR_WORKSPACE and launches nothing.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *     Every GPU that loads the library holds the 40 MiB array until exit.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.  A failed lookup returns
+ *     LWM_ERR_CUDA.
+ *   - Sharing: all calls on a device share the one array, which keeps the
+ *     last call's contents (the call clears what must start at zero).  Calls
+ *     that overlap on the GPU (different streams, or host threads) race on
+ *     it; serialise them.
+ *   - lwm_attn_read_status reads nothing for this entry point (there is no
+ *     caller workspace); device-side errors stay in the library's array. */
+lwm_status lwm_attn_fwd_noalloc(const lwm_attn_desc* desc, const void* q, const void* k,
+                                const void* v, void* o, float* lse, void* stream);
+
 /* y = R(p) x (inverse = 0) or R(p)^T x (inverse != 0) for x of [B,S,H,D]
  * (research note, "模型架构": standard RoPE; theta per "训练方法").  Angles
  * p*w_t are formed and reduced modulo 2*pi in fp64, cos/sin taken in fp32,

@@ -28,7 +28,7 @@ STATUS_NAMES = {
 
 ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_rope_apply",
                 "lwm_attn_read_status", "lwm_status_string", "lwm_attn_set_timing_events",
-                "lwm_attn_kernel_launches")
+                "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc")
 
 
 class LwmAttnDesc(ctypes.Structure):
@@ -75,6 +75,8 @@ def _load():
     lib.lwm_status_string.restype = ctypes.c_char_p
     lib.lwm_attn_set_timing_events.argtypes = [P, P, P, P]
     lib.lwm_attn_set_timing_events.restype = None
+    lib.lwm_attn_fwd_noalloc.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P]
+    lib.lwm_attn_fwd_noalloc.restype = ctypes.c_int
     lib.lwm_attn_kernel_launches.argtypes = []
     lib.lwm_attn_kernel_launches.restype = ctypes.c_uint64
     return lib
