@@ -54,6 +54,8 @@ WORKLOADS = {
                           segments="packed_video_text"),
     "long_128k": Workload("long_128k", 1, 131072, 32, 128, "bf16", 1e7),
     "million_1m": Workload("million_1m", 1, 1048576, 32, 128, "bf16", 5e7),
+    # profiling case: same head shape, 16K tokens (each tensor 128 MiB, above L2)
+    "prof_16k": Workload("prof_16k", 1, 16384, 32, 128, "bf16", 1e6),
 }
 ORDER = ["tiny_packed_fp32", "fwd_32k", "packed_8k", "long_128k", "million_1m"]
 
