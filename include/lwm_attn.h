@@ -154,7 +154,9 @@ lwm_status lwm_rope_apply(int64_t batch, int64_t seqlen, int64_t heads,
                           const void* x, void* y, int inverse, void* stream);
 
 /* Waits for `stream`, then returns the status word the kernels of the last
- * call on `ws` left (LWM_OK or LWM_ERR_TIMEOUT), or LWM_ERR_CUDA. */
+ * call on `ws` left: LWM_OK, LWM_ERR_TIMEOUT (a bounded wait ran out) or
+ * LWM_ERR_UNSUPPORTED (a kernel could not lay out its shared memory); or
+ * LWM_ERR_CUDA if the read itself failed. */
 lwm_status lwm_attn_read_status(const void* ws, void* stream);
 
 /* Static, human-readable name of a status code. */

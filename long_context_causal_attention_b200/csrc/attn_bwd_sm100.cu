@@ -25,7 +25,11 @@
 // columns 0-31, queries 64-127 into 64-95, so each warpgroup overwrites only
 // S^T columns it read itself), dP^T then dQ [128,256), dV [256,384),
 // dK [384,512).  MMA issue order per step:
-//   S(i) | dP(i) after drain(i-1) | dV(i) after P(i) | dK(i) dQ(i) after dS(i) | S(i+1)
+//   dP(i) after drain(i-1) | dV(i) after P(i) | S(i+1) | dK(i) dQ(i) after dS(i)
+// and the element-wise warps run P(i+1), drain(i), dS(i+1), so the
+// exponentials of one step overlap the dK/dQ products of the previous one.
+// LSE*log2(e) and D for each query tile arrive in shared memory with the
+// Q/dO tiles (1-D bulk copies on the same barrier).
 #include <cuda.h>
 
 #include <mutex>
@@ -48,14 +52,20 @@ constexpr int kThreads = 384;
 constexpr uint32_t kTileBytes = 128 * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;
 
+// Small region at the start of dynamic shared memory (16-byte aligned):
+constexpr uint32_t SOFF_BAR = 0;                       // mbarriers
+constexpr uint32_t SOFF_MISC = 256;                    // TMEM base, abort flag
+constexpr uint32_t SOFF_LD = 320;                      // 2 stages x (LSE2[128], D[128]) fp32
+constexpr uint32_t kLdStageBytes = 2 * 128 * 4;
+constexpr uint32_t kSmallBytes = SOFF_LD + 2 * kLdStageBytes;
+// Tiles after it, from the next 1024-byte boundary (128-byte swizzle atoms):
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = OFF_K + kTileBytes;
 constexpr uint32_t OFF_Q = OFF_V + kTileBytes;       // 2 stages
 constexpr uint32_t OFF_DO = OFF_Q + 2 * kTileBytes;  // 2 stages
 constexpr uint32_t OFF_DS = OFF_DO + 2 * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_DS + kTileBytes;
-constexpr uint32_t OFF_MISC = OFF_BAR + 256;
-constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
+constexpr uint32_t kTilesBytes = OFF_DS + kTileBytes;  // 224 KB
+constexpr uint32_t kSmemBytes = 232448;                // the sm_100 per-block maximum
 
 enum : uint32_t {
   B_KV_FULL = 0, B_KV_EMPTY = 1,
@@ -153,14 +163,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t bar0 = base + OFF_BAR;
+  const uint32_t base = (raw + kSmallBytes + 1023u) & ~1023u;
+  if (base - raw + kTilesBytes > kSmemBytes) {
+    // the tiles would not fit after aligning (never seen: the dynamic shared
+    // memory window starts 1024-byte aligned); refuse instead of overrunning
+    if (threadIdx.x == 0) report_status(p.status, LWM_ERR_UNSUPPORTED, 99);
+    return;
+  }
+  const uint32_t bar0 = raw + SOFF_BAR;
   auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem_raw + SOFF_MISC);
+  const float* ld_smem = reinterpret_cast<const float*>(smem_raw + SOFF_LD);
   const Abort ab{abort_flag, p.status};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.B * p.H * p.n_tiles;
@@ -204,6 +220,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t q_it = 0;
       int items = 0;
       bool ok = true;
+      const size_t hstride = (size_t)p.n_tiles * 128;
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
         const Item it = decode(p, idx);
         if (items > 0 && !mbar_wait(bar(B_KV_EMPTY), (items - 1) & 1, ab, 21)) { ok = false; break; }
@@ -213,16 +230,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_4d(base + OFF_V, &tm_v, bar(B_KV_FULL), 0, it.h, it.j * 128, it.b);
         tma_load_4d(base + OFF_V + kBoxBytes, &tm_v, bar(B_KV_FULL), 64, it.h, it.j * 128, it.b);
         kv_issued = items + 1;
+        const float* lse2 = p.lse2 + ((size_t)it.b * p.H + it.h) * hstride;
+        const float* dpad = p.dpad + ((size_t)it.b * p.H + it.h) * hstride;
         int i = rel(p, it, it.lo) ? it.lo : next_rel(p, it, it.lo);
         while (i >= 0) {
           const uint32_t s = q_it & 1;
           if (!mbar_wait(bar(B_QD_EMPTY + s), ((q_it >> 1) & 1) ^ 1, ab, 22)) { ok = false; break; }
-          mbar_expect_tx(bar(B_QD_FULL + s), 2 * kTileBytes);
+          mbar_expect_tx(bar(B_QD_FULL + s), 2 * kTileBytes + kLdStageBytes);
           const uint32_t dq = base + OFF_Q + s * kTileBytes, dd = base + OFF_DO + s * kTileBytes;
           tma_load_4d(dq, &tm_q, bar(B_QD_FULL + s), 0, it.h, i * 128, it.b);
           tma_load_4d(dq + kBoxBytes, &tm_q, bar(B_QD_FULL + s), 64, it.h, i * 128, it.b);
           tma_load_4d(dd, &tm_do, bar(B_QD_FULL + s), 0, it.h, i * 128, it.b);
           tma_load_4d(dd + kBoxBytes, &tm_do, bar(B_QD_FULL + s), 64, it.h, i * 128, it.b);
+          const uint32_t ld = raw + SOFF_LD + s * kLdStageBytes;
+          bulk_load(ld, lse2 + (size_t)i * 128, 512, bar(B_QD_FULL + s));
+          bulk_load(ld + 512, dpad + (size_t)i * 128, 512, bar(B_QD_FULL + s));
           ++q_it;
           q_issued = q_it;
           i = next_rel(p, it, i);
@@ -247,43 +269,52 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
       // MN-major SW128 tile (rows = K, 64-wide boxes along MN): k-step = 16 rows.
       auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
+      auto sq_of = [&](uint32_t n) { return base + OFF_Q + (n & 1) * kTileBytes; };
+      auto sdo_of = [&](uint32_t n) { return base + OFF_DO + (n & 1) * kTileBytes; };
+      auto issue_s = [&](uint32_t n) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, kdesc(sK, kk), kdesc(sq_of(n), kk), kIdKK, kk > 0);
+        mma_commit(bar(B_S_FULL));
+      };
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
         const Item it = decode(p, idx);
         if (!mbar_wait(bar(B_KV_FULL), items & 1, ab, 23)) { ok = false; break; }
         tc_fence_after();
         int i = rel(p, it, it.lo) ? it.lo : next_rel(p, it, it.lo);
         bool first = true;
-        auto issue_s = [&]() {
-          const uint32_t sq = base + OFF_Q + (q_it & 1) * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ss(tS, kdesc(sK, kk), kdesc(sq, kk), kIdKK, kk > 0);
-          mma_commit(bar(B_S_FULL));
-        };
         if (i >= 0) {
           if (!mbar_wait(bar(B_QD_FULL + (q_it & 1)), (q_it >> 1) & 1, ab, 24)) { ok = false; break; }
           tc_fence_after();
-          issue_s();
+          issue_s(q_it);
         }
         while (i >= 0) {
-          const uint32_t sq = base + OFF_Q + (q_it & 1) * kTileBytes;
-          const uint32_t sdo = base + OFF_DO + (q_it & 1) * kTileBytes;
+          // dP^T(i) into the dQ columns once dQ(i-1) has been drained
           if (steps > 0 && !mbar_wait(bar(B_DRAIN), (steps - 1) & 1, ab, 25)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, kdesc(sV, kk), kdesc(sdo, kk), kIdKK, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDP, kdesc(sV, kk), kdesc(sdo_of(q_it), kk), kIdKK, kk > 0);
           mma_commit(bar(B_DP_FULL));
           if (first && dkv > 0 && !mbar_wait(bar(B_DKV_EMPTY), (dkv - 1) & 1, ab, 26)) { ok = false; break; }
           if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 27)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // P^T: queries 0-63 at cols 0-31, 64-127 at 64-95
-            mma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, mdesc(sdo, kk), kIdKM,
+            mma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, mdesc(sdo_of(q_it), kk), kIdKM,
                    (kk > 0 || !first) ? 1u : 0u);
+          // S^T(i+1) goes in now (dV(i) has taken P^T(i) from those columns, in
+          // issue order), so the next exponentials overlap dK(i) and dQ(i)
+          const int inext = next_rel(p, it, i);
+          if (inext >= 0) {
+            if (!mbar_wait(bar(B_QD_FULL + ((q_it + 1) & 1)), ((q_it + 1) >> 1) & 1, ab, 29)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(q_it + 1);
+          }
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 28)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDK, kdesc(sDS, kk), mdesc(sq, kk), kIdKM, (kk > 0 || !first) ? 1u : 0u);
+            mma_ss(tDK, kdesc(sDS, kk), mdesc(sq_of(q_it), kk), kIdKM, (kk > 0 || !first) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, mdesc(sDS, kk), mdesc(sK, kk), kIdMM, kk > 0);
           mma_commit(bar(B_DQ_FULL));
@@ -291,12 +322,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           ++q_it;
           ++steps;
           first = false;
-          i = next_rel(p, it, i);
-          if (i >= 0) {
-            if (!mbar_wait(bar(B_QD_FULL + (q_it & 1)), (q_it >> 1) & 1, ab, 29)) { ok = false; break; }
-            tc_fence_after();
-            issue_s();
-          }
+          i = inext;
         }
         if (!ok) break;
         if (!first) {
@@ -319,15 +345,42 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                          (uint32_t)(row & 7) * 128u;
     uint32_t steps = 0, dkv = 0;
     bool ok = true;
-    const size_t hstride = (size_t)p.n_tiles * 128;
+
+    // dQ partial of step `s` (query tile i; TMEM lane = query) -> fp32 accumulator
+    auto drain = [&](const Item& it, int i, uint32_t s) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), s & 1, ab, 34 + w))) return false;
+      tc_fence_after();
+      const int64_t q = (int64_t)i * 128 + row;
+      float* dst = p.dq_acc + (((size_t)it.b * p.S + (q < p.S ? q : 0)) * p.H + it.h) * kD + 64 * w;
+      // two 32-column chunks; the columns are free for dP(i+1) once both are in registers
+      uint32_t r[32];
+      tmem_ld32(tDP + 64 * w, r);
+      tmem_wait_ld();
+      if (q < p.S) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          red_add_v4(dst + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                     __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+      }
+      tmem_ld32(tDP + 64 * w + 32, r);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_DRAIN));
+      if (q < p.S) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          red_add_v4(dst + 32 + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                     __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+      }
+      return true;
+    };
+
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
       const Item it = decode(p, idx);
       const int64_t key = (int64_t)it.j * 128 + row;
       const bool key_ok = key < p.S;
       const int32_t seg_k = key_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + key] : 0) : -1;
-      const float* lse2 = p.lse2 + ((size_t)it.b * p.H + it.h) * hstride;
-      const float* dpad = p.dpad + ((size_t)it.b * p.H + it.h) * hstride;
-      int n = 0;
+      int n = 0, pend = -1;  // pend: query tile whose dQ partial is not drained yet
       for (int i = it.lo; i <= it.hi; ++i) {
         if (!rel(p, it, i)) continue;
         const int64_t q0 = (int64_t)i * 128 + 64 * w;  // first query column of this half
@@ -365,8 +418,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mw0 = m[0];
           mw1 = m[1];
         }
+        const uint32_t stage = steps & 1;
+        const float* lse2 = ld_smem + stage * (kLdStageBytes / 4) + 64 * w;
+        const float* dsum = lse2 + 128;
         // ---- P^T = exp2(S^T * scale*log2e - LSE2[q]) ----
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 30 + w))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 30 + w) &&
+                                         mbar_wait(bar(B_QD_FULL + stage), (steps >> 1) & 1, ab, 38 + w))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         float pr[64];
 #pragma unroll
@@ -375,10 +435,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_ld32(tS + 64 * w + 32 * h2, r);
           tmem_wait_ld();
           const uint32_t mword = h2 == 0 ? mw0 : mw1;
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + q0 + 32 * h2);
+          const float4* l4 = reinterpret_cast<const float4*>(lse2 + 32 * h2);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float4 L = __ldg(l4 + u);
+            const float4 L = l4[u];
             const float Ls[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -400,6 +460,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL));
+        // ---- the previous step's dQ partial, while dK/dQ of this one run ----
+        if (pend >= 0) {
+          if (!drain(it, pend, steps - 1)) { ok = false; break; }
+          pend = -1;
+        }
         // ---- dS^T = P^T o (dP^T - D[q]) -> shared memory ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 32 + w))) { ok = false; break; }
         tc_fence_after();
@@ -408,10 +473,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           uint32_t r[32];
           tmem_ld32(tDP + 64 * w + 32 * h2, r);
           tmem_wait_ld();
-          const float4* d4 = reinterpret_cast<const float4*>(dpad + q0 + 32 * h2);
+          const float4* d4 = reinterpret_cast<const float4*>(dsum + 32 * h2);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float4 Dv = __ldg(d4 + u);
+            const float4 Dv = d4[u];
             const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -430,29 +495,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_DS_FULL));
-        // ---- drain dQ partial (row = query) into the fp32 accumulator ----
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), steps & 1, ab, 34 + w))) { ok = false; break; }
-        tc_fence_after();
-        {
-          const int64_t q = (int64_t)i * 128 + row;
-          float* dst = p.dq_acc + (((size_t)it.b * p.S + (q < p.S ? q : 0)) * p.H + it.h) * kD + 64 * w;
-          uint32_t r[64];
-          tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar(B_DRAIN));
-          if (q < p.S) {
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-              red_add_v4(dst + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                         __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
-          }
-        }
+        pend = i;
         ++steps;
         ++n;
       }
       if (!ok) break;
+      if (pend >= 0 && !drain(it, pend, steps - 1)) { ok = false; break; }
       // ---- dK, dV epilogue for this key tile ----
       __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
       __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;

@@ -20,6 +20,14 @@ struct DeviceStatus {
 };
 static_assert(sizeof(DeviceStatus) == 256, "status block is 256 bytes");
 
+__device__ __forceinline__ void report_status(DeviceStatus* st, lwm_status code, int where) {
+  if (st) {
+    atomicCAS(&st->code, 0, (int)code);
+    st->where = where;
+    st->block = (int)blockIdx.x;
+  }
+}
+
 __device__ __forceinline__ void report_timeout(DeviceStatus* st, int where) {
   if (st) {
     atomicCAS(&st->code, 0, (int)LWM_ERR_TIMEOUT);
