@@ -12,11 +12,12 @@
 // One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
 // walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
 // tensor memory for the whole walk, dQ partials are added into an fp32
-// buffer with vector reductions.  Roles (384 threads):
+// buffer with TMA bulk reductions.  Roles (384 threads):
 //   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i per step
 //               through a 2-stage ring.
 //   warp 1      MMA issuer (one thread).
 //   warp 2      tensor-memory allocation.
+//   warp 3      dQ reduce issuer (one thread).
 //   warps 4-7   element-wise work on query columns 0-63, warps 8-11 on
 //               columns 64-127: P^T into TMEM (bf16, over S^T), dS^T into
 //               shared memory (bf16, 128-byte swizzle), the dQ drain, and
@@ -41,6 +42,7 @@
 namespace lwm {
 
 bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
+bool make_f32_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
 int sm_count();
 
 namespace {
@@ -72,7 +74,7 @@ enum : uint32_t {
   B_QD_FULL = 2,   // 2 stages
   B_QD_EMPTY = 4,  // 2 stages
   B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_DS_FULL = 9, B_DQ_FULL = 10, B_DRAIN = 11,
-  B_DKV_FULL = 12, B_DKV_EMPTY = 13, B_FIN = 14
+  B_DKV_FULL = 12, B_DKV_EMPTY = 13, B_FIN = 14, B_STAGED = 15
 };
 
 struct BwdParams {
@@ -146,12 +148,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -162,7 +158,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + kSmallBytes + 1023u) & ~1023u;
@@ -187,7 +183,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(bar(B_KV_EMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_QD_FULL + s), 1);
-      mbar_init(bar(B_QD_EMPTY + s), 1);
+      mbar_init(bar(B_QD_EMPTY + s), 1);  // arrived by the dQ reduce issuer
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_DP_FULL), 1);
@@ -198,11 +194,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(bar(B_DKV_FULL), 1);
     mbar_init(bar(B_DKV_EMPTY), 256);
     mbar_init(bar(B_FIN), 1);
+    mbar_init(bar(B_STAGED), 256);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -318,7 +316,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, mdesc(sDS, kk), mdesc(sK, kk), kIdMM, kk > 0);
           mma_commit(bar(B_DQ_FULL));
-          mma_commit(bar(B_QD_EMPTY + (q_it & 1)));
           ++q_it;
           ++steps;
           first = false;
@@ -331,6 +328,34 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mma_commit(bar(B_KV_EMPTY));
       }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------ dQ reduce issuer
+    // Each step's dQ partial is staged (fp32, 128-byte swizzle) in that step's
+    // own Q~/dO stage buffers, which its MMAs no longer need; this thread adds
+    // it into the fp32 accumulator with four 32-column TMA reductions and hands
+    // the stage back to the producer once the reductions have read it.
+    if (lane == 0) {
+      uint32_t steps = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const Item it = decode(p, idx);
+        for (int i = it.lo; i <= it.hi && ok; ++i) {
+          if (!rel(p, it, i)) continue;
+          const uint32_t s = steps & 1;
+          if (!mbar_wait(bar(B_STAGED), steps & 1, ab, 40)) { ok = false; break; }
+          const uint32_t bq = base + OFF_Q + s * kTileBytes, bd = base + OFF_DO + s * kTileBytes;
+          tma_reduce_add_4d(&tm_dq, bq, 0, it.h, i * 128, it.b);
+          tma_reduce_add_4d(&tm_dq, bq + kBoxBytes, 32, it.h, i * 128, it.b);
+          tma_reduce_add_4d(&tm_dq, bd, 64, it.h, i * 128, it.b);
+          tma_reduce_add_4d(&tm_dq, bd + kBoxBytes, 96, it.h, i * 128, it.b);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(bar(B_QD_EMPTY + s));
+          ++steps;
+        }
+      }
+      bulk_wait_all();  // the accumulator must hold every partial when the kernel ends
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- element-wise work
@@ -346,32 +371,30 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t steps = 0, dkv = 0;
     bool ok = true;
 
-    // dQ partial of step `s` (query tile i; TMEM lane = query) -> fp32 accumulator
-    auto drain = [&](const Item& it, int i, uint32_t s) -> bool {
+    // dQ partial of step `s` (query tile i; TMEM lane = query): TMEM -> registers
+    // -> the step's free stage buffer (this half's 64 columns = two 32-column
+    // fp32 boxes, 128-byte swizzle) for the reduce issuer.
+    auto drain = [&](uint32_t s) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), s & 1, ab, 34 + w))) return false;
       tc_fence_after();
-      const int64_t q = (int64_t)i * 128 + row;
-      float* dst = p.dq_acc + (((size_t)it.b * p.S + (q < p.S ? q : 0)) * p.H + it.h) * kD + 64 * w;
-      // two 32-column chunks; the columns are free for dP(i+1) once both are in registers
+      const uint32_t stage_buf = base + (w == 0 ? OFF_Q : OFF_DO) + (s & 1) * kTileBytes;
+      const uint32_t rbase = stage_buf + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
       uint32_t r[32];
-      tmem_ld32(tDP + 64 * w, r);
-      tmem_wait_ld();
-      if (q < p.S) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          red_add_v4(dst + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                     __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
-      }
-      tmem_ld32(tDP + 64 * w + 32, r);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_DRAIN));
-      if (q < p.S) {
+      for (int lb = 0; lb < 2; ++lb) {
+        tmem_ld32(tDP + 64 * w + 32 * lb, r);
+        tmem_wait_ld();
+        if (lb == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(B_DRAIN));  // the dQ columns may take dP(i+1) now
+        }
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          red_add_v4(dst + 32 + 4 * u, __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                     __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(rbase + (uint32_t)lb * kBoxBytes + (uint32_t)((c ^ (row & 7)) << 4),
+                       r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
       }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_STAGED));
       return true;
     };
 
@@ -462,7 +485,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_arrive(bar(B_P_FULL));
         // ---- the previous step's dQ partial, while dK/dQ of this one run ----
         if (pend >= 0) {
-          if (!drain(it, pend, steps - 1)) { ok = false; break; }
+          if (!drain(steps - 1)) { ok = false; break; }
           pend = -1;
         }
         // ---- dS^T = P^T o (dP^T - D[q]) -> shared memory ----
@@ -500,7 +523,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ++n;
       }
       if (!ok) break;
-      if (pend >= 0 && !drain(it, pend, steps - 1)) { ok = false; break; }
+      if (pend >= 0 && !drain(steps - 1)) { ok = false; break; }
       // ---- dK, dV epilogue for this key tile ----
       __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
       __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
@@ -583,11 +606,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 cudaError_t launch_sm100_bwd(const Problem& pb, const Workspace& ws, const void* v,
                              const void* d_o, void* dk, void* dv, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
+      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D) ||
+      !make_f32_map(&tdq, ws.dq_acc, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
   BwdParams p{};
   p.seg = pb.seg;
@@ -619,7 +643,7 @@ cudaError_t launch_sm100_bwd(const Problem& pb, const Workspace& ws, const void*
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
-  attn_bwd_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, p);
+  attn_bwd_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, tdq, p);
   note_launches(1);
   return cudaGetLastError();
 }
