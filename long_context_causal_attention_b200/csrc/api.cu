@@ -77,7 +77,6 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
       const size_t padded = (size_t)p.B * p.H * (size_t)p.n_tiles * kTile * sizeof(float);
       w.lse2_pad = static_cast<float*>(take(padded));
       w.delta_pad = static_cast<float*>(take(padded));
-      w.dq_acc = static_cast<float*>(take(nel * sizeof(float)));
     }
   }
   w.bytes = align_up(off, 1024);
@@ -196,16 +195,12 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
   cudaError_t e = prologue(p, w, q, k, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   if (choose_bwd_path(p) == Path::kSm100) {
-    const size_t nel = (size_t)p.B * p.S * p.H * p.D;
-    e = cudaMemsetAsync(w.dq_acc, 0, nel * sizeof(float), st);
-    if (e != cudaSuccess) return LWM_ERR_CUDA;
     e = launch_bwd_prep(p, o, d_o, lse, w, st);
     if (e != cudaSuccess) return LWM_ERR_CUDA;
     record_event(2, st);
-    e = launch_sm100_bwd(p, w, v, d_o, dk, dv, st);
+    e = launch_sm100_bwd_dkdv(p, w, v, d_o, dk, dv, st);
+    if (e == cudaSuccess) e = launch_sm100_bwd_dq(p, w, v, d_o, dq, st);
     record_event(3, st);
-    if (e != cudaSuccess) return LWM_ERR_CUDA;
-    e = launch_dq_post(p, w, dq, st);
     return cuda_status(e);
   }
   e = launch_delta(p, o, d_o, w.delta, st);

@@ -1,0 +1,475 @@
+// Backward attention, part 2 of 2: dQ, on the 5th-generation tensor cores
+// (sm_100a), bf16, D=128.
+//
+// Per (query tile i, key tile j), recomputing P from the saved LSE (the
+// FlashAttention recipe the paper card's references name):
+//   S  = Q~_i K~_j^T        P  = exp(S * scale - LSE_i)
+//   dP = dO_i V_j^T         dS = P o (dP - D_i),  D_i = dO_i . O_i
+//   dQ~_i += dS K~_j        dq_i = R(p)^T scale dQ~_i
+// One persistent CTA per SM owns a query tile i of one (b, h) and sweeps the
+// key tiles j it may attend to; dQ~_i accumulates in tensor memory, and the
+// epilogue applies the scale and the inverse rotation and writes bf16 dq, so
+// no partial sums leave the CTA.  Roles (384 threads):
+//   warp 0      TMA producer: Q~_i and dO_i once per item, K~_j and V_j per
+//               step through a 2-stage ring.
+//   warp 1      MMA issuer (one thread).
+//   warp 2      tensor-memory allocation.
+//   warps 4-7   element-wise work on key columns 0-63, warps 8-11 on 64-127
+//               (one query row per thread), then the dq epilogue.
+// TMEM columns: S [0,128), dP [128,256) with dS (bf16) over it, dQ~ [256,384).
+// MMA issue order per step:
+//   S(j+1) once S(j) is in registers | dQ(j) after dS(j) | dP(j+1) ...
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace lwm {
+
+bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
+int sm_count();
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = 128 * kD * 2;
+constexpr uint32_t kBoxBytes = kTileBytes / 2;
+
+constexpr uint32_t SOFF_BAR = 0;
+constexpr uint32_t SOFF_MISC = 256;
+constexpr uint32_t kSmallBytes = 320;
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_DO = OFF_Q + kTileBytes;
+constexpr uint32_t OFF_K = OFF_DO + kTileBytes;   // 2 stages
+constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;  // 2 stages
+constexpr uint32_t kTilesBytes = OFF_V + 2 * kTileBytes;  // 192 KB
+constexpr uint32_t kSmemBytes = kTilesBytes + kSmallBytes + 1024;
+
+enum : uint32_t {
+  B_Q_FULL = 0, B_Q_EMPTY = 1,
+  B_KV_FULL = 2,   // 2 stages
+  B_KV_EMPTY = 4,  // 2 stages
+  B_S_FULL = 6, B_S_READ = 7, B_DP_FULL = 8, B_DS_FULL = 9,
+  B_DQ_FULL = 10, B_DQ_EMPTY = 11, B_FIN = 12
+};
+
+struct DqParams {
+  const int32_t* seg;
+  const int32_t* tmin;
+  const int32_t* tmax;
+  const int32_t* q_lo;
+  const float* lse2;   // [B, H, nT*128]: LSE * log2(e), +inf where the row has no keys
+  const float* dpad;   // [B, H, nT*128]: dot(dO, O), 0 past the end
+  __nv_bfloat16* dq;
+  DeviceStatus* status;
+  int64_t S;
+  int H, B, n_tiles;
+  float scale, scale_log2;
+  int causal, rotate;
+  double log2_theta;
+};
+
+struct Item {
+  int b, h, i;
+  int lo, hi;          // key tile range
+  int32_t qmin, qmax;  // query tile id range
+};
+
+__device__ __forceinline__ bool meet(int32_t a0, int32_t a1, int32_t b0, int32_t b1) {
+  return a1 >= 0 && b1 >= 0 && a0 <= b1 && b0 <= a1;
+}
+
+__device__ __forceinline__ Item decode(const DqParams& p, int idx) {
+  Item it;
+  const int bh = idx / p.n_tiles;
+  it.i = p.n_tiles - 1 - (idx % p.n_tiles);  // most key tiles first (causal)
+  it.b = bh / p.H;
+  it.h = bh % p.H;
+  it.lo = 0;
+  it.hi = p.causal ? it.i : p.n_tiles - 1;
+  it.qmin = 0;
+  it.qmax = 0;
+  if (p.seg) {
+    const size_t qi = (size_t)it.b * p.n_tiles + it.i;
+    it.lo = p.q_lo[qi];
+    it.qmin = p.tmin[qi];
+    it.qmax = p.tmax[qi];
+  }
+  return it;
+}
+
+__device__ __forceinline__ bool rel(const DqParams& p, const Item& it, int j) {
+  if (j < it.lo || j > it.hi) return false;
+  if (!p.seg) return true;
+  const size_t kj = (size_t)it.b * p.n_tiles + j;
+  return meet(it.qmin, it.qmax, p.tmin[kj], p.tmax[kj]);
+}
+
+__device__ __forceinline__ int next_rel(const DqParams& p, const Item& it, int j) {
+  for (++j; j <= it.hi; ++j)
+    if (rel(p, it, j)) return j;
+  return -1;
+}
+
+__device__ __forceinline__ int first_rel(const DqParams& p, const Item& it) {
+  if (it.lo > it.hi) return -1;
+  return rel(p, it, it.lo) ? it.lo : next_rel(p, it, it.lo);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const DqParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + kSmallBytes + 1023u) & ~1023u;
+  const uint32_t bar0 = raw + SOFF_BAR;
+  auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem_raw + SOFF_MISC);
+  const Abort ab{abort_flag, p.status};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = p.B * p.H * p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(B_Q_FULL), 1);
+    mbar_init(bar(B_Q_EMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_KV_FULL + s), 1);
+      mbar_init(bar(B_KV_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_S_FULL), 1);
+    mbar_init(bar(B_S_READ), 256);
+    mbar_init(bar(B_DP_FULL), 1);
+    mbar_init(bar(B_DS_FULL), 256);
+    mbar_init(bar(B_DQ_FULL), 1);
+    mbar_init(bar(B_DQ_EMPTY), 256);
+    mbar_init(bar(B_FIN), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  uint32_t kv_issued = 0, q_issued = 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      uint32_t kv_it = 0;
+      int items = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+        const Item it = decode(p, idx);
+        if (items > 0 && !mbar_wait(bar(B_Q_EMPTY), (items - 1) & 1, ab, 51)) { ok = false; break; }
+        mbar_expect_tx(bar(B_Q_FULL), 2 * kTileBytes);
+        tma_load_4d(base + OFF_Q, &tm_q, bar(B_Q_FULL), 0, it.h, it.i * 128, it.b);
+        tma_load_4d(base + OFF_Q + kBoxBytes, &tm_q, bar(B_Q_FULL), 64, it.h, it.i * 128, it.b);
+        tma_load_4d(base + OFF_DO, &tm_do, bar(B_Q_FULL), 0, it.h, it.i * 128, it.b);
+        tma_load_4d(base + OFF_DO + kBoxBytes, &tm_do, bar(B_Q_FULL), 64, it.h, it.i * 128, it.b);
+        q_issued = items + 1;
+        for (int j = first_rel(p, it); j >= 0; j = next_rel(p, it, j)) {
+          const uint32_t s = kv_it & 1;
+          if (!mbar_wait(bar(B_KV_EMPTY + s), ((kv_it >> 1) & 1) ^ 1, ab, 52)) { ok = false; break; }
+          mbar_expect_tx(bar(B_KV_FULL + s), 2 * kTileBytes);
+          const uint32_t sk = base + OFF_K + s * kTileBytes, sv = base + OFF_V + s * kTileBytes;
+          tma_load_4d(sk, &tm_k, bar(B_KV_FULL + s), 0, it.h, j * 128, it.b);
+          tma_load_4d(sk + kBoxBytes, &tm_k, bar(B_KV_FULL + s), 64, it.h, j * 128, it.b);
+          tma_load_4d(sv, &tm_v, bar(B_KV_FULL + s), 0, it.h, j * 128, it.b);
+          tma_load_4d(sv + kBoxBytes, &tm_v, bar(B_KV_FULL + s), 64, it.h, j * 128, it.b);
+          ++kv_it;
+          kv_issued = kv_it;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);   // K-major x K-major
+      constexpr uint32_t kIdTM = idesc_bf16(128, 128, 0, 1);   // TMEM (K-major) x MN-major
+      const uint32_t sQ = base + OFF_Q, sDO = base + OFF_DO;
+      const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
+      uint32_t kv_it = 0, steps = 0, dqc = 0;
+      int items = 0;
+      bool ok = true;
+      auto kdesc = [](uint32_t t, int kk) {
+        return smem_desc_sw128(t + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+      };
+      auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
+      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 2) * 64 + (kk & 3) * 8; };
+      auto sk_of = [&](uint32_t n) { return base + OFF_K + (n & 1) * kTileBytes; };
+      auto sv_of = [&](uint32_t n) { return base + OFF_V + (n & 1) * kTileBytes; };
+      auto issue_s = [&](uint32_t n) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, kdesc(sQ, kk), kdesc(sk_of(n), kk), kIdKK, kk > 0);
+        mma_commit(bar(B_S_FULL));
+      };
+      auto issue_dp = [&](uint32_t n) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, kdesc(sDO, kk), kdesc(sv_of(n), kk), kIdKK, kk > 0);
+        mma_commit(bar(B_DP_FULL));
+      };
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+        const Item it = decode(p, idx);
+        if (!mbar_wait(bar(B_Q_FULL), items & 1, ab, 53)) { ok = false; break; }
+        tc_fence_after();
+        int j = first_rel(p, it);
+        bool first = true;
+        if (j >= 0) {
+          if (!mbar_wait(bar(B_KV_FULL + (kv_it & 1)), (kv_it >> 1) & 1, ab, 54)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(kv_it);
+          issue_dp(kv_it);
+        }
+        while (j >= 0) {
+          const int jn = next_rel(p, it, j);
+          // S(j+1) as soon as S(j) is in the element-wise warps' registers
+          if (!mbar_wait(bar(B_S_READ), steps & 1, ab, 55)) { ok = false; break; }
+          if (jn >= 0) {
+            if (!mbar_wait(bar(B_KV_FULL + ((kv_it + 1) & 1)), ((kv_it + 1) >> 1) & 1, ab, 56)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(kv_it + 1);
+          }
+          if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 57)) { ok = false; break; }
+          if (first && dqc > 0 && !mbar_wait(bar(B_DQ_EMPTY), (dqc - 1) & 1, ab, 58)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tDQ, tcol(tDP, kk), mdesc(sk_of(kv_it), kk), kIdTM, (kk > 0 || !first) ? 1u : 0u);
+          mma_commit(bar(B_KV_EMPTY + (kv_it & 1)));
+          ++kv_it;
+          // dP(j+1): dS(j) in these columns went to dQ(j) just before (issue order)
+          if (jn >= 0) issue_dp(kv_it);
+          ++steps;
+          first = false;
+          j = jn;
+        }
+        if (!ok) break;
+        if (!first) {
+          mma_commit(bar(B_DQ_FULL));
+          ++dqc;
+        }
+        mma_commit(bar(B_Q_EMPTY));
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------- element-wise work
+    const int w = (warp - 4) >> 2;                // key column half
+    const int row = ((warp & 3) << 5) + lane;     // TMEM lane = query in the tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tDP = tmem + lane_base + 128u;
+    const uint32_t tDQ = tmem + lane_base + 256u;
+    const size_t hstride = (size_t)p.n_tiles * 128;
+    uint32_t steps = 0, dqc = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const Item it = decode(p, idx);
+      const int64_t q = (int64_t)it.i * 128 + row;
+      const bool q_ok = q < p.S;
+      const int32_t seg_q = q_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + q] : 0) : -1;
+      const size_t lrow = ((size_t)it.b * p.H + it.h) * hstride + (size_t)q;
+      const float L2 = p.lse2[lrow];
+      const float Dq = p.dpad[lrow];
+      int n = 0;
+      for (int j = it.lo; j <= it.hi; ++j) {
+        if (!rel(p, it, j)) continue;
+        const int64_t k0 = (int64_t)j * 128 + 64 * w;  // first key column of this half
+        bool partial = (p.causal && j == it.i) || ((int64_t)(j + 1) * 128 > p.S) ||
+                       ((int64_t)(it.i + 1) * 128 > p.S);
+        if (p.seg) {
+          const size_t kj = (size_t)it.b * p.n_tiles + j;
+          const int32_t a0 = p.tmin[kj], a1 = p.tmax[kj];
+          partial |= !(it.qmin >= 0 && it.qmin == it.qmax && a0 == it.qmin && a1 == it.qmin);
+        }
+        uint32_t mw0 = 0xffffffffu, mw1 = 0xffffffffu;
+        if (partial) {
+          // keep key k = k0 + c iff k < S, same segment, and k <= q when causal
+          int hi = 64;  // exclusive
+          if (p.causal) {
+            const int64_t d = q - k0 + 1;
+            hi = d < 0 ? 0 : (d > 64 ? 64 : (int)d);
+          }
+          const int64_t kv = p.S - k0;
+          if (kv < hi) hi = kv < 0 ? 0 : (int)kv;
+          if (seg_q < 0) hi = 0;
+          const int32_t* ks = p.seg ? p.seg + (size_t)it.b * p.S + k0 : nullptr;
+          uint32_t m[2] = {0, 0};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t bits = 0;
+#pragma unroll 4
+            for (int c = 0; c < 32; ++c) {
+              const int cc = h2 * 32 + c;
+              const bool keep = cc < hi && (ks == nullptr || __ldg(ks + cc) == seg_q);
+              bits |= (uint32_t)keep << c;
+            }
+            m[h2] = bits;
+          }
+          mw0 = m[0];
+          mw1 = m[1];
+        }
+        // ---- S -> registers; P = exp2(S * scale*log2e - LSE2[q]) ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 60 + w))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(tS + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tS + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_S_READ));
+        float pr[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const bool keep = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
+          pr[c] = keep ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -L2)) : 0.f;
+        }
+        // ---- dS = P o (dP - D[q]) back into tensor memory over dP ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 62 + w))) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            pk[u] = pack_bf16(pr[2 * u] * (__uint_as_float(r[2 * u]) - Dq),
+                              pr[2 * u + 1] * (__uint_as_float(r[2 * u + 1]) - Dq));
+          tmem_st32(tDP + 64 * w, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_DS_FULL));
+        ++steps;
+        ++n;
+      }
+      if (!ok) break;
+      // ---- dq epilogue: scale, inverse rotation, bf16 ----
+      __nv_bfloat16* dqrow = p.dq + (((size_t)it.b * p.S + (q_ok ? q : 0)) * p.H + it.h) * kD + 64 * w;
+      if (n == 0) {
+        if (q_ok) {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) reinterpret_cast<uint4*>(dqrow)[c] = z;
+        }
+        continue;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), dqc & 1, ab, 64 + w))) { ok = false; break; }
+      ++dqc;
+      tc_fence_after();
+      uint32_t r[64];
+      tmem_ld32(tDQ + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(tDQ + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_DQ_EMPTY));
+      uint32_t out[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
+        if (p.rotate) {
+          float c, s;
+          rope_cos_sin_fast(q, rope_freq(32 * w + u, kD, p.log2_theta), &c, &s);
+          const float a2 = a * c + b * s, b2 = b * c - a * s;
+          a = a2;
+          b = b2;
+        }
+        out[u] = pack_bf16(a, b);
+      }
+      if (q_ok) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          reinterpret_cast<uint4*>(dqrow)[c] =
+              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 1 && lane == 0) {
+      mma_commit(bar(B_FIN));
+      drain_wait(bar(B_FIN), 0);
+    }
+    if (warp == 0 && lane == 0) {
+      if (q_issued > 0) drain_wait(bar(B_Q_FULL), (q_issued - 1) & 1);
+      for (uint32_t n = (kv_issued > 2 ? kv_issued - 2 : 0); n < kv_issued; ++n)
+        drain_wait(bar(B_KV_FULL + (n & 1)), (n >> 1) & 1);
+    }
+  }
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sm100_bwd_dq(const Problem& pb, const Workspace& ws, const void* v,
+                                const void* d_o, void* dq, cudaStream_t st) {
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
+    return cudaErrorInvalidValue;
+  DqParams p{};
+  p.seg = pb.seg;
+  p.tmin = ws.tile_min;
+  p.tmax = ws.tile_max;
+  p.q_lo = ws.q_lo;
+  p.lse2 = ws.lse2_pad;
+  p.dpad = ws.delta_pad;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.status = ws.status;
+  p.S = pb.S;
+  p.H = (int)pb.H;
+  p.B = (int)pb.B;
+  p.n_tiles = (int)pb.n_tiles;
+  p.scale = pb.scale;
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.causal = pb.causal;
+  p.rotate = pb.theta > 0.0;
+  p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
+  const int64_t n_items = pb.B * pb.H * pb.n_tiles;
+  if (n_items == 0) return cudaSuccess;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
+  attn_bwd_dq_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace lwm

@@ -1,36 +1,35 @@
-// Backward attention on the 5th-generation tensor cores (sm_100a), bf16, D=128.
+// Backward attention, part 1 of 2: dK and dV, on the 5th-generation tensor
+// cores (sm_100a), bf16, D=128.
 //
 // Gradients of sum(O * dO) for exact causal attention with a packing mask
 // (LWM research note, "训练方法": training through the layer, Masked Sequence
 // Packing).  P is recomputed from the saved LSE, as in the FlashAttention
-// entry of the paper card's references; the backward is FlashAttention's
-// five products per (query tile i, key tile j):
+// entry of the paper card's references.  Per (query tile i, key tile j):
 //   S^T  = K~_j Q~_i^T            P^T  = exp(S^T * scale - LSE_i)
 //   dP^T = V_j dO_i^T             dS^T = P^T o (dP^T - D_i),  D_i = dO_i . O_i
-//   dV_j += P^T dO_i              dK~_j += dS^T Q~_i      dQ~_i += dS K~_j
+//   dV_j += P^T dO_i              dK~_j += dS^T Q~_i
+// dQ is computed by the query-stationary kernel of part 2, so nothing here
+// has to be reduced across CTAs.
 //
 // One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
 // walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
-// tensor memory for the whole walk, dQ partials are added into an fp32
-// buffer with TMA bulk reductions.  Roles (384 threads):
-//   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i per step
-//               through a 2-stage ring.
+// tensor memory for the whole walk.  Roles (384 threads):
+//   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i, and the
+//               tile's LSE*log2(e) and D (1-D bulk copies) per step, through a
+//               2-stage ring.
 //   warp 1      MMA issuer (one thread).
 //   warp 2      tensor-memory allocation.
-//   warp 3      dQ reduce issuer (one thread).
 //   warps 4-7   element-wise work on query columns 0-63, warps 8-11 on
-//               columns 64-127: P^T into TMEM (bf16, over S^T), dS^T into
-//               shared memory (bf16, 128-byte swizzle), the dQ drain, and
-//               the dK/dV epilogue (scale, inverse RoPE, bf16).
-// TMEM columns: S^T [0,128) with P^T over it (queries 0-63 packed into
-// columns 0-31, queries 64-127 into 64-95, so each warpgroup overwrites only
-// S^T columns it read itself), dP^T then dQ [128,256), dV [256,384),
-// dK [384,512).  MMA issue order per step:
-//   dP(i) after drain(i-1) | dV(i) after P(i) | S(i+1) | dK(i) dQ(i) after dS(i)
-// and the element-wise warps run P(i+1), drain(i), dS(i+1), so the
-// exponentials of one step overlap the dK/dQ products of the previous one.
-// LSE*log2(e) and D for each query tile arrive in shared memory with the
-// Q/dO tiles (1-D bulk copies on the same barrier).
+//               columns 64-127: P^T and dS^T (bf16) back into tensor memory,
+//               then the dK/dV epilogue (scale, inverse RoPE, bf16).
+// TMEM columns: S^T [0,128) with P^T over it, dP^T [128,256) with dS^T over
+// it, dV [256,384), dK [384,512).  A half's bf16 result goes into the first
+// 32 columns of that half's own 64-column range (queries 0-63 -> +0..31,
+// 64-127 -> +64..95), so no warpgroup overwrites columns the other still
+// reads; dV and dK take P^T and dS^T straight from tensor memory.
+// MMA issue order per step:
+//   dP(i) | dV(i) after P(i) | S(i+1) | dK(i) after dS(i) | dP(i+1) ...
+// so the exponentials of step i+1 overlap dK(i) and dP(i+1).
 #include <cuda.h>
 
 #include <mutex>
@@ -42,7 +41,6 @@
 namespace lwm {
 
 bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
-bool make_f32_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
 int sm_count();
 
 namespace {
@@ -65,16 +63,15 @@ constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = OFF_K + kTileBytes;
 constexpr uint32_t OFF_Q = OFF_V + kTileBytes;       // 2 stages
 constexpr uint32_t OFF_DO = OFF_Q + 2 * kTileBytes;  // 2 stages
-constexpr uint32_t OFF_DS = OFF_DO + 2 * kTileBytes;
-constexpr uint32_t kTilesBytes = OFF_DS + kTileBytes;  // 224 KB
-constexpr uint32_t kSmemBytes = 232448;                // the sm_100 per-block maximum
+constexpr uint32_t kTilesBytes = OFF_DO + 2 * kTileBytes;  // 192 KB
+constexpr uint32_t kSmemBytes = kTilesBytes + kSmallBytes + 1024;
 
 enum : uint32_t {
   B_KV_FULL = 0, B_KV_EMPTY = 1,
   B_QD_FULL = 2,   // 2 stages
   B_QD_EMPTY = 4,  // 2 stages
-  B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_DS_FULL = 9, B_DQ_FULL = 10, B_DRAIN = 11,
-  B_DKV_FULL = 12, B_DKV_EMPTY = 13, B_FIN = 14, B_STAGED = 15
+  B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_DS_FULL = 9,
+  B_DKV_FULL = 10, B_DKV_EMPTY = 11, B_FIN = 12
 };
 
 struct BwdParams {
@@ -84,7 +81,6 @@ struct BwdParams {
   const int32_t* k_hi;
   const float* lse2;   // [B, H, nT*128]: LSE * log2(e), +inf where the row has no keys
   const float* dpad;   // [B, H, nT*128]: dot(dO, O), 0 past the end
-  float* dq_acc;       // [B, S, H, D]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   DeviceStatus* status;
@@ -144,30 +140,13 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const BwdParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + kSmallBytes + 1023u) & ~1023u;
-  if (base - raw + kTilesBytes > kSmemBytes) {
-    // the tiles would not fit after aligning (never seen: the dynamic shared
-    // memory window starts 1024-byte aligned); refuse instead of overrunning
-    if (threadIdx.x == 0) report_status(p.status, LWM_ERR_UNSUPPORTED, 99);
-    return;
-  }
   const uint32_t bar0 = raw + SOFF_BAR;
   auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 8);
@@ -183,24 +162,20 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(bar(B_KV_EMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_QD_FULL + s), 1);
-      mbar_init(bar(B_QD_EMPTY + s), 1);  // arrived by the dQ reduce issuer
+      mbar_init(bar(B_QD_EMPTY + s), 1);
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_DP_FULL), 1);
     mbar_init(bar(B_P_FULL), 256);
     mbar_init(bar(B_DS_FULL), 256);
-    mbar_init(bar(B_DQ_FULL), 1);
-    mbar_init(bar(B_DRAIN), 256);
     mbar_init(bar(B_DKV_FULL), 1);
     mbar_init(bar(B_DKV_EMPTY), 256);
     mbar_init(bar(B_FIN), 1);
-    mbar_init(bar(B_STAGED), 256);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
-    tma_prefetch_desc(&tm_dq);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -253,20 +228,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);   // K-major x K-major
-      constexpr uint32_t kIdKM = idesc_bf16(128, 128, 0, 1);   // K-major (or TMEM) x MN-major
-      constexpr uint32_t kIdMM = idesc_bf16(128, 128, 1, 1);   // MN-major x MN-major
-      const uint32_t sK = base + OFF_K, sV = base + OFF_V, sDS = base + OFF_DS;
+      constexpr uint32_t kIdTM = idesc_bf16(128, 128, 0, 1);   // TMEM (K-major) x MN-major
+      const uint32_t sK = base + OFF_K, sV = base + OFF_V;
       const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
       uint32_t q_it = 0, steps = 0, dkv = 0;
       int items = 0;
       bool ok = true;
-      // A, B both K-major SW128 128x128 tiles: k-step kk walks 32 bytes inside a
-      // 128-byte row, then jumps to the second 64-column box.
+      // K-major SW128 128x128 tile: k-step kk walks 32 bytes inside a 128-byte
+      // row, then jumps to the second 64-column box.
       auto kdesc = [](uint32_t t, int kk) {
         return smem_desc_sw128(t + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
       };
       // MN-major SW128 tile (rows = K, 64-wide boxes along MN): k-step = 16 rows.
       auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
+      // bf16 A operand in TMEM, packed per half as described above
+      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 2) * 64 + (kk & 3) * 8; };
       auto sq_of = [&](uint32_t n) { return base + OFF_Q + (n & 1) * kTileBytes; };
       auto sdo_of = [&](uint32_t n) { return base + OFF_DO + (n & 1) * kTileBytes; };
       auto issue_s = [&](uint32_t n) {
@@ -286,9 +262,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           issue_s(q_it);
         }
         while (i >= 0) {
-          // dP^T(i) into the dQ columns once dQ(i-1) has been drained
-          if (steps > 0 && !mbar_wait(bar(B_DRAIN), (steps - 1) & 1, ab, 25)) { ok = false; break; }
-          tc_fence_after();
+          // dP^T(i): dS^T(i-1) in these columns went to dK(i-1), issued before
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(tDP, kdesc(sV, kk), kdesc(sdo_of(q_it), kk), kIdKK, kk > 0);
@@ -297,11 +271,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 27)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // P^T: queries 0-63 at cols 0-31, 64-127 at 64-95
-            mma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, mdesc(sdo_of(q_it), kk), kIdKM,
-                   (kk > 0 || !first) ? 1u : 0u);
-          // S^T(i+1) goes in now (dV(i) has taken P^T(i) from those columns, in
-          // issue order), so the next exponentials overlap dK(i) and dQ(i)
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tDV, tcol(tS, kk), mdesc(sdo_of(q_it), kk), kIdTM, (kk > 0 || !first) ? 1u : 0u);
+          // S^T(i+1) now: dV(i) has taken P^T(i) from these columns (issue order)
           const int inext = next_rel(p, it, i);
           if (inext >= 0) {
             if (!mbar_wait(bar(B_QD_FULL + ((q_it + 1) & 1)), ((q_it + 1) >> 1) & 1, ab, 29)) { ok = false; break; }
@@ -312,10 +284,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDK, kdesc(sDS, kk), mdesc(sq_of(q_it), kk), kIdKM, (kk > 0 || !first) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, mdesc(sDS, kk), mdesc(sK, kk), kIdMM, kk > 0);
-          mma_commit(bar(B_DQ_FULL));
+            mma_ts(tDK, tcol(tDP, kk), mdesc(sq_of(q_it), kk), kIdTM, (kk > 0 || !first) ? 1u : 0u);
+          mma_commit(bar(B_QD_EMPTY + (q_it & 1)));
           ++q_it;
           ++steps;
           first = false;
@@ -329,81 +299,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_commit(bar(B_KV_EMPTY));
       }
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------ dQ reduce issuer
-    // Each step's dQ partial is staged (fp32, 128-byte swizzle) in that step's
-    // own Q~/dO stage buffers, which its MMAs no longer need; this thread adds
-    // it into the fp32 accumulator with four 32-column TMA reductions and hands
-    // the stage back to the producer once the reductions have read it.
-    if (lane == 0) {
-      uint32_t steps = 0;
-      bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-        const Item it = decode(p, idx);
-        for (int i = it.lo; i <= it.hi && ok; ++i) {
-          if (!rel(p, it, i)) continue;
-          const uint32_t s = steps & 1;
-          if (!mbar_wait(bar(B_STAGED), steps & 1, ab, 40)) { ok = false; break; }
-          const uint32_t bq = base + OFF_Q + s * kTileBytes, bd = base + OFF_DO + s * kTileBytes;
-          tma_reduce_add_4d(&tm_dq, bq, 0, it.h, i * 128, it.b);
-          tma_reduce_add_4d(&tm_dq, bq + kBoxBytes, 32, it.h, i * 128, it.b);
-          tma_reduce_add_4d(&tm_dq, bd, 64, it.h, i * 128, it.b);
-          tma_reduce_add_4d(&tm_dq, bd + kBoxBytes, 96, it.h, i * 128, it.b);
-          bulk_commit_group();
-          bulk_wait_read_all();
-          mbar_arrive(bar(B_QD_EMPTY + s));
-          ++steps;
-        }
-      }
-      bulk_wait_all();  // the accumulator must hold every partial when the kernel ends
-    }
   } else if (warp >= 4) {
     // ------------------------------------------------- element-wise work
     const int w = (warp - 4) >> 2;                // column half
-    const int row = ((warp & 3) << 5) + lane;     // TMEM lane
+    const int row = ((warp & 3) << 5) + lane;     // TMEM lane = key in the tile
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base;
     const uint32_t tDP = tmem + lane_base + 128u;
     const uint32_t tDV = tmem + lane_base + 256u;
     const uint32_t tDK = tmem + lane_base + 384u;
-    const uint32_t sDS = base + OFF_DS + (uint32_t)w * kBoxBytes + (uint32_t)(row >> 3) * 1024u +
-                         (uint32_t)(row & 7) * 128u;
     uint32_t steps = 0, dkv = 0;
     bool ok = true;
-
-    // dQ partial of step `s` (query tile i; TMEM lane = query): TMEM -> registers
-    // -> the step's free stage buffer (this half's 64 columns = two 32-column
-    // fp32 boxes, 128-byte swizzle) for the reduce issuer.
-    auto drain = [&](uint32_t s) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), s & 1, ab, 34 + w))) return false;
-      tc_fence_after();
-      const uint32_t stage_buf = base + (w == 0 ? OFF_Q : OFF_DO) + (s & 1) * kTileBytes;
-      const uint32_t rbase = stage_buf + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
-      uint32_t r[32];
-#pragma unroll
-      for (int lb = 0; lb < 2; ++lb) {
-        tmem_ld32(tDP + 64 * w + 32 * lb, r);
-        tmem_wait_ld();
-        if (lb == 1) {
-          tc_fence_before();
-          mbar_arrive(bar(B_DRAIN));  // the dQ columns may take dP(i+1) now
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(rbase + (uint32_t)lb * kBoxBytes + (uint32_t)((c ^ (row & 7)) << 4),
-                       r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_STAGED));
-      return true;
-    };
-
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
       const Item it = decode(p, idx);
       const int64_t key = (int64_t)it.j * 128 + row;
       const bool key_ok = key < p.S;
       const int32_t seg_k = key_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + key] : 0) : -1;
-      int n = 0, pend = -1;  // pend: query tile whose dQ partial is not drained yet
+      int n = 0;
       for (int i = it.lo; i <= it.hi; ++i) {
         if (!rel(p, it, i)) continue;
         const int64_t q0 = (int64_t)i * 128 + 64 * w;  // first query column of this half
@@ -476,19 +388,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           uint32_t pk[32];
 #pragma unroll
           for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
-          // P^T for this half goes into the first 32 columns of the half's own
-          // S^T range, which no other warpgroup reads.
           tmem_st32(tS + 64 * w, pk);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL));
-        // ---- the previous step's dQ partial, while dK/dQ of this one run ----
-        if (pend >= 0) {
-          if (!drain(steps - 1)) { ok = false; break; }
-          pend = -1;
-        }
-        // ---- dS^T = P^T o (dP^T - D[q]) -> shared memory ----
+        // ---- dS^T = P^T o (dP^T - D[q]) back into tensor memory ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 32 + w))) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -508,22 +413,19 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
           }
         }
+        {
+          uint32_t pk[32];
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          const int c = c16 * 8;
-          st_shared_v4(sDS + (uint32_t)((c16 ^ (row & 7)) << 4), pack_bf16(pr[c], pr[c + 1]),
-                       pack_bf16(pr[c + 2], pr[c + 3]), pack_bf16(pr[c + 4], pr[c + 5]),
-                       pack_bf16(pr[c + 6], pr[c + 7]));
+          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
+          tmem_st32(tDP + 64 * w, pk);
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_DS_FULL));
-        pend = i;
         ++steps;
         ++n;
       }
       if (!ok) break;
-      if (pend >= 0 && !drain(steps - 1)) { ok = false; break; }
       // ---- dK, dV epilogue for this key tile ----
       __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
       __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
@@ -604,14 +506,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 }  // namespace
 
-cudaError_t launch_sm100_bwd(const Problem& pb, const Workspace& ws, const void* v,
-                             const void* d_o, void* dk, void* dv, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, tdo, tdq;
+cudaError_t launch_sm100_bwd_dkdv(const Problem& pb, const Workspace& ws, const void* v,
+                                  const void* d_o, void* dk, void* dv, cudaStream_t st) {
+  CUtensorMap tq, tk, tv, tdo;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D) ||
-      !make_f32_map(&tdq, ws.dq_acc, pb.B, pb.S, pb.H, pb.D))
+      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
   BwdParams p{};
   p.seg = pb.seg;
@@ -620,7 +521,6 @@ cudaError_t launch_sm100_bwd(const Problem& pb, const Workspace& ws, const void*
   p.k_hi = ws.k_hi;
   p.lse2 = ws.lse2_pad;
   p.dpad = ws.delta_pad;
-  p.dq_acc = ws.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.status = ws.status;
@@ -638,12 +538,12 @@ cudaError_t launch_sm100_bwd(const Problem& pb, const Workspace& ws, const void*
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes);
+    attr_err = cudaFuncSetAttribute(attn_bwd_dkdv_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
-  attn_bwd_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, tdq, p);
+  attn_bwd_dkdv_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, p);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -560,21 +560,6 @@ bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64
   return r == CUDA_SUCCESS;
 }
 
-// [B, S, H, D] fp32 as a 4-D tensor map with 32 x 1 x 128 x 1 boxes (128 bytes
-// inner), 128-byte swizzle: the dQ accumulator the backward reduces into.
-bool make_f32_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)(D * 4), (cuuint64_t)(H * D * 4), (cuuint64_t)(S * H * D * 4)};
-  cuuint32_t box[4] = {32, 1, 128, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 int sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);

@@ -32,7 +32,6 @@ struct Workspace {
   int32_t* k_hi;       // [B, n_tiles] last query tile a key tile may feed
   void* q_rot;         // [B, S, H, D] rotated q (dtype)
   void* k_rot;         // [B, S, H, D] rotated k (dtype)
-  float* dq_acc;       // [B, S, H, D] fp32 (backward, tensor-core path)
   float* delta;        // [B, H, S] fp32 dot(dO, O) per row (backward, CUDA-core path)
   float* lse2_pad;     // [B, H, n_tiles*128] LSE*log2(e) or +inf (backward, tensor-core path)
   float* delta_pad;    // [B, H, n_tiles*128] dot(dO, O) or 0 (backward, tensor-core path)
@@ -62,11 +61,12 @@ cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float
 cudaError_t launch_sm100_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                              float* lse, cudaStream_t st);
 
-cudaError_t launch_sm100_bwd(const Problem& p, const Workspace& ws, const void* v,
-                             const void* d_o, void* dk, void* dv, cudaStream_t st);
 cudaError_t launch_bwd_prep(const Problem& p, const void* o, const void* d_o, const float* lse,
                             const Workspace& ws, cudaStream_t st);
-cudaError_t launch_dq_post(const Problem& p, const Workspace& ws, void* dq, cudaStream_t st);
+cudaError_t launch_sm100_bwd_dkdv(const Problem& p, const Workspace& ws, const void* v,
+                                  const void* d_o, void* dk, void* dv, cudaStream_t st);
+cudaError_t launch_sm100_bwd_dq(const Problem& p, const Workspace& ws, const void* v,
+                                const void* d_o, void* dq, cudaStream_t st);
 
 cudaError_t launch_simt_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                             float* lse, cudaStream_t st);

@@ -110,45 +110,6 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
   }
 }
 
-// dq = R(p)^T (scale * dq_acc) rounded to bf16; dq_acc is [B, S, H, D] fp32.
-// Same thread layout as rope_kernel (fp32 in: 4 elements = 2 pairs a thread).
-__global__ void __launch_bounds__(128) dq_post_kernel(const float* __restrict__ acc,
-                                                      __nv_bfloat16* __restrict__ dq,
-                                                      int64_t n_tok, int64_t S, int H, int D,
-                                                      float scale, double log2_theta,
-                                                      int rotate) {
-  const int per_head = D / 4;
-  const int c = threadIdx.x % per_head;
-  const int hg = threadIdx.x / per_head;
-  const int heads_per_pass = blockDim.x / per_head;
-  if (hg >= heads_per_pass) return;
-  double w[2] = {0.0, 0.0};
-  if (rotate) {
-    w[0] = rope_freq(2 * c, D, log2_theta);
-    w[1] = rope_freq(2 * c + 1, D, log2_theta);
-  }
-  for (int64_t tok = blockIdx.x; tok < n_tok; tok += gridDim.x) {
-    float cs[2] = {1.f, 1.f}, sn[2] = {0.f, 0.f};
-    if (rotate) {
-      const int64_t pos = tok % S;
-      rope_cos_sin_w(pos, w[0], &cs[0], &sn[0]);
-      rope_cos_sin_w(pos, w[1], &cs[1], &sn[1]);
-    }
-    const size_t base = (size_t)tok * H * D;
-    for (int h = hg; h < H; h += heads_per_pass) {
-      const size_t off = base + (size_t)h * D + (size_t)c * 4;
-      const float4 x = *reinterpret_cast<const float4*>(acc + off);
-      const float a0 = x.x * scale, b0 = x.y * scale, a1 = x.z * scale, b1 = x.w * scale;
-      __nv_bfloat162 y0 = __floats2bfloat162_rn(a0 * cs[0] + b0 * sn[0], b0 * cs[0] - a0 * sn[0]);
-      __nv_bfloat162 y1 = __floats2bfloat162_rn(a1 * cs[1] + b1 * sn[1], b1 * cs[1] - a1 * sn[1]);
-      uint2 outv;
-      outv.x = *reinterpret_cast<uint32_t*>(&y0);
-      outv.y = *reinterpret_cast<uint32_t*>(&y1);
-      *reinterpret_cast<uint2*>(dq + off) = outv;
-    }
-  }
-}
-
 int grid_for(int64_t n) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -209,17 +170,6 @@ cudaError_t launch_bwd_prep(const Problem& p, const void* o, const void* d_o, co
   bwd_prep_kernel<<<(unsigned)grid, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse,
       ws.lse2_pad, ws.delta_pad, rows, p.S, s_pad, (int)p.H, (int)p.D);
-  note_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dq_post(const Problem& p, const Workspace& ws, void* dq, cudaStream_t st) {
-  const int64_t n_tok = p.B * p.S;
-  if (n_tok == 0) return cudaSuccess;
-  const int rotate = p.theta > 0.0;
-  dq_post_kernel<<<grid_for(n_tok), 128, 0, st>>>(ws.dq_acc, static_cast<__nv_bfloat16*>(dq), n_tok,
-                                                  p.S, (int)p.H, (int)p.D, p.scale,
-                                                  rotate ? log2(p.theta) : 0.0, rotate);
   note_launches(1);
   return cudaGetLastError();
 }
