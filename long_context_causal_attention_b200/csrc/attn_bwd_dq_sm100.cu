@@ -9,14 +9,15 @@
 // One persistent CTA per SM owns a query tile i of one (b, h) and sweeps the
 // key tiles j it may attend to; dQ~_i accumulates in tensor memory, and the
 // epilogue applies the scale and the inverse rotation and writes bf16 dq, so
-// no partial sums leave the CTA.  Roles (384 threads):
+// no partial sums leave the CTA.  Roles (640 threads):
 //   warp 0      TMA producer: Q~_i and dO_i once per item, K~_j and V_j per
 //               step through a 2-stage ring.
 //   warp 1      MMA issuer (one thread).
 //   warp 2      tensor-memory allocation.
-//   warps 4-7   element-wise work on key columns 0-63, warps 8-11 on 64-127
+//   warps 4-19  element-wise work, four warpgroups on 32 key columns each
 //               (one query row per thread), then the dq epilogue.
-// TMEM columns: S [0,128), dP [128,256) with dS (bf16) over it, dQ~ [256,384).
+// TMEM columns: S [0,128), dP [128,256) with dS (bf16) over it (each quarter
+// packs its dS into the first 16 of its own 32 columns), dQ~ [256,384).
 // MMA issue order per step:
 //   S(j+1) once S(j) is in registers | dQ(j) after dS(j) | dP(j+1) ...
 #include <cuda.h>
@@ -37,7 +38,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;   // 4 control warps + 4 element-wise warpgroups
+constexpr int kEW = 512;        // element-wise threads
 constexpr uint32_t kTileBytes = 128 * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;
 
@@ -153,11 +155,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(bar(B_KV_EMPTY + s), 1);
     }
     mbar_init(bar(B_S_FULL), 1);
-    mbar_init(bar(B_S_READ), 256);
+    mbar_init(bar(B_S_READ), kEW);
     mbar_init(bar(B_DP_FULL), 1);
-    mbar_init(bar(B_DS_FULL), 256);
+    mbar_init(bar(B_DS_FULL), kEW);
     mbar_init(bar(B_DQ_FULL), 1);
-    mbar_init(bar(B_DQ_EMPTY), 256);
+    mbar_init(bar(B_DQ_EMPTY), kEW);
     mbar_init(bar(B_FIN), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -218,7 +220,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         return smem_desc_sw128(t + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
       };
       auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
-      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 2) * 64 + (kk & 3) * 8; };
+      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 1) * 32 + (kk & 1) * 8; };
       auto sk_of = [&](uint32_t n) { return base + OFF_K + (n & 1) * kTileBytes; };
       auto sv_of = [&](uint32_t n) { return base + OFF_V + (n & 1) * kTileBytes; };
       auto issue_s = [&](uint32_t n) {
@@ -276,12 +278,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- element-wise work
-    const int w = (warp - 4) >> 2;                // key column half
+    const int w = (warp - 4) >> 2;                // key-column quarter
     const int row = ((warp & 3) << 5) + lane;     // TMEM lane = query in the tile
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tDP = tmem + lane_base + 128u;
-    const uint32_t tDQ = tmem + lane_base + 256u;
+    const uint32_t tS = tmem + lane_base + 32u * w;
+    const uint32_t tDP = tmem + lane_base + 128u + 32u * w;
+    const uint32_t tDQ = tmem + lane_base + 256u + 32u * w;
     const size_t hstride = (size_t)p.n_tiles * 128;
     uint32_t steps = 0, dqc = 0;
     bool ok = true;
@@ -296,7 +298,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int n = 0;
       for (int j = it.lo; j <= it.hi; ++j) {
         if (!rel(p, it, j)) continue;
-        const int64_t k0 = (int64_t)j * 128 + 64 * w;  // first key column of this half
+        const int64_t k0 = (int64_t)j * 128 + 32 * w;  // first key column of this quarter
         bool partial = (p.causal && j == it.i) || ((int64_t)(j + 1) * 128 > p.S) ||
                        ((int64_t)(it.i + 1) * 128 > p.S);
         if (p.seg) {
@@ -304,61 +306,55 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const int32_t a0 = p.tmin[kj], a1 = p.tmax[kj];
           partial |= !(it.qmin >= 0 && it.qmin == it.qmax && a0 == it.qmin && a1 == it.qmin);
         }
-        uint32_t mw0 = 0xffffffffu, mw1 = 0xffffffffu;
+        uint32_t mw = 0xffffffffu;
         if (partial) {
           // keep key k = k0 + c iff k < S, same segment, and k <= q when causal
-          int hi = 64;  // exclusive
+          int hi = 32;  // exclusive
           if (p.causal) {
             const int64_t d = q - k0 + 1;
-            hi = d < 0 ? 0 : (d > 64 ? 64 : (int)d);
+            hi = d < 0 ? 0 : (d > 32 ? 32 : (int)d);
           }
           const int64_t kv = p.S - k0;
           if (kv < hi) hi = kv < 0 ? 0 : (int)kv;
           if (seg_q < 0) hi = 0;
           const int32_t* ks = p.seg ? p.seg + (size_t)it.b * p.S + k0 : nullptr;
-          uint32_t m[2] = {0, 0};
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t bits = 0;
+          uint32_t bits = 0;
 #pragma unroll 4
-            for (int c = 0; c < 32; ++c) {
-              const int cc = h2 * 32 + c;
-              const bool keep = cc < hi && (ks == nullptr || __ldg(ks + cc) == seg_q);
-              bits |= (uint32_t)keep << c;
-            }
-            m[h2] = bits;
+          for (int c = 0; c < 32; ++c) {
+            const bool keep = c < hi && (ks == nullptr || __ldg(ks + c) == seg_q);
+            bits |= (uint32_t)keep << c;
           }
-          mw0 = m[0];
-          mw1 = m[1];
+          mw = bits;
         }
         // ---- S -> registers; P = exp2(S * scale*log2e - LSE2[q]) ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 60 + w))) { ok = false; break; }
         tc_fence_after();
-        uint32_t r[64];
-        tmem_ld32(tS + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tS + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        uint32_t r[32];
+        tmem_ld32(tS, r);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(B_S_READ));
-        float pr[64];
+        float pr[32];
+        if (partial) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool keep = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-          pr[c] = keep ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -L2)) : 0.f;
+          for (int c = 0; c < 32; ++c)
+            pr[c] = ((mw >> c) & 1u) ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -L2)) : 0.f;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pr[c] = fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -L2));
         }
         // ---- dS = P o (dP - D[q]) back into tensor memory over dP ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 62 + w))) { ok = false; break; }
         tc_fence_after();
-        tmem_ld32(tDP + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tDP + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(tDP, r);
         tmem_wait_ld();
         {
-          uint32_t pk[32];
+          uint32_t pk[16];
 #pragma unroll
-          for (int u = 0; u < 32; ++u)
+          for (int u = 0; u < 16; ++u)
             pk[u] = pack_bf16(pr[2 * u] * (__uint_as_float(r[2 * u]) - Dq),
                               pr[2 * u + 1] * (__uint_as_float(r[2 * u + 1]) - Dq));
-          tmem_st32(tDP + 64 * w, pk);
+          tmem_st16(tDP, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -367,32 +363,31 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ++n;
       }
       if (!ok) break;
-      // ---- dq epilogue: scale, inverse rotation, bf16 ----
-      __nv_bfloat16* dqrow = p.dq + (((size_t)it.b * p.S + (q_ok ? q : 0)) * p.H + it.h) * kD + 64 * w;
+      // ---- dq epilogue (this quarter's 32 columns): scale, inverse rotation, bf16 ----
+      __nv_bfloat16* dqrow = p.dq + (((size_t)it.b * p.S + (q_ok ? q : 0)) * p.H + it.h) * kD + 32 * w;
       if (n == 0) {
         if (q_ok) {
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) reinterpret_cast<uint4*>(dqrow)[c] = z;
+          for (int c = 0; c < 4; ++c) reinterpret_cast<uint4*>(dqrow)[c] = z;
         }
         continue;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), dqc & 1, ab, 64 + w))) { ok = false; break; }
       ++dqc;
       tc_fence_after();
-      uint32_t r[64];
-      tmem_ld32(tDQ + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tDQ + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      uint32_t r[32];
+      tmem_ld32(tDQ, r);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(B_DQ_EMPTY));
-      uint32_t out[32];
+      uint32_t out[16];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
+      for (int u = 0; u < 16; ++u) {
         float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
         if (p.rotate) {
           float c, s;
-          rope_cos_sin_fast(q, rope_freq(32 * w + u, kD, p.log2_theta), &c, &s);
+          rope_cos_sin_fast(q, rope_freq(16 * w + u, kD, p.log2_theta), &c, &s);
           const float a2 = a * c + b * s, b2 = b * c - a * s;
           a = a2;
           b = b2;
@@ -401,7 +396,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       if (q_ok) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c)
           reinterpret_cast<uint4*>(dqrow)[c] =
               make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
       }

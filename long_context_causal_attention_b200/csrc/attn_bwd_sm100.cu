@@ -13,20 +13,20 @@
 //
 // One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
 // walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
-// tensor memory for the whole walk.  Roles (384 threads):
+// tensor memory for the whole walk.  Roles (640 threads):
 //   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i, and the
 //               tile's LSE*log2(e) and D (1-D bulk copies) per step, through a
 //               2-stage ring.
 //   warp 1      MMA issuer (one thread).
 //   warp 2      tensor-memory allocation.
-//   warps 4-7   element-wise work on query columns 0-63, warps 8-11 on
-//               columns 64-127: P^T and dS^T (bf16) back into tensor memory,
-//               then the dK/dV epilogue (scale, inverse RoPE, bf16).
+//   warps 4-19  element-wise work, four warpgroups on 32 query columns each:
+//               P^T and dS^T (bf16) back into tensor memory, then the dK/dV
+//               epilogue (scale, inverse RoPE, bf16).
 // TMEM columns: S^T [0,128) with P^T over it, dP^T [128,256) with dS^T over
-// it, dV [256,384), dK [384,512).  A half's bf16 result goes into the first
-// 32 columns of that half's own 64-column range (queries 0-63 -> +0..31,
-// 64-127 -> +64..95), so no warpgroup overwrites columns the other still
-// reads; dV and dK take P^T and dS^T straight from tensor memory.
+// it, dV [256,384), dK [384,512).  A quarter's bf16 result goes into the
+// first 16 columns of that quarter's own 32-column range, so no warpgroup
+// overwrites columns another still reads; dV and dK take P^T and dS^T
+// straight from tensor memory.
 // MMA issue order per step:
 //   dP(i) | dV(i) after P(i) | S(i+1) | dK(i) after dS(i) | dP(i+1) ...
 // so the exponentials of step i+1 overlap dK(i) and dP(i+1).
@@ -48,7 +48,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;   // 4 control warps + 4 element-wise warpgroups
+constexpr int kEW = 512;        // element-wise threads
 constexpr uint32_t kTileBytes = 128 * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;
 
@@ -166,10 +167,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_DP_FULL), 1);
-    mbar_init(bar(B_P_FULL), 256);
-    mbar_init(bar(B_DS_FULL), 256);
+    mbar_init(bar(B_P_FULL), kEW);
+    mbar_init(bar(B_DS_FULL), kEW);
     mbar_init(bar(B_DKV_FULL), 1);
-    mbar_init(bar(B_DKV_EMPTY), 256);
+    mbar_init(bar(B_DKV_EMPTY), kEW);
     mbar_init(bar(B_FIN), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -241,8 +242,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       };
       // MN-major SW128 tile (rows = K, 64-wide boxes along MN): k-step = 16 rows.
       auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
-      // bf16 A operand in TMEM, packed per half as described above
-      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 2) * 64 + (kk & 3) * 8; };
+      // bf16 A operand in TMEM, packed per quarter as described above
+      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 1) * 32 + (kk & 1) * 8; };
       auto sq_of = [&](uint32_t n) { return base + OFF_Q + (n & 1) * kTileBytes; };
       auto sdo_of = [&](uint32_t n) { return base + OFF_DO + (n & 1) * kTileBytes; };
       auto issue_s = [&](uint32_t n) {
@@ -301,13 +302,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- element-wise work
-    const int w = (warp - 4) >> 2;                // column half
+    const int w = (warp - 4) >> 2;                // query-column quarter
     const int row = ((warp & 3) << 5) + lane;     // TMEM lane = key in the tile
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tDP = tmem + lane_base + 128u;
-    const uint32_t tDV = tmem + lane_base + 256u;
-    const uint32_t tDK = tmem + lane_base + 384u;
+    const uint32_t tS = tmem + lane_base + 32u * w;
+    const uint32_t tDP = tmem + lane_base + 128u + 32u * w;
+    const uint32_t tDV = tmem + lane_base + 256u + 32u * w;
+    const uint32_t tDK = tmem + lane_base + 384u + 32u * w;
     uint32_t steps = 0, dkv = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
@@ -318,7 +319,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       int n = 0;
       for (int i = it.lo; i <= it.hi; ++i) {
         if (!rel(p, it, i)) continue;
-        const int64_t q0 = (int64_t)i * 128 + 64 * w;  // first query column of this half
+        const int64_t q0 = (int64_t)i * 128 + 32 * w;  // first query column of this quarter
         bool partial = (p.causal && i == it.j) || ((int64_t)(i + 1) * 128 > p.S) ||
                        ((int64_t)(it.j + 1) * 128 > p.S);
         if (p.seg) {
@@ -326,35 +327,28 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           const int32_t a0 = p.tmin[qi], a1 = p.tmax[qi];
           partial |= !(it.kmin >= 0 && it.kmin == it.kmax && a0 == it.kmin && a1 == it.kmin);
         }
-        uint32_t mw0 = 0xffffffffu, mw1 = 0xffffffffu;
+        uint32_t mw = 0xffffffffu;
         if (partial) {
           // keep query q = q0 + c iff q < S, same segment, and q >= key when causal
           int lo = 0;
           if (p.causal) {
             const int64_t d = key - q0;
-            lo = d < 0 ? 0 : (d > 64 ? 64 : (int)d);
+            lo = d < 0 ? 0 : (d > 32 ? 32 : (int)d);
           }
           const int64_t qv = p.S - q0;
-          const int hi = qv > 64 ? 64 : (int)qv;  // exclusive
+          const int hi = qv > 32 ? 32 : (qv < 0 ? 0 : (int)qv);  // exclusive
           const int32_t* qs = p.seg ? p.seg + (size_t)it.b * p.S + q0 : nullptr;
-          uint32_t m[2] = {0, 0};
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t bits = 0;
+          uint32_t bits = 0;
 #pragma unroll 4
-            for (int c = 0; c < 32; ++c) {
-              const int cc = h2 * 32 + c;
-              const bool keep = seg_k >= 0 && cc >= lo && cc < hi &&
-                                (qs == nullptr || __ldg(qs + cc) == seg_k);
-              bits |= (uint32_t)keep << c;
-            }
-            m[h2] = bits;
+          for (int c = 0; c < 32; ++c) {
+            const bool keep = seg_k >= 0 && c >= lo && c < hi &&
+                              (qs == nullptr || __ldg(qs + c) == seg_k);
+            bits |= (uint32_t)keep << c;
           }
-          mw0 = m[0];
-          mw1 = m[1];
+          mw = bits;
         }
         const uint32_t stage = steps & 1;
-        const float* lse2 = ld_smem + stage * (kLdStageBytes / 4) + 64 * w;
+        const float* lse2 = ld_smem + stage * (kLdStageBytes / 4) + 32 * w;
         const float* dsum = lse2 + 128;
         // ---- P^T = exp2(S^T * scale*log2e - LSE2[q]) ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), steps & 1, ab, 30 + w) &&
@@ -363,32 +357,40 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           break;
         }
         tc_fence_after();
-        float pr[64];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
+        float pr[32];
+        {
           uint32_t r[32];
-          tmem_ld32(tS + 64 * w + 32 * h2, r);
+          tmem_ld32(tS, r);
           tmem_wait_ld();
-          const uint32_t mword = h2 == 0 ? mw0 : mw1;
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + 32 * h2);
+          const float4* l4 = reinterpret_cast<const float4*>(lse2);
+          if (partial) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 L = l4[u];
-            const float Ls[4] = {L.x, L.y, L.z, L.w};
+            for (int u = 0; u < 8; ++u) {
+              const float4 L = l4[u];
+              const float Ls[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * u + e;
-              const bool keep = (mword >> c) & 1u;
-              pr[32 * h2 + c] =
-                  keep ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -Ls[e])) : 0.f;
+              for (int e = 0; e < 4; ++e) {
+                const int c = 4 * u + e;
+                pr[c] = ((mw >> c) & 1u) ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -Ls[e]))
+                                         : 0.f;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float4 L = l4[u];
+              const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                pr[4 * u + e] = fast_exp2(fmaf(__uint_as_float(r[4 * u + e]), p.scale_log2, -Ls[e]));
             }
           }
         }
         {
-          uint32_t pk[32];
+          uint32_t pk[16];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
-          tmem_st32(tS + 64 * w, pk);
+          for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
+          tmem_st16(tS, pk);  // first 16 of this quarter's own 32 columns
         }
         tmem_wait_st();
         tc_fence_before();
@@ -396,28 +398,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ---- dS^T = P^T o (dP^T - D[q]) back into tensor memory ----
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 32 + w))) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
+        {
           uint32_t r[32];
-          tmem_ld32(tDP + 64 * w + 32 * h2, r);
+          tmem_ld32(tDP, r);
           tmem_wait_ld();
-          const float4* d4 = reinterpret_cast<const float4*>(dsum + 32 * h2);
+          const float4* d4 = reinterpret_cast<const float4*>(dsum);
+          uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const float4 Dv = d4[u];
-            const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 32 * h2 + 4 * u + e;
-              pr[c] = pr[c] * (__uint_as_float(r[4 * u + e]) - Ds[e]);
-            }
+            pk[2 * u] = pack_bf16(pr[4 * u] * (__uint_as_float(r[4 * u]) - Dv.x),
+                                  pr[4 * u + 1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
+            pk[2 * u + 1] = pack_bf16(pr[4 * u + 2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
+                                      pr[4 * u + 3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
           }
-        }
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
-          tmem_st32(tDP + 64 * w, pk);
+          tmem_st16(tDP, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -426,14 +421,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ++n;
       }
       if (!ok) break;
-      // ---- dK, dV epilogue for this key tile ----
-      __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
-      __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 64 * w;
+      // ---- dK, dV epilogue for this key tile (this quarter's 32 columns) ----
+      __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 32 * w;
+      __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 32 * w;
       if (n == 0) {
         if (key_ok) {
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             reinterpret_cast<uint4*>(dkrow)[c] = z;
             reinterpret_cast<uint4*>(dvrow)[c] = z;
           }
@@ -443,17 +438,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DKV_FULL), dkv & 1, ab, 36 + w))) { ok = false; break; }
       ++dkv;
       tc_fence_after();
-      uint32_t r[64];
-      tmem_ld32(tDK + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tDK + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      uint32_t r[32], rv[32];
+      tmem_ld32(tDK, r);
+      tmem_ld32(tDV, rv);
       tmem_wait_ld();
-      uint32_t out[32];
+      tc_fence_before();
+      mbar_arrive(bar(B_DKV_EMPTY));
+      uint32_t out[16];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
+      for (int u = 0; u < 16; ++u) {
         float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
         if (p.rotate) {
           float c, s;
-          rope_cos_sin_fast(key, rope_freq(32 * w + u, kD, p.log2_theta), &c, &s);
+          rope_cos_sin_fast(key, rope_freq(16 * w + u, kD, p.log2_theta), &c, &s);
           const float a2 = a * c + b * s, b2 = b * c - a * s;
           a = a2;
           b = b2;
@@ -462,23 +459,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       if (key_ok) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c) {
           reinterpret_cast<uint4*>(dkrow)[c] =
               make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
-      }
-      tmem_ld32(tDV + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tDV + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_DKV_EMPTY));
-      if (key_ok) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
           reinterpret_cast<uint4*>(dvrow)[c] = make_uint4(
-              pack_bf16(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
-              pack_bf16(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
-              pack_bf16(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
-              pack_bf16(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+              pack_bf16(__uint_as_float(rv[8 * c]), __uint_as_float(rv[8 * c + 1])),
+              pack_bf16(__uint_as_float(rv[8 * c + 2]), __uint_as_float(rv[8 * c + 3])),
+              pack_bf16(__uint_as_float(rv[8 * c + 4]), __uint_as_float(rv[8 * c + 5])),
+              pack_bf16(__uint_as_float(rv[8 * c + 6]), __uint_as_float(rv[8 * c + 7])));
+        }
       }
     }
   }
