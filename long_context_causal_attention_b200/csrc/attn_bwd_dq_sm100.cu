@@ -216,21 +216,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       uint32_t kv_it = 0, steps = 0, dqc = 0;
       int items = 0;
       bool ok = true;
-      auto kdesc = [](uint32_t t, int kk) {
-        return smem_desc_sw128(t + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-      };
-      auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
-      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 1) * 32 + (kk & 1) * 8; };
+      const uint64_t dQ = kmajor_desc(sQ), dDO = kmajor_desc(sDO);
       auto sk_of = [&](uint32_t n) { return base + OFF_K + (n & 1) * kTileBytes; };
       auto sv_of = [&](uint32_t n) { return base + OFF_V + (n & 1) * kTileBytes; };
       auto issue_s = [&](uint32_t n) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, kdesc(sQ, kk), kdesc(sk_of(n), kk), kIdKK, kk > 0);
+        mma_kk128(tS, dQ, kmajor_desc(sk_of(n)), kIdKK, 0u);
         mma_commit(bar(B_S_FULL));
       };
       auto issue_dp = [&](uint32_t n) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tDP, kdesc(sDO, kk), kdesc(sv_of(n), kk), kIdKK, kk > 0);
+        mma_kk128(tDP, dDO, kmajor_desc(sv_of(n)), kIdKK, 0u);
         mma_commit(bar(B_DP_FULL));
       };
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
@@ -257,9 +251,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 57)) { ok = false; break; }
           if (first && dqc > 0 && !mbar_wait(bar(B_DQ_EMPTY), (dqc - 1) & 1, ab, 58)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDQ, tcol(tDP, kk), mdesc(sk_of(kv_it), kk), kIdTM, (kk > 0 || !first) ? 1u : 0u);
+          mma_tm128<true>(tDQ, tDP, mnmajor_desc(sk_of(kv_it)), kIdTM, first ? 0u : 1u);
           mma_commit(bar(B_KV_EMPTY + (kv_it & 1)));
           ++kv_it;
           // dP(j+1): dS(j) in these columns went to dQ(j) just before (issue order)

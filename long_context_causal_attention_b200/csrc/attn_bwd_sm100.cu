@@ -235,20 +235,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       uint32_t q_it = 0, steps = 0, dkv = 0;
       int items = 0;
       bool ok = true;
-      // K-major SW128 128x128 tile: k-step kk walks 32 bytes inside a 128-byte
-      // row, then jumps to the second 64-column box.
-      auto kdesc = [](uint32_t t, int kk) {
-        return smem_desc_sw128(t + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-      };
-      // MN-major SW128 tile (rows = K, 64-wide boxes along MN): k-step = 16 rows.
-      auto mdesc = [](uint32_t t, int kk) { return smem_desc_sw128(t + kk * 2048, kBoxBytes, 1024); };
-      // bf16 A operand in TMEM, packed per quarter as described above
-      auto tcol = [](uint32_t t, int kk) { return t + (kk >> 1) * 32 + (kk & 1) * 8; };
+      const uint64_t dK = kmajor_desc(sK), dV = kmajor_desc(sV);
       auto sq_of = [&](uint32_t n) { return base + OFF_Q + (n & 1) * kTileBytes; };
       auto sdo_of = [&](uint32_t n) { return base + OFF_DO + (n & 1) * kTileBytes; };
       auto issue_s = [&](uint32_t n) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, kdesc(sK, kk), kdesc(sq_of(n), kk), kIdKK, kk > 0);
+        mma_kk128(tS, dK, kmajor_desc(sq_of(n)), kIdKK, 0u);
         mma_commit(bar(B_S_FULL));
       };
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
@@ -264,16 +255,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         while (i >= 0) {
           // dP^T(i): dS^T(i-1) in these columns went to dK(i-1), issued before
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDP, kdesc(sV, kk), kdesc(sdo_of(q_it), kk), kIdKK, kk > 0);
+          mma_kk128(tDP, dV, kmajor_desc(sdo_of(q_it)), kIdKK, 0u);
           mma_commit(bar(B_DP_FULL));
           if (first && dkv > 0 && !mbar_wait(bar(B_DKV_EMPTY), (dkv - 1) & 1, ab, 26)) { ok = false; break; }
           if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 27)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDV, tcol(tS, kk), mdesc(sdo_of(q_it), kk), kIdTM, (kk > 0 || !first) ? 1u : 0u);
+          mma_tm128<true>(tDV, tS, mnmajor_desc(sdo_of(q_it)), kIdTM, first ? 0u : 1u);
           // S^T(i+1) now: dV(i) has taken P^T(i) from these columns (issue order)
           const int inext = next_rel(p, it, i);
           if (inext >= 0) {
@@ -283,9 +270,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           }
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 28)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDK, tcol(tDP, kk), mdesc(sq_of(q_it), kk), kIdTM, (kk > 0 || !first) ? 1u : 0u);
+          mma_tm128<true>(tDK, tDP, mnmajor_desc(sq_of(q_it)), kIdTM, first ? 0u : 1u);
           mma_commit(bar(B_QD_EMPTY + (q_it & 1)));
           ++q_it;
           ++steps;

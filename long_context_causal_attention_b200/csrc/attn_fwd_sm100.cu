@@ -273,26 +273,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool first_pv[2] = {true, true}, active[2] = {false, false};
 
         auto issue_s = [&](int t) {
-          const uint32_t ks = base + OFF_K + (k_it & 1) * kTileBytes;
-          const uint32_t qs = sq0 + t * kTileBytes;
-          const uint32_t d = tmem + (uint32_t)(t * 128);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            mma_ss(d, smem_desc_sw128(qs + off, 16, 1024), smem_desc_sw128(ks + off, 16, 1024),
-                   kIdS, kk > 0);
-          }
+          mma_kk128(tmem + (uint32_t)(t * 128), kmajor_desc(sq0 + t * kTileBytes),
+                    kmajor_desc(base + OFF_K + (k_it & 1) * kTileBytes), kIdS, 0u);
           mma_commit(bar(B_S_FULL + t));
         };
         auto issue_pv = [&](int t) {
-          const uint32_t vs = base + OFF_V + (v_it & 1) * kTileBytes;
-          const uint32_t d = tmem + 256u + (uint32_t)(t * 128);
-          const uint32_t a = tmem + (uint32_t)(t * 128);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            mma_ts(d, a + kk * 8, smem_desc_sw128(vs + kk * 2048, kBoxBytes, 1024), kIdPV,
-                   (kk > 0 || !first_pv[t]) ? 1u : 0u);
-          }
+          mma_tm128<false>(tmem + 256u + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128),
+                           mnmajor_desc(base + OFF_V + (v_it & 1) * kTileBytes), kIdPV,
+                           first_pv[t] ? 0u : 1u);
           first_pv[t] = false;
         };
 

@@ -218,6 +218,43 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// 128 x 128 bf16 operand tiles as TMA lays them down: two 64-column boxes of
+// 16 KB, 128-byte swizzle.  Base descriptors for the two majors; the k-steps
+// of one 128-deep product are then constant offsets on the start address.
+constexpr uint32_t kOperandBoxBytes = 16384;
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
+  return smem_desc_sw128(saddr, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr) {
+  return smem_desc_sw128(saddr, kOperandBoxBytes, 1024);
+}
+
+// D (+)= A * B^T over K = 128, A and B K-major tiles (8 MMAs of K = 16): a
+// k-step walks 32 bytes inside the 128-byte row, then moves to the second box.
+__device__ __forceinline__ void mma_kk128(uint32_t d, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t off = (uint64_t)(((kk >> 2) * kOperandBoxBytes + (kk & 3) * 32) >> 4);
+    mma_ss(d, a_desc + off, b_desc + off, idesc, kk > 0 ? 1u : acc);
+  }
+}
+
+// D (+)= A * B over K = 128 with A (bf16) in tensor memory and B an MN-major
+// tile whose rows are K (a k-step is 16 rows = 2048 bytes).  A's k-step kk
+// starts at column a_col(kk): QUARTERS = false packs the 128 K values into 64
+// consecutive columns; QUARTERS = true has each 32-wide quarter of K packed into
+// the first 16 of its own 32 columns.
+template <bool QUARTERS>
+__device__ __forceinline__ void mma_tm128(uint32_t d, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t col = QUARTERS ? (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8) : (uint32_t)(kk * 8);
+    mma_ts(d, a_tmem + col, b_desc + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : acc);
+  }
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
