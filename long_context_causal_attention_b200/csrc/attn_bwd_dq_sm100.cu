@@ -10,8 +10,8 @@
 // key tiles j it may attend to; dQ~_i accumulates in tensor memory, and the
 // epilogue applies the scale and the inverse rotation and writes bf16 dq, so
 // no partial sums leave the CTA.  Roles (640 threads):
-//   warp 0      TMA producer: Q~_i and dO_i once per item, K~_j and V_j per
-//               step through a 2-stage ring.
+//   warp 0      TMA producer: Q~_i and dO_i once per item, K~_j (3-stage
+//               ring, issued two tiles ahead) and V_j (2-stage ring) per step.
 //   warp 1      MMA issuer (one thread).
 //   warp 2      tensor-memory allocation.
 //   warps 4-19  element-wise work, four warpgroups on 32 key columns each
@@ -48,17 +48,21 @@ constexpr uint32_t SOFF_MISC = 256;
 constexpr uint32_t kSmallBytes = 320;
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_DO = OFF_Q + kTileBytes;
-constexpr uint32_t OFF_K = OFF_DO + kTileBytes;   // 2 stages
-constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;  // 2 stages
-constexpr uint32_t kTilesBytes = OFF_V + 2 * kTileBytes;  // 192 KB
+constexpr int kKStages = 3;  // K~_j is read first (S) and last (dQ): deepest ring
+constexpr int kVStages = 2;
+constexpr uint32_t OFF_K = OFF_DO + kTileBytes;
+constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
+constexpr uint32_t kTilesBytes = OFF_V + kVStages * kTileBytes;  // 224 KB
 constexpr uint32_t kSmemBytes = kTilesBytes + kSmallBytes + 1024;
 
 enum : uint32_t {
   B_Q_FULL = 0, B_Q_EMPTY = 1,
-  B_KV_FULL = 2,   // 2 stages
-  B_KV_EMPTY = 4,  // 2 stages
-  B_S_FULL = 6, B_S_READ = 7, B_DP_FULL = 8, B_DS_FULL = 9,
-  B_DQ_FULL = 10, B_DQ_EMPTY = 11, B_FIN = 12
+  B_K_FULL = 2,    // kKStages
+  B_K_EMPTY = 5,   // kKStages
+  B_V_FULL = 8,    // kVStages
+  B_V_EMPTY = 10,  // kVStages
+  B_S_FULL = 12, B_S_READ = 13, B_DP_FULL = 14, B_DS_FULL = 15,
+  B_DQ_FULL = 16, B_DQ_EMPTY = 17, B_FIN = 18
 };
 
 struct DqParams {
@@ -150,9 +154,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     *abort_flag = 0;
     mbar_init(bar(B_Q_FULL), 1);
     mbar_init(bar(B_Q_EMPTY), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(B_KV_FULL + s), 1);
-      mbar_init(bar(B_KV_EMPTY + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(B_K_FULL + s), 1);
+      mbar_init(bar(B_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(B_V_FULL + s), 1);
+      mbar_init(bar(B_V_EMPTY + s), 1);
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_S_READ), kEW);
@@ -175,12 +183,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  uint32_t kv_issued = 0, q_issued = 0;
+  uint32_t k_issued = 0, v_issued = 0, q_issued = 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
-      uint32_t kv_it = 0;
+      uint32_t k_it = 0, v_it = 0;
       int items = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
@@ -192,17 +200,35 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_load_4d(base + OFF_DO, &tm_do, bar(B_Q_FULL), 0, it.h, it.i * 128, it.b);
         tma_load_4d(base + OFF_DO + kBoxBytes, &tm_do, bar(B_Q_FULL), 64, it.h, it.i * 128, it.b);
         q_issued = items + 1;
-        for (int j = first_rel(p, it); j >= 0; j = next_rel(p, it, j)) {
-          const uint32_t s = kv_it & 1;
-          if (!mbar_wait(bar(B_KV_EMPTY + s), ((kv_it >> 1) & 1) ^ 1, ab, 52)) { ok = false; break; }
-          mbar_expect_tx(bar(B_KV_FULL + s), 2 * kTileBytes);
-          const uint32_t sk = base + OFF_K + s * kTileBytes, sv = base + OFF_V + s * kTileBytes;
-          tma_load_4d(sk, &tm_k, bar(B_KV_FULL + s), 0, it.h, j * 128, it.b);
-          tma_load_4d(sk + kBoxBytes, &tm_k, bar(B_KV_FULL + s), 64, it.h, j * 128, it.b);
-          tma_load_4d(sv, &tm_v, bar(B_KV_FULL + s), 0, it.h, j * 128, it.b);
-          tma_load_4d(sv + kBoxBytes, &tm_v, bar(B_KV_FULL + s), 64, it.h, j * 128, it.b);
-          ++kv_it;
-          kv_issued = kv_it;
+        auto load_k = [&](int j) -> bool {
+          const uint32_t s = k_it % kKStages, n = k_it / kKStages;
+          if (!mbar_wait(bar(B_K_EMPTY + s), (n & 1) ^ 1, ab, 52)) return false;
+          mbar_expect_tx(bar(B_K_FULL + s), kTileBytes);
+          const uint32_t dst = base + OFF_K + s * kTileBytes;
+          tma_load_4d(dst, &tm_k, bar(B_K_FULL + s), 0, it.h, j * 128, it.b);
+          tma_load_4d(dst + kBoxBytes, &tm_k, bar(B_K_FULL + s), 64, it.h, j * 128, it.b);
+          k_issued = ++k_it;
+          return true;
+        };
+        auto load_v = [&](int j) -> bool {
+          const uint32_t s = v_it % kVStages, n = v_it / kVStages;
+          if (!mbar_wait(bar(B_V_EMPTY + s), (n & 1) ^ 1, ab, 50)) return false;
+          mbar_expect_tx(bar(B_V_FULL + s), kTileBytes);
+          const uint32_t dst = base + OFF_V + s * kTileBytes;
+          tma_load_4d(dst, &tm_v, bar(B_V_FULL + s), 0, it.h, j * 128, it.b);
+          tma_load_4d(dst + kBoxBytes, &tm_v, bar(B_V_FULL + s), 64, it.h, j * 128, it.b);
+          v_issued = ++v_it;
+          return true;
+        };
+        // K runs two tiles ahead of V in issue order
+        int jk = first_rel(p, it);
+        for (int a = 0; a < 2 && jk >= 0 && ok; ++a, jk = next_rel(p, it, jk)) ok = load_k(jk);
+        for (int j = first_rel(p, it); j >= 0 && ok; j = next_rel(p, it, j)) {
+          ok = load_v(j);
+          if (ok && jk >= 0) {
+            ok = load_k(jk);
+            jk = next_rel(p, it, jk);
+          }
         }
       }
     }
@@ -213,19 +239,28 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       constexpr uint32_t kIdTM = idesc_bf16(128, 128, 0, 1);   // TMEM (K-major) x MN-major
       const uint32_t sQ = base + OFF_Q, sDO = base + OFF_DO;
       const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
-      uint32_t kv_it = 0, steps = 0, dqc = 0;
+      uint32_t k_it = 0, v_it = 0, steps = 0, dqc = 0;
       int items = 0;
       bool ok = true;
       const uint64_t dQ = kmajor_desc(sQ), dDO = kmajor_desc(sDO);
-      auto sk_of = [&](uint32_t n) { return base + OFF_K + (n & 1) * kTileBytes; };
-      auto sv_of = [&](uint32_t n) { return base + OFF_V + (n & 1) * kTileBytes; };
+      auto sk_of = [&](uint32_t n) { return base + OFF_K + (n % kKStages) * kTileBytes; };
+      auto sv_of = [&](uint32_t n) { return base + OFF_V + (n % kVStages) * kTileBytes; };
+      auto wait_k = [&](uint32_t n) {
+        return mbar_wait(bar(B_K_FULL + n % kKStages), (n / kKStages) & 1, ab, 54);
+      };
       auto issue_s = [&](uint32_t n) {
         mma_kk128(tS, dQ, kmajor_desc(sk_of(n)), kIdKK, 0u);
         mma_commit(bar(B_S_FULL));
       };
-      auto issue_dp = [&](uint32_t n) {
-        mma_kk128(tDP, dDO, kmajor_desc(sv_of(n)), kIdKK, 0u);
+      // dP(j) with the next V tile; V_j is free again once dP(j) completes
+      auto issue_dp = [&]() -> bool {
+        if (!mbar_wait(bar(B_V_FULL + v_it % kVStages), (v_it / kVStages) & 1, ab, 56)) return false;
+        tc_fence_after();
+        mma_kk128(tDP, dDO, kmajor_desc(sv_of(v_it)), kIdKK, 0u);
         mma_commit(bar(B_DP_FULL));
+        mma_commit(bar(B_V_EMPTY + v_it % kVStages));
+        ++v_it;
+        return true;
       };
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
         const Item it = decode(p, idx);
@@ -234,28 +269,28 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int j = first_rel(p, it);
         bool first = true;
         if (j >= 0) {
-          if (!mbar_wait(bar(B_KV_FULL + (kv_it & 1)), (kv_it >> 1) & 1, ab, 54)) { ok = false; break; }
+          if (!wait_k(k_it)) { ok = false; break; }
           tc_fence_after();
-          issue_s(kv_it);
-          issue_dp(kv_it);
+          issue_s(k_it);
+          if (!issue_dp()) { ok = false; break; }
         }
         while (j >= 0) {
           const int jn = next_rel(p, it, j);
           // S(j+1) as soon as S(j) is in the element-wise warps' registers
           if (!mbar_wait(bar(B_S_READ), steps & 1, ab, 55)) { ok = false; break; }
           if (jn >= 0) {
-            if (!mbar_wait(bar(B_KV_FULL + ((kv_it + 1) & 1)), ((kv_it + 1) >> 1) & 1, ab, 56)) { ok = false; break; }
+            if (!wait_k(k_it + 1)) { ok = false; break; }
             tc_fence_after();
-            issue_s(kv_it + 1);
+            issue_s(k_it + 1);
           }
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 57)) { ok = false; break; }
           if (first && dqc > 0 && !mbar_wait(bar(B_DQ_EMPTY), (dqc - 1) & 1, ab, 58)) { ok = false; break; }
           tc_fence_after();
-          mma_tm128<true>(tDQ, tDP, mnmajor_desc(sk_of(kv_it)), kIdTM, first ? 0u : 1u);
-          mma_commit(bar(B_KV_EMPTY + (kv_it & 1)));
-          ++kv_it;
+          mma_tm128<true>(tDQ, tDP, mnmajor_desc(sk_of(k_it)), kIdTM, first ? 0u : 1u);
+          mma_commit(bar(B_K_EMPTY + k_it % kKStages));
+          ++k_it;
           // dP(j+1): dS(j) in these columns went to dQ(j) just before (issue order)
-          if (jn >= 0) issue_dp(kv_it);
+          if (jn >= 0 && !issue_dp()) { ok = false; break; }
           ++steps;
           first = false;
           j = jn;
@@ -405,8 +440,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (warp == 0 && lane == 0) {
       if (q_issued > 0) drain_wait(bar(B_Q_FULL), (q_issued - 1) & 1);
-      for (uint32_t n = (kv_issued > 2 ? kv_issued - 2 : 0); n < kv_issued; ++n)
-        drain_wait(bar(B_KV_FULL + (n & 1)), (n >> 1) & 1);
+      for (uint32_t n = (k_issued > kKStages ? k_issued - kKStages : 0); n < k_issued; ++n)
+        drain_wait(bar(B_K_FULL + n % kKStages), (n / kKStages) & 1);
+      for (uint32_t n = (v_issued > kVStages ? v_issued - kVStages : 0); n < v_issued; ++n)
+        drain_wait(bar(B_V_FULL + n % kVStages), (n / kVStages) & 1);
     }
   }
   __syncthreads();
