@@ -9,15 +9,21 @@
 // One persistent CTA per SM owns a query tile i of one (b, h) and sweeps the
 // key tiles j it may attend to; dQ~_i accumulates in tensor memory, and the
 // epilogue applies the scale and the inverse rotation and writes bf16 dq, so
-// no partial sums leave the CTA.  Roles (640 threads):
-//   warp 0      TMA producer: Q~_i and dO_i once per item, K~_j (3-stage
-//               ring, issued two tiles ahead) and V_j (2-stage ring) per step.
+// no partial sums leave the CTA.  Q~_i and dO_i are the A operands of S and
+// dP for the whole sweep, so they sit in tensor memory and every product of
+// the sweep reads only its B operand (K~_j or V_j) from shared memory.
+// Roles (640 threads):
+//   warp 0      TMA producer: K~_j and V_j per step, 3-stage rings, K issued
+//               two tiles ahead of V.
 //   warp 1      MMA issuer (one thread).
 //   warp 2      tensor-memory allocation.
 //   warps 4-19  element-wise work, four warpgroups on 32 key columns each
-//               (one query row per thread), then the dq epilogue.
+//               (one query row per thread): Q~_i / dO_i rows into tensor
+//               memory at the start of an item, P and dS per step, then the
+//               dq epilogue.
 // TMEM columns: S [0,128), dP [128,256) with dS (bf16) over it (each quarter
-// packs its dS into the first 16 of its own 32 columns), dQ~ [256,384).
+// packs its dS into the first 16 of its own 32 columns), dQ~ [256,384),
+// Q~_i [384,448), dO_i [448,512) (bf16, two per column).
 // MMA issue order per step:
 //   S(j+1) once S(j) is in registers | dQ(j) after dS(j) | dP(j+1) ...
 #include <cuda.h>
@@ -46,23 +52,20 @@ constexpr uint32_t kBoxBytes = kTileBytes / 2;
 constexpr uint32_t SOFF_BAR = 0;
 constexpr uint32_t SOFF_MISC = 256;
 constexpr uint32_t kSmallBytes = 320;
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_DO = OFF_Q + kTileBytes;
-constexpr int kKStages = 3;  // K~_j is read first (S) and last (dQ): deepest ring
-constexpr int kVStages = 2;
-constexpr uint32_t OFF_K = OFF_DO + kTileBytes;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
-constexpr uint32_t kTilesBytes = OFF_V + kVStages * kTileBytes;  // 224 KB
+constexpr uint32_t kTilesBytes = OFF_V + kVStages * kTileBytes;  // 192 KB
 constexpr uint32_t kSmemBytes = kTilesBytes + kSmallBytes + 1024;
 
 enum : uint32_t {
-  B_Q_FULL = 0, B_Q_EMPTY = 1,
-  B_K_FULL = 2,    // kKStages
-  B_K_EMPTY = 5,   // kKStages
-  B_V_FULL = 8,    // kVStages
-  B_V_EMPTY = 10,  // kVStages
-  B_S_FULL = 12, B_S_READ = 13, B_DP_FULL = 14, B_DS_FULL = 15,
-  B_DQ_FULL = 16, B_DQ_EMPTY = 17, B_FIN = 18
+  B_K_FULL = 0,    // kKStages
+  B_K_EMPTY = 3,   // kKStages
+  B_V_FULL = 6,    // kVStages
+  B_V_EMPTY = 9,   // kVStages
+  B_Q_READY = 12, B_S_FULL = 13, B_S_READ = 14, B_DP_FULL = 15, B_DS_FULL = 16,
+  B_DQ_FULL = 17, B_DQ_EMPTY = 18, B_FIN = 19
 };
 
 struct DqParams {
@@ -72,6 +75,8 @@ struct DqParams {
   const int32_t* q_lo;
   const float* lse2;   // [B, H, nT*128]: LSE * log2(e), +inf where the row has no keys
   const float* dpad;   // [B, H, nT*128]: dot(dO, O), 0 past the end
+  const __nv_bfloat16* q_rot;  // [B, S, H, D] rotated q
+  const __nv_bfloat16* d_o;    // [B, S, H, D]
   __nv_bfloat16* dq;
   DeviceStatus* status;
   int64_t S;
@@ -136,8 +141,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const DqParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -152,8 +156,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar(B_Q_FULL), 1);
-    mbar_init(bar(B_Q_EMPTY), 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(B_K_FULL + s), 1);
       mbar_init(bar(B_K_EMPTY + s), 1);
@@ -162,6 +164,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(bar(B_V_FULL + s), 1);
       mbar_init(bar(B_V_EMPTY + s), 1);
     }
+    mbar_init(bar(B_Q_READY), kEW);
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_S_READ), kEW);
     mbar_init(bar(B_DP_FULL), 1);
@@ -170,10 +173,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(bar(B_DQ_EMPTY), kEW);
     mbar_init(bar(B_FIN), 1);
     fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_do);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -183,23 +184,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  uint32_t k_issued = 0, v_issued = 0, q_issued = 0;
+  uint32_t k_issued = 0, v_issued = 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       uint32_t k_it = 0, v_it = 0;
-      int items = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
         const Item it = decode(p, idx);
-        if (items > 0 && !mbar_wait(bar(B_Q_EMPTY), (items - 1) & 1, ab, 51)) { ok = false; break; }
-        mbar_expect_tx(bar(B_Q_FULL), 2 * kTileBytes);
-        tma_load_4d(base + OFF_Q, &tm_q, bar(B_Q_FULL), 0, it.h, it.i * 128, it.b);
-        tma_load_4d(base + OFF_Q + kBoxBytes, &tm_q, bar(B_Q_FULL), 64, it.h, it.i * 128, it.b);
-        tma_load_4d(base + OFF_DO, &tm_do, bar(B_Q_FULL), 0, it.h, it.i * 128, it.b);
-        tma_load_4d(base + OFF_DO + kBoxBytes, &tm_do, bar(B_Q_FULL), 64, it.h, it.i * 128, it.b);
-        q_issued = items + 1;
         auto load_k = [&](int j) -> bool {
           const uint32_t s = k_it % kKStages, n = k_it / kKStages;
           if (!mbar_wait(bar(B_K_EMPTY + s), (n & 1) ^ 1, ab, 52)) return false;
@@ -235,45 +228,43 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
-      constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);   // K-major x K-major
+      constexpr uint32_t kIdTK = idesc_bf16(128, 128, 0, 0);   // TMEM (K-major) x K-major
       constexpr uint32_t kIdTM = idesc_bf16(128, 128, 0, 1);   // TMEM (K-major) x MN-major
-      const uint32_t sQ = base + OFF_Q, sDO = base + OFF_DO;
-      const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
-      uint32_t k_it = 0, v_it = 0, steps = 0, dqc = 0;
-      int items = 0;
+      const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256, tQ = tmem + 384,
+                     tDO = tmem + 448;
+      uint32_t k_it = 0, v_it = 0, steps = 0, dqc = 0, qrc = 0;
       bool ok = true;
-      const uint64_t dQ = kmajor_desc(sQ), dDO = kmajor_desc(sDO);
       auto sk_of = [&](uint32_t n) { return base + OFF_K + (n % kKStages) * kTileBytes; };
       auto sv_of = [&](uint32_t n) { return base + OFF_V + (n % kVStages) * kTileBytes; };
       auto wait_k = [&](uint32_t n) {
         return mbar_wait(bar(B_K_FULL + n % kKStages), (n / kKStages) & 1, ab, 54);
       };
       auto issue_s = [&](uint32_t n) {
-        mma_kk128(tS, dQ, kmajor_desc(sk_of(n)), kIdKK, 0u);
+        mma_tk128(tS, tQ, kmajor_desc(sk_of(n)), kIdTK, 0u);
         mma_commit(bar(B_S_FULL));
       };
       // dP(j) with the next V tile; V_j is free again once dP(j) completes
       auto issue_dp = [&]() -> bool {
         if (!mbar_wait(bar(B_V_FULL + v_it % kVStages), (v_it / kVStages) & 1, ab, 56)) return false;
         tc_fence_after();
-        mma_kk128(tDP, dDO, kmajor_desc(sv_of(v_it)), kIdKK, 0u);
+        mma_tk128(tDP, tDO, kmajor_desc(sv_of(v_it)), kIdTK, 0u);
         mma_commit(bar(B_DP_FULL));
         mma_commit(bar(B_V_EMPTY + v_it % kVStages));
         ++v_it;
         return true;
       };
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
         const Item it = decode(p, idx);
-        if (!mbar_wait(bar(B_Q_FULL), items & 1, ab, 53)) { ok = false; break; }
-        tc_fence_after();
         int j = first_rel(p, it);
+        if (j < 0) continue;  // nothing to do: the element-wise warps write zeros
         bool first = true;
-        if (j >= 0) {
-          if (!wait_k(k_it)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(k_it);
-          if (!issue_dp()) { ok = false; break; }
-        }
+        // Q~_i and dO_i in tensor memory (and the previous item's dQ read out)
+        if (!mbar_wait(bar(B_Q_READY), qrc & 1, ab, 53)) { ok = false; break; }
+        ++qrc;
+        if (!wait_k(k_it)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(k_it);
+        if (!issue_dp()) { ok = false; break; }
         while (j >= 0) {
           const int jn = next_rel(p, it, j);
           // S(j+1) as soon as S(j) is in the element-wise warps' registers
@@ -296,11 +287,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           j = jn;
         }
         if (!ok) break;
-        if (!first) {
-          mma_commit(bar(B_DQ_FULL));
-          ++dqc;
-        }
-        mma_commit(bar(B_Q_EMPTY));
+        mma_commit(bar(B_DQ_FULL));
+        ++dqc;
       }
     }
   } else if (warp >= 4) {
@@ -311,6 +299,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tS = tmem + lane_base + 32u * w;
     const uint32_t tDP = tmem + lane_base + 128u + 32u * w;
     const uint32_t tDQ = tmem + lane_base + 256u + 32u * w;
+    const uint32_t tQ = tmem + lane_base + 384u;
+    const uint32_t tDO = tmem + lane_base + 448u;
     const size_t hstride = (size_t)p.n_tiles * 128;
     uint32_t steps = 0, dqc = 0;
     bool ok = true;
@@ -323,6 +313,29 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const float L2 = p.lse2[lrow];
       const float Dq = p.dpad[lrow];
       int n = 0;
+      if (first_rel(p, it) >= 0) {
+        // this quarter's 32 values of the row of Q~_i and of dO_i -> 16 columns each
+        uint32_t qa[16], da[16];
+        if (q_ok) {
+          const size_t off = (((size_t)it.b * p.S + q) * p.H + it.h) * kD + 32 * w;
+          const uint4* qs4 = reinterpret_cast<const uint4*>(p.q_rot + off);
+          const uint4* ds4 = reinterpret_cast<const uint4*>(p.d_o + off);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 a = qs4[c], d = ds4[c];
+            qa[4 * c] = a.x; qa[4 * c + 1] = a.y; qa[4 * c + 2] = a.z; qa[4 * c + 3] = a.w;
+            da[4 * c] = d.x; da[4 * c + 1] = d.y; da[4 * c + 2] = d.z; da[4 * c + 3] = d.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) qa[c] = da[c] = 0u;
+        }
+        tmem_st16(tQ + 16 * w, qa);
+        tmem_st16(tDO + 16 * w, da);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_Q_READY));
+      }
       for (int j = it.lo; j <= it.hi; ++j) {
         if (!rel(p, it, j)) continue;
         const int64_t k0 = (int64_t)j * 128 + 32 * w;  // first key column of this quarter
@@ -439,7 +452,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       drain_wait(bar(B_FIN), 0);
     }
     if (warp == 0 && lane == 0) {
-      if (q_issued > 0) drain_wait(bar(B_Q_FULL), (q_issued - 1) & 1);
       for (uint32_t n = (k_issued > kKStages ? k_issued - kKStages : 0); n < k_issued; ++n)
         drain_wait(bar(B_K_FULL + n % kKStages), (n / kKStages) & 1);
       for (uint32_t n = (v_issued > kVStages ? v_issued - kVStages : 0); n < v_issued; ++n)
@@ -457,13 +469,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 cudaError_t launch_sm100_bwd_dq(const Problem& pb, const Workspace& ws, const void* v,
                                 const void* d_o, void* dq, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
+  CUtensorMap tk, tv;
+  if (!make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
   DqParams p{};
+  p.q_rot = static_cast<const __nv_bfloat16*>(ws.q_rot);
+  p.d_o = static_cast<const __nv_bfloat16*>(d_o);
   p.seg = pb.seg;
   p.tmin = ws.tile_min;
   p.tmax = ws.tile_max;
@@ -491,7 +503,7 @@ cudaError_t launch_sm100_bwd_dq(const Problem& pb, const Workspace& ws, const vo
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
-  attn_bwd_dq_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, p);
+  attn_bwd_dq_kernel<<<grid, kThreads, kSmemBytes, st>>>(tk, tv, p);
   note_launches(1);
   return cudaGetLastError();
 }

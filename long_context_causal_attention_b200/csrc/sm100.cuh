@@ -255,6 +255,17 @@ __device__ __forceinline__ void mma_tm128(uint32_t d, uint32_t a_tmem, uint64_t 
   }
 }
 
+// D (+)= A * B^T over K = 128 with A (bf16) in tensor memory (K packed two per
+// column, 8 columns per k-step) and B a K-major tile.
+__device__ __forceinline__ void mma_tk128(uint32_t d, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t off = (uint64_t)(((kk >> 2) * kOperandBoxBytes + (kk & 3) * 32) >> 4);
+    mma_ts(d, a_tmem + (uint32_t)(kk * 8), b_desc + off, idesc, kk > 0 ? 1u : acc);
+  }
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
