@@ -36,6 +36,13 @@ METRIC = "causal attn fwd+bwd TFLOP/s (32x128 heads, bf16) and % of B200 BF16 pe
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 L2_BYTES = 126 * 2 ** 20
 
+# DRAM traffic of one attn_bwd_dkdv_kernel launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from an ncu capture of the 16K-token profiling case,
+# scaled to each workload by its tile pairs; valid only for the kernel source
+# it was taken on (sha256 of the kernel file and the headers it includes).
+DKDV_TRAFFIC = {"bytes_per_tile_pair": None, "source_sha256": None,
+                "profile": "profiles/attn_bwd_dkdv_kernel_prof_16k.md"}
+
 
 def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
     total = 0
@@ -105,6 +112,57 @@ def dist_setup():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws an independent problem of the same shape."""
+    return seed + rank
+
+
+def max_over_ranks(values, ws: int, device):
+    """Element-wise max of a list of floats over all ranks (identity at ws=1)."""
+    if ws == 1:
+        return [float(x) for x in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(flops_per_rank_step: float, ws: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return flops_per_rank_step * ws / (ms_per_step * 1e-3) / 1e12
+
+
+def tile_pairs(seg: np.ndarray, heads: int, causal: bool = True, tile: int = 128) -> int:
+    """(query tile, key tile) pairs that share a segment id range, over all
+    rows and heads: the units the dK/dV kernel streams."""
+    total = 0
+    for row in seg:
+        n = (len(row) + tile - 1) // tile
+        lo = np.full(n, np.iinfo(np.int64).max)
+        hi = np.full(n, np.iinfo(np.int64).min)
+        for t in range(n):
+            r = row[t * tile:(t + 1) * tile]
+            r = r[r >= 0]
+            if len(r):
+                lo[t], hi[t] = r.min(), r.max()
+        valid = hi >= lo
+        for qt in np.nonzero(valid)[0]:
+            kt = slice(0, qt + 1) if causal else slice(0, n)
+            total += int(np.count_nonzero(valid[kt] & (lo[kt] <= hi[qt]) & (hi[kt] >= lo[qt])))
+    return total * heads
+
+
+def kernel_source_sha256(name: str) -> str:
+    import hashlib
+    d = os.path.join(ROOT, "long_context_causal_attention_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (name, "sm100.cuh", "common.cuh", "internal.h"):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def time_oracle_sample(w, seg, rows: int, seed: int):
@@ -192,7 +250,7 @@ def ours(args):
             dist.barrier()
 
     w = WORKLOADS[args.workload]
-    seed = args.seed + rank
+    seed = rank_seed(args.seed, rank)
     seg = segment_ids(w, seed=seed)
     single = w.segments == "single"
     seg_d = None if single else torch.as_tensor(seg, dtype=torch.int32, device=dev)
@@ -221,7 +279,7 @@ def ours(args):
     torch.cuda.synchronize()
 
     # per-step events around the main kernels (recorded by the library)
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     for evs in kev:
         for e in evs:
             e.record(stream)
@@ -247,12 +305,10 @@ def ours(args):
     ms = start.elapsed_time(stop)
     fwd_k = sum(e[0].elapsed_time(e[1]) for e in kev) / args.steps
     bwd_k = sum(e[2].elapsed_time(e[3]) for e in kev) / args.steps
-    if ws > 1:
-        tt = torch.tensor([ms, fwd_k, bwd_k], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, fwd_k, bwd_k = tt.tolist()
+    dkdv_k = sum(e[2].elapsed_time(e[4]) for e in kev) / args.steps
+    ms, fwd_k, bwd_k, dkdv_k = max_over_ranks([ms, fwd_k, bwd_k, dkdv_k], ws, dev)
     ms_step = ms / args.steps
-    value = step_flops * ws / (ms_step * 1e-3) / 1e12
+    value = job_tflops(step_flops, ws, ms_step)
 
     # end to end through the public API: pinned host inputs in, gradients out
     e2e = None
@@ -279,25 +335,35 @@ def ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = e0.elapsed_time(e1)
-        if ws > 1:
-            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = tt.item()
+        ems, = max_over_ranks([e0.elapsed_time(e1)], ws, dev)
         nb = q.numel() * q.element_size()
-        e2e = {"value": step_flops * ws / (ems / n_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_tflops(step_flops, ws, ems / n_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 3 * nb, "steps": n_e2e}
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    # dominant kernel: dK/dV, whose four GEMMs per kept pair (S^T, dP^T, dV,
+    # dK) are all algorithmic work: 8*D flops per pair and head
+    dkdv_flops = 8.0 * w.head_dim * w.heads * pairs
+    achieved = dkdv_flops / (dkdv_k * 1e-3) / 1e12
+    traffic = None
+    units = tile_pairs(seg, w.heads, w.causal)
+    if (DKDV_TRAFFIC["bytes_per_tile_pair"] and
+            DKDV_TRAFFIC["source_sha256"] == kernel_source_sha256("attn_bwd_sm100.cu")):
+        traffic = DKDV_TRAFFIC["bytes_per_tile_pair"] * units
     bwd_flops = 2.5 * fwd_flops
-    achieved = bwd_flops / (bwd_k * 1e-3) / 1e12
+    dq_k = bwd_k - dkdv_k
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
-                "kernel": "backward main kernel(s)",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "attn_bwd_dkdv_kernel",
+                "algorithmic": "8*D*H flops per kept (query, key) pair: S^T, dP^T, dV, dK",
+                "tile_pairs": units,
                 "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "dkdv_kernel_ms": dkdv_k, "dq_kernel_ms": dq_k, "fwd_kernel_ms": fwd_k,
                 "fwd_kernel_tflops": fwd_flops / (fwd_k * 1e-3) / 1e12,
-                "fwd_kernel_ms": fwd_k, "bwd_kernel_ms": bwd_k}
+                "bwd_kernels_tflops": bwd_flops / (bwd_k * 1e-3) / 1e12,
+                "dq_kernel_tflops_incl_recompute": 6.0 * w.head_dim * w.heads * pairs
+                / (dq_k * 1e-3) / 1e12}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

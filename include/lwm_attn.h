@@ -166,12 +166,14 @@ const char* lwm_status_string(lwm_status status);
  * lwm_attn_set_timing_events: cudaEvent_t handles (as void*, any may be
  * NULL) that the next calls record on their stream immediately before and
  * after the main attention kernel(s) of lwm_attn_fwd / lwm_attn_bwd, so the
- * caller can time those kernels alone.  The handles stay in effect until
+ * caller can time those kernels alone; bwd_split is recorded between the
+ * dK/dV kernel and the dQ kernel of the tensor-core backward (not by the
+ * fp32 / head_dim 64 backward).  The handles stay in effect until
  * replaced; pass NULLs to stop.  Process-wide; guarded by a mutex.
  * lwm_attn_kernel_launches: number of kernels this library has launched
  * since it was loaded. */
 void lwm_attn_set_timing_events(void* fwd_start, void* fwd_stop, void* bwd_start,
-                                void* bwd_stop);
+                                void* bwd_stop, void* bwd_split);
 uint64_t lwm_attn_kernel_launches(void);
 
 #ifdef __cplusplus

@@ -73,7 +73,7 @@ def _load():
     lib.lwm_attn_read_status.restype = ctypes.c_int
     lib.lwm_status_string.argtypes = [ctypes.c_int]
     lib.lwm_status_string.restype = ctypes.c_char_p
-    lib.lwm_attn_set_timing_events.argtypes = [P, P, P, P]
+    lib.lwm_attn_set_timing_events.argtypes = [P, P, P, P, P]
     lib.lwm_attn_set_timing_events.restype = None
     lib.lwm_attn_fwd_noalloc.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P]
     lib.lwm_attn_fwd_noalloc.restype = ctypes.c_int
@@ -218,9 +218,11 @@ def lwm_attn_read_status(workspace, stream=None) -> int:
     return int(_lib.lwm_attn_read_status(workspace.data_ptr(), _stream(stream)))
 
 
-def lwm_attn_set_timing_events(fwd_start=None, fwd_stop=None, bwd_start=None, bwd_stop=None):
+def lwm_attn_set_timing_events(fwd_start=None, fwd_stop=None, bwd_start=None, bwd_stop=None,
+                               bwd_split=None):
     """Have the next calls record these torch.cuda.Event objects around their
-    main attention kernels (None leaves that slot empty)."""
+    main attention kernels, bwd_split between the two backward kernels (None
+    leaves that slot empty)."""
     def handle(e):
         if e is None:
             return None
@@ -228,7 +230,7 @@ def lwm_attn_set_timing_events(fwd_start=None, fwd_stop=None, bwd_start=None, bw
             e.record()
         return ctypes.c_void_p(e.cuda_event)
     _lib.lwm_attn_set_timing_events(handle(fwd_start), handle(fwd_stop), handle(bwd_start),
-                                    handle(bwd_stop))
+                                    handle(bwd_stop), handle(bwd_split))
 
 
 def lwm_attn_kernel_launches() -> int:

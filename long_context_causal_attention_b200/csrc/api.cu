@@ -16,7 +16,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 namespace {
 std::atomic<uint64_t> g_launches{0};
 std::mutex g_events_mu;
-cudaEvent_t g_events[4] = {nullptr, nullptr, nullptr, nullptr};
+cudaEvent_t g_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 
 void record_event(int which, cudaStream_t st) {
   std::lock_guard<std::mutex> lk(g_events_mu);
@@ -199,6 +199,7 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
     if (e != cudaSuccess) return LWM_ERR_CUDA;
     record_event(2, st);
     e = launch_sm100_bwd_dkdv(p, w, v, d_o, dk, dv, st);
+    record_event(4, st);
     if (e == cudaSuccess) e = launch_sm100_bwd_dq(p, w, v, d_o, dq, st);
     record_event(3, st);
     return cuda_status(e);
@@ -250,12 +251,13 @@ const char* lwm_status_string(lwm_status status) {
 }
 
 void lwm_attn_set_timing_events(void* fwd_start, void* fwd_stop, void* bwd_start,
-                                void* bwd_stop) {
+                                void* bwd_stop, void* bwd_split) {
   std::lock_guard<std::mutex> lk(g_events_mu);
   g_events[0] = static_cast<cudaEvent_t>(fwd_start);
   g_events[1] = static_cast<cudaEvent_t>(fwd_stop);
   g_events[2] = static_cast<cudaEvent_t>(bwd_start);
   g_events[3] = static_cast<cudaEvent_t>(bwd_stop);
+  g_events[4] = static_cast<cudaEvent_t>(bwd_split);
 }
 
 uint64_t lwm_attn_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
