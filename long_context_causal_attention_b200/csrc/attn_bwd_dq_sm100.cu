@@ -12,12 +12,13 @@
 // no partial sums leave the CTA.  Q~_i and dO_i are the A operands of S and
 // dP for the whole sweep, so they sit in tensor memory and every product of
 // the sweep reads only its B operand (K~_j or V_j) from shared memory.
-// Roles (640 threads):
+// Roles (576 threads, so that each may hold 112 registers):
 //   warp 0      TMA producer: K~_j and V_j per step, 3-stage rings, K issued
 //               two tiles ahead of V.
-//   warp 1      MMA issuer (one thread).
-//   warp 2      tensor-memory allocation.
-//   warps 4-19  element-wise work, four warpgroups on 32 key columns each
+//   warp 1      MMA issuer (one thread); the whole warp allocates and frees
+//               the tensor memory.
+//   warps 2-17  element-wise work, four groups of four warps (one per TMEM
+//               lane quarter, warp % 4) on 32 key columns each
 //               (one query row per thread): Q~_i / dO_i rows into tensor
 //               memory at the start of an item, P and dS per step, then the
 //               dq epilogue.
@@ -44,14 +45,15 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 640;   // 4 control warps + 4 element-wise warpgroups
+constexpr int kThreads = 576;   // 2 control warps + 4 element-wise warpgroups
 constexpr int kEW = 512;        // element-wise threads
 constexpr uint32_t kTileBytes = 128 * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;
 
 constexpr uint32_t SOFF_BAR = 0;
 constexpr uint32_t SOFF_MISC = 256;
-constexpr uint32_t kSmallBytes = 320;
+constexpr uint32_t SOFF_FREQ = 320;  // 64 RoPE frequencies, fp64
+constexpr uint32_t kSmallBytes = SOFF_FREQ + (kD / 2) * 8;
 constexpr int kKStages = 3;
 constexpr int kVStages = 3;
 constexpr uint32_t OFF_K = 0;
@@ -150,6 +152,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem_raw + SOFF_MISC);
+  double* freq = reinterpret_cast<double*>(smem_raw + SOFF_FREQ);
   const Abort ab{abort_flag, p.status};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.B * p.H * p.n_tiles;
@@ -164,19 +167,21 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       mbar_init(bar(B_V_FULL + s), 1);
       mbar_init(bar(B_V_EMPTY + s), 1);
     }
-    mbar_init(bar(B_Q_READY), kEW);
+    mbar_init(bar(B_Q_READY), kEW / 32);
     mbar_init(bar(B_S_FULL), 1);
-    mbar_init(bar(B_S_READ), kEW);
+    mbar_init(bar(B_S_READ), kEW / 32);
     mbar_init(bar(B_DP_FULL), 1);
-    mbar_init(bar(B_DS_FULL), kEW);
+    mbar_init(bar(B_DS_FULL), kEW / 32);
     mbar_init(bar(B_DQ_FULL), 1);
-    mbar_init(bar(B_DQ_EMPTY), kEW);
+    mbar_init(bar(B_DQ_EMPTY), kEW / 32);
     mbar_init(bar(B_FIN), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 2) {
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + kD / 2 && p.rotate)
+    freq[threadIdx.x - 64] = rope_freq(threadIdx.x - 64, kD, p.log2_theta);
+  if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -291,9 +296,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         ++dqc;
       }
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------- element-wise work
-    const int w = (warp - 4) >> 2;                // key-column quarter
+    const int w = (warp - 2) >> 2;                // key-column quarter
     const int row = ((warp & 3) << 5) + lane;     // TMEM lane = query in the tile
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + 32u * w;
@@ -334,7 +339,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tmem_st16(tDO + 16 * w, da);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_Q_READY));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_Q_READY));
       }
       for (int j = it.lo; j <= it.hi; ++j) {
         if (!rel(p, it, j)) continue;
@@ -373,7 +379,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tmem_ld32(tS, r);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(bar(B_S_READ));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_READ));
         float pr[32];
         if (partial) {
 #pragma unroll
@@ -398,7 +405,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_DS_FULL));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_DS_FULL));
         ++steps;
         ++n;
       }
@@ -420,14 +428,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       tmem_ld32(tDQ, r);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(B_DQ_EMPTY));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_DQ_EMPTY));
       uint32_t out[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
         if (p.rotate) {
           float c, s;
-          rope_cos_sin_fast(q, rope_freq(16 * w + u, kD, p.log2_theta), &c, &s);
+          rope_cos_sin_fast(q, freq[16 * w + u], &c, &s);
           const float a2 = a * c + b * s, b2 = b * c - a * s;
           a = a2;
           b = b2;
@@ -459,7 +468,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
   }
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -13,23 +13,27 @@
 //
 // One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
 // walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
-// tensor memory for the whole walk.  Roles (640 threads):
+// tensor memory for the whole walk.  Roles (576 threads, so that each may
+// hold 112 registers):
 //   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i, and the
 //               tile's LSE*log2(e) and D (1-D bulk copies) per step, through a
 //               2-stage ring.
-//   warp 1      MMA issuer (one thread).
-//   warp 2      tensor-memory allocation.
-//   warps 4-19  element-wise work, four warpgroups on 32 query columns each:
-//               P^T and dS^T (bf16) back into tensor memory, then the dK/dV
-//               epilogue (scale, inverse RoPE, bf16).
-// TMEM columns: S^T [0,128) with P^T over it, dP^T [128,256) with dS^T over
-// it, dV [256,384), dK [384,512).  A quarter's bf16 result goes into the
-// first 16 columns of that quarter's own 32-column range, so no warpgroup
-// overwrites columns another still reads; dV and dK take P^T and dS^T
-// straight from tensor memory.
+//   warp 1      MMA issuer (one thread); the whole warp allocates and frees
+//               the tensor memory.
+//   warps 2-17  element-wise work, four groups of four warps (one per TMEM
+//               lane quarter, warp % 4) on 32 query columns each:
+//               P^T (bf16) into shared memory, dS^T (bf16) back into tensor
+//               memory, then the dK/dV epilogue (scale, inverse RoPE, bf16).
+// TMEM columns: S^T [0,128), dP^T [128,256) with dS^T over it, dV [256,384),
+// dK [384,512).  A quarter's dS^T goes into the first 16 columns of that
+// quarter's own 32-column range, so no warpgroup overwrites columns another
+// still reads; dK takes dS^T straight from tensor memory, dV takes P^T from
+// a 128-byte-swizzled K-major shared-memory tile.
 // MMA issue order per step:
-//   dP(i) | dV(i) after P(i) | S(i+1) | dK(i) after dS(i) | dP(i+1) ...
-// so the exponentials of step i+1 overlap dK(i) and dP(i+1).
+//   dP(i) | S(i+1) once S^T(i) is in registers | dV(i) after P(i) |
+//   dK(i) after dS(i) | dP(i+1) ...
+// S^T(i+1) is computed while the element-wise warps are still on the
+// exponentials of step i, so they find it ready when they finish dS(i).
 #include <cuda.h>
 
 #include <mutex>
@@ -48,32 +52,37 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 640;   // 4 control warps + 4 element-wise warpgroups
+constexpr int kThreads = 576;   // 2 control warps + 4 element-wise warpgroups
 constexpr int kEW = 512;        // element-wise threads
 constexpr uint32_t kTileBytes = 128 * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;
 
-// Small region at the start of dynamic shared memory (16-byte aligned):
-constexpr uint32_t SOFF_BAR = 0;                       // mbarriers
-constexpr uint32_t SOFF_MISC = 256;                    // TMEM base, abort flag
-constexpr uint32_t SOFF_LD = 320;                      // 2 stages x (LSE2[128], D[128]) fp32
-constexpr uint32_t kLdStageBytes = 2 * 128 * 4;
-constexpr uint32_t kSmallBytes = SOFF_LD + 2 * kLdStageBytes;
-// Tiles after it, from the next 1024-byte boundary (128-byte swizzle atoms):
+// Tiles from the first 1024-byte boundary of dynamic shared memory (128-byte
+// swizzle atoms):
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = OFF_K + kTileBytes;
 constexpr uint32_t OFF_Q = OFF_V + kTileBytes;       // 2 stages
 constexpr uint32_t OFF_DO = OFF_Q + 2 * kTileBytes;  // 2 stages
-constexpr uint32_t kTilesBytes = OFF_DO + 2 * kTileBytes;  // 192 KB
-constexpr uint32_t kSmemBytes = kTilesBytes + kSmallBytes + 1024;
+constexpr uint32_t OFF_P = OFF_DO + 2 * kTileBytes;  // P^T, K-major
+constexpr uint32_t kTilesBytes = OFF_P + kTileBytes;  // 224 KB
+// Small region after the tiles (16-byte aligned):
+constexpr uint32_t SOFF_BAR = 0;                       // mbarriers
+constexpr uint32_t SOFF_MISC = 256;                    // TMEM base, abort flag
+constexpr uint32_t SOFF_LD = 320;                      // 2 stages x (LSE2[128], D[128]) fp32
+constexpr uint32_t kLdStageBytes = 2 * 128 * 4;
+constexpr uint32_t SOFF_FREQ = SOFF_LD + 2 * kLdStageBytes;  // 64 RoPE frequencies, fp64
+constexpr uint32_t kSmallBytes = SOFF_FREQ + (kD / 2) * 8;
+constexpr uint32_t kSmemBytes = 232448;                // the sm_100 per-block maximum
+static_assert(kTilesBytes + kSmallBytes <= kSmemBytes, "shared memory layout");
 
 enum : uint32_t {
   B_KV_FULL = 0, B_KV_EMPTY = 1,
   B_QD_FULL = 2,   // 2 stages
   B_QD_EMPTY = 4,  // 2 stages
   B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_DS_FULL = 9,
-  B_DKV_FULL = 10, B_DKV_EMPTY = 11, B_FIN = 12
+  B_DKV_FULL = 10, B_DKV_EMPTY = 11, B_FIN = 12, B_S_READ = 13, B_PT_FREE = 14
 };
+constexpr uint32_t kEWWarps = kEW / 32;  // element-wise barriers take one arrival per warp
 
 struct BwdParams {
   const int32_t* seg;
@@ -147,12 +156,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const BwdParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + kSmallBytes + 1023u) & ~1023u;
-  const uint32_t bar0 = raw + SOFF_BAR;
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t small = base + kTilesBytes;
+  if (small + kSmallBytes > raw + kSmemBytes) {  // same outcome in every thread
+    if (threadIdx.x == 0) report_status(p.status, LWM_ERR_UNSUPPORTED, 0);
+    return;
+  }
+  uint8_t* small_ptr = smem_raw + (small - raw);
+  const uint32_t bar0 = small + SOFF_BAR;
   auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem_raw + SOFF_MISC);
-  const float* ld_smem = reinterpret_cast<const float*>(smem_raw + SOFF_LD);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(small_ptr + SOFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small_ptr + SOFF_MISC);
+  const float* ld_smem = reinterpret_cast<const float*>(small_ptr + SOFF_LD);
+  double* freq = reinterpret_cast<double*>(small_ptr + SOFF_FREQ);
   const Abort ab{abort_flag, p.status};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.B * p.H * p.n_tiles;
@@ -167,18 +183,22 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_DP_FULL), 1);
-    mbar_init(bar(B_P_FULL), kEW);
-    mbar_init(bar(B_DS_FULL), kEW);
+    mbar_init(bar(B_P_FULL), kEWWarps);
+    mbar_init(bar(B_DS_FULL), kEWWarps);
     mbar_init(bar(B_DKV_FULL), 1);
-    mbar_init(bar(B_DKV_EMPTY), kEW);
+    mbar_init(bar(B_DKV_EMPTY), kEWWarps);
     mbar_init(bar(B_FIN), 1);
+    mbar_init(bar(B_S_READ), kEWWarps);
+    mbar_init(bar(B_PT_FREE), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
   }
-  if (warp == 2) {
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + kD / 2 && p.rotate)
+    freq[threadIdx.x - 64] = rope_freq(threadIdx.x - 64, kD, p.log2_theta);
+  if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -216,7 +236,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           tma_load_4d(dq + kBoxBytes, &tm_q, bar(B_QD_FULL + s), 64, it.h, i * 128, it.b);
           tma_load_4d(dd, &tm_do, bar(B_QD_FULL + s), 0, it.h, i * 128, it.b);
           tma_load_4d(dd + kBoxBytes, &tm_do, bar(B_QD_FULL + s), 64, it.h, i * 128, it.b);
-          const uint32_t ld = raw + SOFF_LD + s * kLdStageBytes;
+          const uint32_t ld = small + SOFF_LD + s * kLdStageBytes;
           bulk_load(ld, lse2 + (size_t)i * 128, 512, bar(B_QD_FULL + s));
           bulk_load(ld + 512, dpad + (size_t)i * 128, 512, bar(B_QD_FULL + s));
           ++q_it;
@@ -229,18 +249,25 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);   // K-major x K-major
-      constexpr uint32_t kIdTM = idesc_bf16(128, 128, 0, 1);   // TMEM (K-major) x MN-major
+      constexpr uint32_t kIdKM = idesc_bf16(128, 128, 0, 1);   // K-major (smem or TMEM) x MN-major
       const uint32_t sK = base + OFF_K, sV = base + OFF_V;
       const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
-      uint32_t q_it = 0, steps = 0, dkv = 0;
+      uint32_t q_it = 0, steps = 0, dkv = 0, s_issued = 0;
       int items = 0;
       bool ok = true;
-      const uint64_t dK = kmajor_desc(sK), dV = kmajor_desc(sV);
+      const uint64_t dK = kmajor_desc(sK), dV = kmajor_desc(sV), dP = kmajor_desc(base + OFF_P);
       auto sq_of = [&](uint32_t n) { return base + OFF_Q + (n & 1) * kTileBytes; };
       auto sdo_of = [&](uint32_t n) { return base + OFF_DO + (n & 1) * kTileBytes; };
-      auto issue_s = [&](uint32_t n) {
+      // S^T(n) into columns [0,128), once every element-wise warp holds the
+      // previous S^T in registers and Q~(n) has landed.
+      auto issue_s = [&](uint32_t n) -> bool {
+        if (s_issued > 0 && !mbar_wait(bar(B_S_READ), (s_issued - 1) & 1, ab, 25)) return false;
+        if (!mbar_wait(bar(B_QD_FULL + (n & 1)), (n >> 1) & 1, ab, 24)) return false;
+        tc_fence_after();
         mma_kk128(tS, dK, kmajor_desc(sq_of(n)), kIdKK, 0u);
         mma_commit(bar(B_S_FULL));
+        ++s_issued;
+        return true;
       };
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
         const Item it = decode(p, idx);
@@ -248,29 +275,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tc_fence_after();
         int i = rel(p, it, it.lo) ? it.lo : next_rel(p, it, it.lo);
         bool first = true;
-        if (i >= 0) {
-          if (!mbar_wait(bar(B_QD_FULL + (q_it & 1)), (q_it >> 1) & 1, ab, 24)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(q_it);
-        }
+        if (i >= 0 && !issue_s(q_it)) { ok = false; break; }
         while (i >= 0) {
           // dP^T(i): dS^T(i-1) in these columns went to dK(i-1), issued before
           mma_kk128(tDP, dV, kmajor_desc(sdo_of(q_it)), kIdKK, 0u);
           mma_commit(bar(B_DP_FULL));
+          const int inext = next_rel(p, it, i);
+          if (inext >= 0 && !issue_s(q_it + 1)) { ok = false; break; }
           if (first && dkv > 0 && !mbar_wait(bar(B_DKV_EMPTY), (dkv - 1) & 1, ab, 26)) { ok = false; break; }
           if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 27)) { ok = false; break; }
           tc_fence_after();
-          mma_tm128<true>(tDV, tS, mnmajor_desc(sdo_of(q_it)), kIdTM, first ? 0u : 1u);
-          // S^T(i+1) now: dV(i) has taken P^T(i) from these columns (issue order)
-          const int inext = next_rel(p, it, i);
-          if (inext >= 0) {
-            if (!mbar_wait(bar(B_QD_FULL + ((q_it + 1) & 1)), ((q_it + 1) >> 1) & 1, ab, 29)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(q_it + 1);
-          }
+          mma_km128(tDV, dP, mnmajor_desc(sdo_of(q_it)), kIdKM, first ? 0u : 1u);
+          mma_commit(bar(B_PT_FREE));
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 28)) { ok = false; break; }
           tc_fence_after();
-          mma_tm128<true>(tDK, tDP, mnmajor_desc(sq_of(q_it)), kIdTM, first ? 0u : 1u);
+          mma_tm128<true>(tDK, tDP, mnmajor_desc(sq_of(q_it)), kIdKM, first ? 0u : 1u);
           mma_commit(bar(B_QD_EMPTY + (q_it & 1)));
           ++q_it;
           ++steps;
@@ -285,15 +304,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         mma_commit(bar(B_KV_EMPTY));
       }
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------- element-wise work
-    const int w = (warp - 4) >> 2;                // query-column quarter
+    const int w = (warp - 2) >> 2;                // query-column quarter
     const int row = ((warp & 3) << 5) + lane;     // TMEM lane = key in the tile
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + 32u * w;
     const uint32_t tDP = tmem + lane_base + 128u + 32u * w;
     const uint32_t tDV = tmem + lane_base + 256u + 32u * w;
     const uint32_t tDK = tmem + lane_base + 384u + 32u * w;
+    // this thread's 64 bytes of the P^T tile: key row `row`, query columns
+    // 32w..32w+31 = 16-byte chunks 4(w&1)..4(w&1)+3 of box w>>1, swizzled
+    const uint32_t sProw = base + OFF_P + (uint32_t)(w >> 1) * kBoxBytes + (uint32_t)row * 128u;
+    const uint32_t chunk0 = (uint32_t)(w & 1) * 4u, swz = (uint32_t)row & 7u;
     uint32_t steps = 0, dkv = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
@@ -347,6 +370,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           uint32_t r[32];
           tmem_ld32(tS, r);
           tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_S_READ));  // S^T(i+1) may overwrite the columns now
           const float4* l4 = reinterpret_cast<const float4*>(lse2);
           if (partial) {
 #pragma unroll
@@ -375,33 +401,47 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
-          tmem_st16(tS, pk);  // first 16 of this quarter's own 32 columns
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(B_P_FULL));
-        // ---- dS^T = P^T o (dP^T - D[q]) back into tensor memory ----
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 32 + w))) { ok = false; break; }
-        tc_fence_after();
-        {
-          uint32_t r[32];
-          tmem_ld32(tDP, r);
-          tmem_wait_ld();
-          const float4* d4 = reinterpret_cast<const float4*>(dsum);
-          uint32_t pk[16];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 Dv = d4[u];
-            pk[2 * u] = pack_bf16(pr[4 * u] * (__uint_as_float(r[4 * u]) - Dv.x),
-                                  pr[4 * u + 1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
-            pk[2 * u + 1] = pack_bf16(pr[4 * u + 2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
-                                      pr[4 * u + 3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
+          // dV(i-1) has read P^T(i-1) from the tile
+          if (steps > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(bar(B_PT_FREE), (steps - 1) & 1, ab, 42 + w))) {
+            ok = false;
+            break;
           }
-          tmem_st16(tDP, pk);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_shared_v4(sProw + (((chunk0 + c) ^ swz) << 4), pk[4 * c], pk[4 * c + 1],
+                         pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_P_FULL));
+        // ---- dS^T = P^T o (dP^T - D[q]) back into tensor memory ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 46 + w))) { ok = false; break; }
+        tc_fence_after();
+        // in two halves of 16 columns: half h's bf16 pairs go to columns
+        // 8h..8h+7, which hold dP^T values this warp has already loaded
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[16];
+          tmem_ld16(tDP + 16u * h, r);
+          tmem_wait_ld();
+          const float4* d4 = reinterpret_cast<const float4*>(dsum + 16 * h);
+          uint32_t pk[8];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 Dv = d4[u];
+            const float* pp = pr + 16 * h + 4 * u;
+            pk[2 * u] = pack_bf16(pp[0] * (__uint_as_float(r[4 * u]) - Dv.x),
+                                  pp[1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
+            pk[2 * u + 1] = pack_bf16(pp[2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
+                                      pp[3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
+          }
+          tmem_st8(tDP + 8u * h, pk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_DS_FULL));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_DS_FULL));
         ++steps;
         ++n;
       }
@@ -423,36 +463,46 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DKV_FULL), dkv & 1, ab, 36 + w))) { ok = false; break; }
       ++dkv;
       tc_fence_after();
-      uint32_t r[32], rv[32];
-      tmem_ld32(tDK, r);
-      tmem_ld32(tDV, rv);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_DKV_EMPTY));
       uint32_t out[16];
+      {
+        uint32_t r[32];
+        tmem_ld32(tDV, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
-        if (p.rotate) {
-          float c, s;
-          rope_cos_sin_fast(key, rope_freq(16 * w + u, kD, p.log2_theta), &c, &s);
-          const float a2 = a * c + b * s, b2 = b * c - a * s;
-          a = a2;
-          b = b2;
-        }
-        out[u] = pack_bf16(a, b);
+        for (int u = 0; u < 16; ++u)
+          out[u] = pack_bf16(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
       }
       if (key_ok) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 4; ++c)
+          reinterpret_cast<uint4*>(dvrow)[c] =
+              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+      }
+      {
+        uint32_t r[32];
+        tmem_ld32(tDK, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_DKV_EMPTY));
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
+          if (p.rotate) {
+            float c, s;
+            rope_cos_sin_fast(key, freq[16 * w + u], &c, &s);
+            const float a2 = a * c + b * s, b2 = b * c - a * s;
+            a = a2;
+            b = b2;
+          }
+          out[u] = pack_bf16(a, b);
+        }
+      }
+      if (key_ok) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
           reinterpret_cast<uint4*>(dkrow)[c] =
               make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
-          reinterpret_cast<uint4*>(dvrow)[c] = make_uint4(
-              pack_bf16(__uint_as_float(rv[8 * c]), __uint_as_float(rv[8 * c + 1])),
-              pack_bf16(__uint_as_float(rv[8 * c + 2]), __uint_as_float(rv[8 * c + 3])),
-              pack_bf16(__uint_as_float(rv[8 * c + 4]), __uint_as_float(rv[8 * c + 5])),
-              pack_bf16(__uint_as_float(rv[8 * c + 6]), __uint_as_float(rv[8 * c + 7])));
-        }
       }
     }
   }
@@ -472,7 +522,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
   }
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -121,6 +121,19 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
+// Generic-proxy shared-memory writes become visible to the async proxy (the
+// tensor cores' operand reads) after this fence and a barrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -195,6 +208,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -237,6 +267,17 @@ __device__ __forceinline__ void mma_kk128(uint32_t d, uint64_t a_desc, uint64_t 
   for (int kk = 0; kk < 8; ++kk) {
     const uint64_t off = (uint64_t)(((kk >> 2) * kOperandBoxBytes + (kk & 3) * 32) >> 4);
     mma_ss(d, a_desc + off, b_desc + off, idesc, kk > 0 ? 1u : acc);
+  }
+}
+
+// D (+)= A * B over K = 128, A a K-major tile and B an MN-major tile whose
+// rows are K (a k-step is 16 rows = 2048 bytes).
+__device__ __forceinline__ void mma_km128(uint32_t d, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t a_off = (uint64_t)(((kk >> 2) * kOperandBoxBytes + (kk & 3) * 32) >> 4);
+    mma_ss(d, a_desc + a_off, b_desc + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : acc);
   }
 }
 
