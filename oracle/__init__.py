@@ -37,6 +37,7 @@ from .attention import (  # noqa: F401
     attention_forward,
     attention_backward,
     attention_rows,
+    attention_decode,
     kept_pairs,
     attention_flops,
 )

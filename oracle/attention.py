@@ -253,6 +253,48 @@ def attention_rows(q, k, v, d_o, samples, seg=None, causal=True, theta=1e4, scal
     return res
 
 
+def attention_decode(q_new, k, v, seg=None, causal=True, theta=1e4, scale=None, heads=None):
+    """Decode step: T new query tokens against a cache of S tokens, in float64.
+
+    The new tokens are the last T positions of each row (their own keys and
+    values are already the last T entries of ``k``/``v``), the generation
+    setting of the research note's sections "模型架构" and "Infra"
+    (inference over a million-token context).  Query t sits at position
+    p_t = S - T + t and attends exactly as row p_t of ``attention_forward``:
+    rotated by R(p_t), keys rotated by R(j), the same mask and softmax.
+
+    q_new [B, T, H, D]; k, v [B, S, H, D] un-rotated; seg [B, S] or None.
+    ``heads`` limits the computation to those heads (others stay NaN).
+    Returns o [B, T, H, D] and lse [B, H, T].
+    """
+    q_new = np.asarray(q_new)
+    B, T, H, D = q_new.shape
+    S = np.asarray(k).shape[1]
+    if T > S:
+        raise ValueError("more new tokens than cache entries")
+    seg = _seg_or_default(seg, B, S)
+    sc = _scale(scale, D)
+    use_rope = theta is not None and theta > 0
+    o = np.full((B, T, H, D), np.nan)
+    lse = np.full((B, H, T), np.nan)
+    pos = np.arange(S - T, S)
+    keys = np.arange(S)
+    for b in range(B):
+        allowed = allowed_mask(seg[b], pos, keys, causal)  # [T, S]
+        for h in (range(H) if heads is None else heads):
+            K = np.asarray(k[b, :, h, :], dtype=np.float64)
+            Q = np.asarray(q_new[b, :, h, :], dtype=np.float64)
+            if use_rope:
+                K = rope_apply(K.reshape(1, S, 1, D), theta).reshape(S, D)
+                Q = rope_apply(Q.reshape(1, T, 1, D), theta,
+                               position_offset=S - T).reshape(T, D)
+            s = sc * (Q @ K.T)
+            l, P = _softmax_rows(s, allowed)
+            lse[b, h] = l
+            o[b, :, h, :] = P @ np.asarray(v[b, :, h, :], dtype=np.float64)
+    return o, lse
+
+
 def kept_pairs(seg, causal=True) -> int:
     """Number of allowed (i, j) pairs summed over rows: sum over segments of
     L(L+1)/2 when causal, L^2 otherwise (each id's tokens counted together)."""

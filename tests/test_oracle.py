@@ -421,3 +421,59 @@ def test_golden_tiny_case_regression():
     res = A.attention_backward(q, k, v, do, seg, causal=g["causal"], theta=g["theta"])
     for key in ("o", "lse", "dq", "dk", "dv"):
         assert _close(res[key], np.array(g["expected"][key], dtype=np.float64), 1e-12), key
+
+
+# ----------------------------------------------------------------- decode step
+def test_decode_equals_the_last_rows_of_the_forward():
+    """A decode step is the forward pass's last T rows: same positions, same
+    mask, same softmax (causal prefix property).  The decode oracle is a
+    separate restatement, pinned here against the pinned forward oracle."""
+    rng = np.random.default_rng(31)
+    B, S, H, D, T = 2, 70, 3, 8, 5
+    q = rng.standard_normal((B, S, H, D))
+    k = rng.standard_normal((B, S, H, D))
+    v = rng.standard_normal((B, S, H, D))
+    seg = np.stack([np.repeat([0, 1, 2], [30, 25, 15]), np.repeat([0, 1], [66, 4])])
+    seg[1, -2] = -1  # a padding token among the new ones
+    for causal in (True, False):
+        o_f, lse_f = oracle.attention_forward(q, k, v, seg, causal=causal, theta=500.0)
+        o_d, lse_d = oracle.attention_decode(q[:, S - T:], k, v, seg, causal=causal, theta=500.0)
+        np.testing.assert_allclose(o_d, o_f[:, S - T:], atol=1e-12)
+        np.testing.assert_array_equal(np.isneginf(lse_d), np.isneginf(lse_f[:, :, S - T:]))
+        fin = np.isfinite(lse_d)
+        np.testing.assert_allclose(lse_d[fin], lse_f[:, :, S - T:][fin], atol=1e-12)
+
+
+def test_decode_no_rope_matches_torch_sdpa():
+    """theta disabled, one segment: each new query is plain softmax attention
+    over the keys up to its position (torch fp64 SDPA with an explicit mask)."""
+    import torch
+    rng = np.random.default_rng(32)
+    B, S, H, D, T = 2, 40, 2, 16, 4
+    q = rng.standard_normal((B, T, H, D))
+    k = rng.standard_normal((B, S, H, D))
+    v = rng.standard_normal((B, S, H, D))
+    o, lse = oracle.attention_decode(q, k, v, None, theta=0.0)
+    mask = torch.arange(S)[None, :] <= torch.arange(S - T, S)[:, None]
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask)
+    np.testing.assert_allclose(o, ref.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    s = torch.einsum("bhtd,bhsd->bhts", tq, tk) / np.sqrt(D)
+    ref_lse = torch.logsumexp(s.masked_fill(~mask, -float("inf")), dim=-1)
+    np.testing.assert_allclose(lse, ref_lse.numpy(), atol=1e-12)
+
+
+def test_decode_oracle_catches_a_position_shift(monkeypatch):
+    """Planted mistake: rotating the new queries as if they started at 0
+    breaks the equality with the forward rows."""
+    rng = np.random.default_rng(33)
+    B, S, H, D, T = 1, 50, 1, 8, 3
+    q, k, v = (rng.standard_normal((B, S, H, D)) for _ in range(3))
+    o_f, _ = oracle.attention_forward(q, k, v, None, theta=100.0)
+    real = oracle.attention.rope_apply
+
+    def shifted(x, theta, inverse=False, position_offset=0):
+        return real(x, theta, inverse, 0)
+    monkeypatch.setattr(oracle.attention, "rope_apply", shifted)
+    o_d, _ = oracle.attention_decode(q[:, S - T:], k, v, None, theta=100.0)
+    assert np.abs(o_d - o_f[:, S - T:]).max() > 1e-3
