@@ -144,6 +144,36 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
 lwm_status lwm_attn_fwd_noalloc(const lwm_attn_desc* desc, const void* q, const void* k,
                                 const void* v, void* o, float* lse, void* stream);
 
+/* Decode step (research note, "模型架构" and "Infra": generation over a
+ * million-token context).  n_new new tokens are the last n_new positions of
+ * each row; their keys and values are already the last entries of the
+ * cache.  New token t (position p_t = S - n_new + t) attends exactly as row
+ * p_t of lwm_attn_fwd: same mask (segment ids over the whole row, causal
+ * order), same scale and RoPE.
+ *   desc:    batch B, seqlen S = cache length (new tokens included), heads
+ *            H, head_dim 128, dtype LWM_DTYPE_BF16 (others return
+ *            LWM_ERR_UNSUPPORTED), causal, rope_theta, softmax_scale,
+ *            segment_ids [B, S] (device, may be NULL).
+ *   n_new:   1 .. min(S, LWM_DECODE_MAX_NEW); more returns
+ *            LWM_ERR_UNSUPPORTED (use lwm_attn_fwd), below 1 or above S
+ *            LWM_ERR_INVALID_ARG.
+ *   q:       [B, n_new, H, D] un-rotated queries (rotated inside, in fp32).
+ *   k_cache: [B, S, H, D] ROTATED keys, R(j) k_j, as lwm_rope_apply writes
+ *            them (a cache keeps keys the way attention consumes them).
+ *   v_cache: [B, S, H, D].
+ *   o:       [B, n_new, H, D] out (bf16);  lse: [B, H, n_new] fp32 out
+ *            (natural log, -inf for a token with no allowed key, o = 0).
+ *   ws:      lwm_attn_decode_workspace_size(desc, n_new) bytes, 256-byte
+ *            aligned (chunk partials of the split-KV reduction).
+ * All device pointers 16-byte aligned.  Asynchronous on `stream`; the
+ * timing-event slots fwd_start / fwd_stop bracket its two kernels.  Reads
+ * each allowed cache row of each head once: bound by HBM bandwidth. */
+#define LWM_DECODE_MAX_NEW 16
+size_t lwm_attn_decode_workspace_size(const lwm_attn_desc* desc, int64_t n_new);
+lwm_status lwm_attn_decode(const lwm_attn_desc* desc, int64_t n_new, const void* q,
+                           const void* k_cache, const void* v_cache, void* o, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
 /* y = R(p) x (inverse = 0) or R(p)^T x (inverse != 0) for x of [B,S,H,D]
  * (research note, "模型架构": standard RoPE; theta per "训练方法").  Angles
  * p*w_t are formed and reduced modulo 2*pi in fp64, cos/sin taken in fp32,

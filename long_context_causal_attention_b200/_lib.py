@@ -28,7 +28,9 @@ STATUS_NAMES = {
 
 ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_rope_apply",
                 "lwm_attn_read_status", "lwm_status_string", "lwm_attn_set_timing_events",
-                "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc")
+                "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc",
+                "lwm_attn_decode_workspace_size", "lwm_attn_decode")
+DECODE_MAX_NEW = 16
 
 
 class LwmAttnDesc(ctypes.Structure):
@@ -77,6 +79,11 @@ def _load():
     lib.lwm_attn_set_timing_events.restype = None
     lib.lwm_attn_fwd_noalloc.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P]
     lib.lwm_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.lwm_attn_decode_workspace_size.argtypes = [ctypes.POINTER(LwmAttnDesc), ctypes.c_int64]
+    lib.lwm_attn_decode_workspace_size.restype = ctypes.c_size_t
+    lib.lwm_attn_decode.argtypes = [ctypes.POINTER(LwmAttnDesc), ctypes.c_int64, P, P, P, P, P, P,
+                                    ctypes.c_size_t, P]
+    lib.lwm_attn_decode.restype = ctypes.c_int
     lib.lwm_attn_kernel_launches.argtypes = []
     lib.lwm_attn_kernel_launches.restype = ctypes.c_uint64
     return lib
@@ -199,6 +206,42 @@ def lwm_attn_bwd(q, k, v, o, lse, d_o, segment_ids=None, causal=True, rope_theta
     if check_status:
         _check(lwm_attn_read_status(workspace, stream), "lwm_attn_bwd (device status)")
     return dq, dk, dv
+
+
+def lwm_attn_decode_workspace_size(desc: LwmAttnDesc, n_new: int) -> int:
+    return int(_lib.lwm_attn_decode_workspace_size(ctypes.byref(desc), int(n_new)))
+
+
+def lwm_attn_decode(q_new, k_cache, v_cache, segment_ids=None, causal=True, rope_theta=1e4,
+                    softmax_scale=0.0, o=None, lse=None, workspace=None, stream=None,
+                    check_status=False):
+    """o [B,T,H,D] and lse [B,H,T] for T new un-rotated queries against a cache
+    of S rotated keys and values (the new tokens are its last T entries)."""
+    _cuda(q_new, "q_new")
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, name)
+        if t.shape != k_cache.shape or t.dtype != q_new.dtype:
+            raise ValueError(f"{name} must be [B, S, H, D] of q_new's dtype")
+    B, T, H, D = q_new.shape
+    if k_cache.dim() != 4 or k_cache.shape[0] != B or k_cache.shape[2:] != q_new.shape[2:]:
+        raise ValueError("k_cache must be [B, S, H, D] with q_new's B, H, D")
+    desc = make_desc(k_cache, segment_ids, causal, rope_theta, softmax_scale)
+    if o is None:
+        o = torch.empty_like(q_new)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q_new.device)
+    if workspace is None:
+        n = lwm_attn_decode_workspace_size(desc, T)
+        if n == 0:
+            raise LwmError(-1, "lwm_attn_decode_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q_new.device)
+    st = _lib.lwm_attn_decode(ctypes.byref(desc), T, q_new.data_ptr(), k_cache.data_ptr(),
+                              v_cache.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                              workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check(st, "lwm_attn_decode")
+    if check_status:
+        _check(lwm_attn_read_status(workspace, stream), "lwm_attn_decode (device status)")
+    return o, lse
 
 
 def lwm_rope_apply(x, theta, inverse=False, out=None, stream=None):

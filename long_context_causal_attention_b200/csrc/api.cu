@@ -84,6 +84,29 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
   return w.bytes;
 }
 
+size_t layout_decode_workspace(const Problem& p, int64_t n_new, void* base, Workspace* ws) {
+  char* b = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    off = align_up(off, 1024);
+    void* r = b ? b + off : nullptr;
+    off += bytes;
+    return r;
+  };
+  Workspace w{};
+  w.status = static_cast<DeviceStatus*>(take(sizeof(DeviceStatus)));
+  const size_t tiles = (size_t)p.B * (size_t)p.n_tiles * sizeof(int32_t);
+  w.tile_min = static_cast<int32_t*>(take(tiles));
+  w.tile_max = static_cast<int32_t*>(take(tiles));
+  const size_t parts = (size_t)p.B * p.H * (size_t)n_new *
+                       (size_t)((p.S + kDecodeChunk - 1) / kDecodeChunk);
+  w.dec_ml = static_cast<float*>(take(parts * 2 * sizeof(float)));
+  w.dec_o = static_cast<float*>(take(parts * (size_t)p.D * sizeof(float)));
+  w.bytes = align_up(off, 1024);
+  if (ws) *ws = w;
+  return w.bytes;
+}
+
 namespace {
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -209,6 +232,42 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
   record_event(2, st);
   e = launch_simt_bwd(p, w, v, lse, d_o, dq, dk, dv, st);
   record_event(3, st);
+  return cuda_status(e);
+}
+
+size_t lwm_attn_decode_workspace_size(const lwm_attn_desc* desc, int64_t n_new) {
+  Problem p{};
+  if (make_problem(desc, &p) != LWM_OK || n_new < 1 || n_new > p.S) return 0;
+  return layout_decode_workspace(p, n_new, nullptr, nullptr);
+}
+
+lwm_status lwm_attn_decode(const lwm_attn_desc* desc, int64_t n_new, const void* q,
+                           const void* k_cache, const void* v_cache, void* o, float* lse,
+                           void* ws, size_t ws_bytes, void* stream) {
+  Problem p{};
+  lwm_status s = make_problem(desc, &p);
+  if (s != LWM_OK) return s;
+  if (p.dtype != LWM_DTYPE_BF16 || p.D != 128) return LWM_ERR_UNSUPPORTED;
+  if (n_new < 1 || n_new > p.S) return p.B == 0 && n_new >= 0 ? LWM_OK : LWM_ERR_INVALID_ARG;
+  if (n_new > LWM_DECODE_MAX_NEW) return LWM_ERR_UNSUPPORTED;
+  if (p.B == 0) return LWM_OK;
+  if ((p.S + kDecodeChunk - 1) / kDecodeChunk > INT32_MAX) return LWM_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !o || !lse) return LWM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(lse))
+    return LWM_ERR_ALIGNMENT;
+  const size_t need = layout_decode_workspace(p, n_new, nullptr, nullptr);
+  if (!ws || ws_bytes < need) return LWM_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return LWM_ERR_ALIGNMENT;
+  Workspace w{};
+  layout_decode_workspace(p, n_new, ws, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
+  if (e == cudaSuccess) e = launch_segment_bounds(p, w, st, false);
+  if (e != cudaSuccess) return LWM_ERR_CUDA;
+  record_event(0, st);
+  e = launch_decode(p, w, n_new, q, k_cache, v_cache, o, lse, st);
+  record_event(1, st);
   return cuda_status(e);
 }
 

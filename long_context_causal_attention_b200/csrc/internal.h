@@ -35,6 +35,8 @@ struct Workspace {
   float* delta;        // [B, H, S] fp32 dot(dO, O) per row (backward, CUDA-core path)
   float* lse2_pad;     // [B, H, n_tiles*128] LSE*log2(e) or +inf (backward, tensor-core path)
   float* delta_pad;    // [B, H, n_tiles*128] dot(dO, O) or 0 (backward, tensor-core path)
+  float* dec_ml;       // [B, H, T, n_chunks, 2] decode chunk max and sum (log2 domain)
+  float* dec_o;        // [B, H, T, n_chunks, D] decode chunk sums of p * v
   size_t bytes;        // total bytes the layout needs
 };
 
@@ -54,7 +56,15 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws);
 // Launchers (return the first CUDA error, or cudaSuccess).
 cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, double theta,
                         const void* x, void* y, int inverse, cudaStream_t st);
-cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st);
+// ranges = false computes only the per-tile bounds (no q_lo / k_hi).
+cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st,
+                                  bool ranges = true);
+// Keys per CTA of the decode kernel (one partial softmax per chunk).
+constexpr int64_t kDecodeChunk = 512;
+size_t layout_decode_workspace(const Problem& p, int64_t n_new, void* base, Workspace* ws);
+cudaError_t launch_decode(const Problem& p, const Workspace& ws, int64_t n_new, const void* q,
+                          const void* k_cache, const void* v_cache, void* o, float* lse,
+                          cudaStream_t st);
 cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float* delta,
                          cudaStream_t st);
 

@@ -73,13 +73,18 @@ __global__ void tile_ranges_kernel(const int32_t* __restrict__ tmin, const int32
 
 }  // namespace
 
-cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st) {
+cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st,
+                                  bool ranges) {
   if (!p.seg) return cudaSuccess;
   const int64_t n = p.B * p.n_tiles;
   if (n == 0) return cudaSuccess;
   const int threads = 128;
   const unsigned grid = (unsigned)((n + threads - 1) / threads);
   tile_bounds_kernel<<<grid, threads, 0, st>>>(p.seg, p.B, p.S, p.n_tiles, ws.tile_min, ws.tile_max);
+  if (!ranges) {
+    note_launches(1);
+    return cudaGetLastError();
+  }
   tile_ranges_kernel<<<grid, threads, 0, st>>>(ws.tile_min, ws.tile_max, p.B, p.n_tiles, p.causal,
                                                ws.q_lo, ws.k_hi);
   note_launches(2);

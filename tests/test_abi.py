@@ -99,6 +99,32 @@ def test_argument_errors_return_before_any_launch(lwm):
     assert lib.lwm_attn_read_status(None, None) == -1
 
 
+def test_decode_workspace_and_argument_errors(lwm):
+    """Decode entry point: sizes and every refusal that happens before a launch."""
+    lib = lwm._lib.lib()
+    P = 0x10000
+    big = 1 << 40
+    d = _desc(lwm)  # B2 S300 H4 D128 bf16
+    ws1 = lwm.lwm_attn_decode_workspace_size(d, 1)
+    ws4 = lwm.lwm_attn_decode_workspace_size(d, 4)
+    chunks = (300 + 511) // 512
+    assert ws1 >= 2 * 4 * chunks * 130 * 4 and ws4 > ws1 and ws4 % 1024 == 0
+    assert lwm.lwm_attn_decode_workspace_size(d, 0) == 0
+    assert lwm.lwm_attn_decode_workspace_size(d, 301) == 0
+    dec = lambda desc, n=1, q=P, ws=P, wsb=big: (ctypes.byref(desc), n, q, P, P, P, P, ws, wsb, None)
+    assert lib.lwm_attn_decode(*dec(_desc(lwm, dtype=1))) == -2       # fp32
+    assert lib.lwm_attn_decode(*dec(_desc(lwm, head_dim=64))) == -2   # D = 64
+    assert lib.lwm_attn_decode(*dec(d, n=0)) == -1
+    assert lib.lwm_attn_decode(*dec(d, n=301)) == -1
+    assert lib.lwm_attn_decode(*dec(d, n=17)) == -2                   # above the maximum
+    assert lib.lwm_attn_decode(*dec(d, q=None)) == -1
+    assert lib.lwm_attn_decode(*dec(d, q=P + 8)) == -3
+    assert lib.lwm_attn_decode(*dec(d, ws=None)) == -4
+    assert lib.lwm_attn_decode(*dec(d, wsb=ws1 - 1)) == -4
+    assert lib.lwm_attn_decode(*dec(d, ws=P + 16)) == -3
+    assert lib.lwm_attn_decode(*dec(_desc(lwm, batch=0))) == 0
+
+
 def test_python_binding_requires_cuda_tensors(lwm):
     import torch
     q = torch.zeros(1, 4, 1, 64)
