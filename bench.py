@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 from workloads import WORKLOADS, segment_ids  # noqa: E402
 
 METRIC = "causal attn fwd+bwd TFLOP/s (32x128 heads, bf16) and % of B200 BF16 peak"
+DECODE_METRIC = "decode attention HBM GB/s (new tokens against a rotated KV cache, 32x128 heads, bf16)"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 L2_BYTES = 126 * 2 ** 20
 
@@ -398,6 +399,206 @@ def ours(args):
     return 0
 
 
+def decode_bytes(w, seg, n_new: int) -> int:
+    """Algorithmic HBM bytes of one decode step: every cache row (key and
+    value, all heads) some new token may attend to, read once, plus the new
+    queries, the outputs and the segment ids of the cache."""
+    row = w.heads * w.head_dim * 2
+    S = w.seqlen
+    total = 0
+    for b in range(w.batch):
+        r = seg[b]
+        sq = r[S - n_new:]
+        need = np.isin(r, sq[sq >= 0]) & (r >= 0)
+        total += 2 * row * int(np.count_nonzero(need))
+    total += 2 * w.batch * n_new * row                  # q in, o out
+    if w.segments != "single":
+        total += 4 * w.batch * S
+    return total
+
+
+def time_oracle_decode(w, seg, seed: int, heads: int = 1):
+    """Oracle decode on the first ``heads`` heads of the workload."""
+    import torch
+    import oracle
+    n_new = w.extra["n_new"]
+    g = torch.Generator()
+    g.manual_seed(seed)
+    shape = (1, w.seqlen, heads, w.head_dim)
+    q = (torch.randn((1, n_new, heads, w.head_dim), generator=g) * w.sigma).to(torch.bfloat16)
+    k = (torch.randn(shape, generator=g) * w.sigma).to(torch.bfloat16)
+    v = (torch.randn(shape, generator=g) * w.sigma).to(torch.bfloat16)
+    f = lambda x: x.double().numpy()
+    t0 = time.perf_counter()
+    oracle.attention_decode(f(q), f(k), f(v), seg[:1], causal=w.causal, theta=w.theta)
+    dt = time.perf_counter() - t0
+    sub = w.with_(batch=1, heads=heads)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    return dt, decode_bytes(sub, seg[:1], n_new), threads
+
+
+def decode_line(w, value, ms, args, ws, extra):
+    line = {"metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "cache_len": w.seqlen,
+                       "n_new": w.extra["n_new"], "heads": w.heads, "head_dim": w.head_dim,
+                       "theta": w.theta, "segments": w.segments,
+                       "parallelism": f"independent problem per GPU x{ws}",
+                       "l2": "cache larger than L2 (16 GiB vs 126 MB), no flush"}}
+    line.update(extra)
+    return line
+
+
+def reference_decode(args):
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    seg = segment_ids(w, seed=args.seed)
+    for _ in range(args.warmup):
+        time_oracle_decode(w, seg, args.seed)
+    tot, nbytes, threads = 0.0, 0, 1
+    for _ in range(args.steps):
+        dt, nbytes, threads = time_oracle_decode(w, seg, args.seed)
+        tot += dt
+    value = nbytes * args.steps / tot / 1e9
+    sample = f"float64 numpy oracle decode, head 0 of {w.name} ({nbytes / 1e9:.2f} GB of cache)"
+    line = decode_line(w, value, 1e3 * tot / args.steps, args, ws, {
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ours_decode(args):
+    import torch
+    import torch.distributed as dist
+
+    import long_context_causal_attention_b200 as lwm
+
+    ws, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = WORKLOADS[args.workload]
+    n_new = w.extra["n_new"]
+    seed = rank_seed(args.seed, rank)
+    seg = segment_ids(w, seed=seed)
+    seg_d = None if w.segments == "single" else torch.as_tensor(seg, dtype=torch.int32,
+                                                                device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    shape = (w.batch, w.seqlen, w.heads, w.head_dim)
+    q = (torch.randn((w.batch, n_new, w.heads, w.head_dim), generator=g, device=dev)
+         * w.sigma).to(torch.bfloat16)
+    k = (torch.randn(shape, generator=g, device=dev) * w.sigma).to(torch.bfloat16)
+    v = (torch.randn(shape, generator=g, device=dev) * w.sigma).to(torch.bfloat16)
+    k_cache = lwm.lwm_rope_apply(k, w.theta, out=k)  # the cache holds rotated keys
+    desc = lwm.make_desc(k_cache, seg_d, w.causal, w.theta, w.scale)
+    wsp = torch.empty(lwm.lwm_attn_decode_workspace_size(desc, n_new), dtype=torch.uint8,
+                      device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.batch, w.heads, n_new), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lwm.lwm_attn_decode(q, k_cache, v, seg_d, w.causal, w.theta, w.scale, o=o, lse=lse,
+                            workspace=wsp, stream=stream)
+
+    nbytes = decode_bytes(w, seg, n_new)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    launches0 = lwm.lwm_attn_kernel_launches()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for s_ in range(args.steps):
+        lwm.lwm_attn_set_timing_events(kev[s_][0], kev[s_][1])
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    lwm.lwm_attn_set_timing_events()
+    launches = lwm.lwm_attn_kernel_launches() - launches0
+    clk = clocks.stop()
+    ms = start.elapsed_time(stop) / args.steps
+    kern = sum(e[0].elapsed_time(e[1]) for e in kev) / args.steps
+    ms, kern = max_over_ranks([ms, kern], ws, dev)
+    value = nbytes * ws / (ms * 1e-3) / 1e9
+    # end to end: the new queries come from the host, outputs go back; the
+    # cache stays resident on the device as it does while generating
+    hq = q.cpu().pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ems, = max_over_ranks([e0.elapsed_time(e1) / args.steps], ws, dev)
+    peaks, src = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = nbytes / (kern * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, nb, threads = time_oracle_decode(w, seg, seed)
+        cpu = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"float64 numpy oracle decode, head 0 of {w.name} "
+                         f"({nb / 1e9:.2f} GB of cache in {dt:.1f} s)"}
+    if rank == 0:
+        line = decode_line(w, value, ms, args, ws, {
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "decode_partial_kernel + decode_merge_kernel",
+                         "algorithmic": "key and value rows the new tokens may attend to, "
+                                        "all heads, once; q in, o out",
+                         "bytes_per_step": nbytes, "kernels_ms": kern,
+                         "peak_source": f"{src} HBM copy bandwidth"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": nbytes * ws / (ems * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+                    "d2h_bytes_per_step": ho.numel() * ho.element_size()
+                    + hl.numel() * hl.element_size()},
+            "gpu_launches": launches,
+            "clocks": clk})
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -410,9 +611,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    decode = "n_new" in WORKLOADS[args.workload].extra
     if args.impl == "reference":
-        return reference_arm(args)
-    return ours(args)
+        return reference_decode(args) if decode else reference_arm(args)
+    return ours_decode(args) if decode else ours(args)
 
 
 if __name__ == "__main__":

@@ -15,6 +15,8 @@ into one sequence)):
   packed_8k         B4 H32 D128 bf16, S=8192 packed video/text, theta 1e6, fwd+bwd
   long_128k         B1 H32 D128 bf16, S=131072, one segment, theta 1e7, fwd+bwd
   million_1m        B1 H32 D128 bf16, S=1048576, one segment, theta 5e7, fwd+bwd
+  decode_1m         B1 H32 D128 bf16, one new token against a 1048576-token
+                    cache (the new token's own key and value included), theta 5e7
 """
 
 from __future__ import annotations
@@ -56,6 +58,12 @@ WORKLOADS = {
     "million_1m": Workload("million_1m", 1, 1048576, 32, 128, "bf16", 5e7),
     # profiling case: same head shape, 16K tokens (each tensor 128 MiB, above L2)
     "prof_16k": Workload("prof_16k", 1, 16384, 32, 128, "bf16", 1e6),
+    # decode step: n_new new tokens, the cache of `seqlen` tokens includes them
+    "decode_1m": Workload("decode_1m", 1, 1048576, 32, 128, "bf16", 5e7, backward=False,
+                          extra={"n_new": 1}),
+    # decode profiling case: 128K-token cache (2 GiB of keys and values, above L2)
+    "prof_decode_128k": Workload("prof_decode_128k", 1, 131072, 32, 128, "bf16", 1e7,
+                                 backward=False, extra={"n_new": 1}),
 }
 ORDER = ["tiny_packed_fp32", "fwd_32k", "packed_8k", "long_128k", "million_1m"]
 
