@@ -38,11 +38,11 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 L2_BYTES = 126 * 2 ** 20
 
 # DRAM traffic of one attn_bwd_dkdv_kernel launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) from an ncu capture of the 16K-token profiling case,
-# scaled to each workload by its tile pairs; valid only for the kernel source
-# it was taken on (sha256 of the kernel file and the headers it includes).
-DKDV_TRAFFIC = {"bytes_per_tile_pair": None, "source_sha256": None,
-                "profile": "profiles/attn_bwd_dkdv_kernel_prof_16k.md"}
+# dram__bytes_write.sum, one-pass ncu capture of the full-size workload, see
+# profiles/attn_bwd_dkdv_traffic_long_128k.md); valid only for the kernel
+# source it was taken on (sha256 of the kernel file and the device headers).
+DKDV_TRAFFIC = {"bytes": {"long_128k": 32.64e9 + 2.14e9},
+                "source_sha256": "d5a5df5cf8c01584d76240667c64fb5ba0c977f72af78561b35e26af58d52586"}
 
 
 def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
@@ -160,7 +160,7 @@ def kernel_source_sha256(name: str) -> str:
     import hashlib
     d = os.path.join(ROOT, "long_context_causal_attention_b200", "csrc")
     h = hashlib.sha256()
-    for f in (name, "sm100.cuh", "common.cuh", "internal.h"):
+    for f in (name, "sm100.cuh", "common.cuh"):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -349,9 +349,9 @@ def ours(args):
     achieved = dkdv_flops / (dkdv_k * 1e-3) / 1e12
     traffic = None
     units = tile_pairs(seg, w.heads, w.causal)
-    if (DKDV_TRAFFIC["bytes_per_tile_pair"] and
+    if (w.name in DKDV_TRAFFIC["bytes"] and
             DKDV_TRAFFIC["source_sha256"] == kernel_source_sha256("attn_bwd_sm100.cu")):
-        traffic = DKDV_TRAFFIC["bytes_per_tile_pair"] * units
+        traffic = DKDV_TRAFFIC["bytes"][w.name]
     bwd_flops = 2.5 * fwd_flops
     dq_k = bwd_k - dkdv_k
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

@@ -147,15 +147,18 @@ decode_partial_kernel(const DecParams p) {
       for (int kb = 0; kb < kKeysPerWarp; kb += KB) {
         const int64_t kbase = k0 + warp * kKeysPerWarp + kb;
         if (kbase >= p.S) break;
-        // scores: 32 partial products per lane, folded across the warp
+        // the batch's key and value rows in one burst of loads (more bytes
+        // in flight per warp), then NP partial products per lane, folded
         float d[NP];
+        uint2 vr[KB];
         {
           uint2 kr[KB];
 #pragma unroll
           for (int j = 0; j < KB; ++j) {
             const int64_t key = kbase + j;
-            kr[j] = key < p.S ? ldg8(p.k + ((rowS + key) * p.H + h) * kD + 4 * lane)
-                              : make_uint2(0u, 0u);
+            const size_t off = ((rowS + key) * p.H + h) * kD + 4 * lane;
+            kr[j] = key < p.S ? ldg8(p.k + off) : make_uint2(0u, 0u);
+            vr[j] = key < p.S ? ldg8(p.v + off) : make_uint2(0u, 0u);
           }
 #pragma unroll
           for (int j = 0; j < KB; ++j) {
@@ -202,13 +205,6 @@ decode_partial_kernel(const DecParams p) {
           for (int e = 0; e < 4; ++e) acc[tt][e] *= ct;
         }
         // p * v
-        uint2 vr[KB];
-#pragma unroll
-        for (int j = 0; j < KB; ++j) {
-          const int64_t kj = kbase + j;
-          vr[j] = kj < p.S ? ldg8(p.v + ((rowS + kj) * p.H + h) * kD + 4 * lane)
-                           : make_uint2(0u, 0u);
-        }
 #pragma unroll
         for (int j = 0; j < KB; ++j) {
           const float4 vf = bf16x4(vr[j]);
@@ -261,37 +257,48 @@ decode_partial_kernel(const DecParams p) {
   }
 }
 
-__global__ void __launch_bounds__(kD) decode_merge_kernel(const DecParams p) {
-  __shared__ float red[kD / 32];
-  __shared__ float bcast;
+constexpr int kMergeSlices = 8;  // chunk slices per merge CTA (one warp group of 128 each)
+
+__global__ void __launch_bounds__(kD * kMergeSlices) decode_merge_kernel(const DecParams p) {
+  __shared__ float red[kD * kMergeSlices / 32];
+  __shared__ float part[kMergeSlices][kD + 1];
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int dd = threadIdx.x, warp = dd >> 5, lane = dd & 31;
+  const int tid = threadIdx.x, dd = tid % kD, slice = tid / kD;
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int kWarpsM = kD * kMergeSlices / 32;
   const size_t base = (((size_t)b * p.H + h) * p.T + t) * p.n_chunks;
   const float* ml = p.part_ml + 2 * base;
   // M = max over chunks
   float M = -INFINITY;
-  for (int c = dd; c < p.n_chunks; c += kD) M = fmaxf(M, ml[2 * c]);
+  for (int c = tid; c < p.n_chunks; c += kD * kMergeSlices) M = fmaxf(M, ml[2 * c]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   if (lane == 0) red[warp] = M;
   __syncthreads();
-  if (dd == 0) {
-    float r = red[0];
-    for (int w = 1; w < kD / 32; ++w) r = fmaxf(r, red[w]);
-    bcast = r;
-  }
-  __syncthreads();
-  M = bcast;
-  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < kWarpsM; ++w) M = fmaxf(M, red[w]);
+  // this slice's share of L and of O[dd]
   float L = 0.f, O = 0.f;
   if (M != -INFINITY) {
-    for (int c = 0; c < p.n_chunks; ++c) {
+#pragma unroll 4
+    for (int c = slice; c < p.n_chunks; c += kMergeSlices) {
       const float mc = ml[2 * c];
-      if (mc == -INFINITY) continue;
-      const float f = exp2f(mc - M);
-      L += ml[2 * c + 1] * f;  // every thread sums the same values in the same order
+      const float f = mc == -INFINITY ? 0.f : exp2f(mc - M);
+      L += ml[2 * c + 1] * f;
       O += p.part_o[(base + c) * kD + dd] * f;
     }
+  }
+  part[slice][dd] = O;
+  if (dd == 0) part[slice][kD] = L;
+  __syncthreads();
+  if (slice != 0) return;
+  O = 0.f;
+  L = 0.f;
+#pragma unroll
+  for (int sl = 0; sl < kMergeSlices; ++sl) {
+    O += part[sl][dd];
+    L += part[sl][kD];
   }
   const size_t orow = (((size_t)b * p.T + t) * p.H + h) * kD;
   if (L > 0.f) {
@@ -336,7 +343,7 @@ cudaError_t launch_decode(const Problem& pb, const Workspace& ws, int64_t n_new,
   else
     decode_partial_kernel<4, 32><<<g1, kThreads, 0, st>>>(p);
   const dim3 g2((unsigned)n_new, (unsigned)pb.H, (unsigned)pb.B);
-  decode_merge_kernel<<<g2, kD, 0, st>>>(p);
+  decode_merge_kernel<<<g2, kD * kMergeSlices, 0, st>>>(p);
   note_launches(2);
   return cudaGetLastError();
 }
