@@ -206,6 +206,17 @@ void lwm_attn_set_timing_events(void* fwd_start, void* fwd_stop, void* bwd_start
                                 void* bwd_stop, void* bwd_split);
 uint64_t lwm_attn_kernel_launches(void);
 
+/* Failure-path self-test (no counterpart on the pages).  Clears the status
+ * word at the start of ws (at least 256 bytes, 256-byte aligned) and runs one
+ * CTA that waits on an mbarrier with the same bounded wait the tensor-core
+ * kernels use, for at most limit_cycles SM clock cycles.  arrive != 0 arms
+ * the barrier first (the wait completes: status stays LWM_OK); arrive == 0
+ * leaves it unarmed (nothing ever arrives: the wait runs out, the kernel
+ * records LWM_ERR_TIMEOUT and returns).  Read the outcome with
+ * lwm_attn_read_status(ws).  Asynchronous; returns launch errors only. */
+lwm_status lwm_attn_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_cycles, int arrive,
+                                  void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,7 +29,7 @@ STATUS_NAMES = {
 ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_rope_apply",
                 "lwm_attn_read_status", "lwm_status_string", "lwm_attn_set_timing_events",
                 "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc",
-                "lwm_attn_decode_workspace_size", "lwm_attn_decode")
+                "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait")
 DECODE_MAX_NEW = 16
 
 
@@ -84,6 +84,8 @@ def _load():
     lib.lwm_attn_decode.argtypes = [ctypes.POINTER(LwmAttnDesc), ctypes.c_int64, P, P, P, P, P, P,
                                     ctypes.c_size_t, P]
     lib.lwm_attn_decode.restype = ctypes.c_int
+    lib.lwm_attn_selftest_wait.argtypes = [P, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int, P]
+    lib.lwm_attn_selftest_wait.restype = ctypes.c_int
     lib.lwm_attn_kernel_launches.argtypes = []
     lib.lwm_attn_kernel_launches.restype = ctypes.c_uint64
     return lib
@@ -274,6 +276,14 @@ def lwm_attn_set_timing_events(fwd_start=None, fwd_stop=None, bwd_start=None, bw
         return ctypes.c_void_p(e.cuda_event)
     _lib.lwm_attn_set_timing_events(handle(fwd_start), handle(fwd_stop), handle(bwd_start),
                                     handle(bwd_stop), handle(bwd_split))
+
+
+def lwm_attn_selftest_wait(workspace, limit_cycles: int, arrive: bool, stream=None) -> int:
+    """Run the bounded-wait self-test; returns the device status it leaves."""
+    _check(_lib.lwm_attn_selftest_wait(workspace.data_ptr(), workspace.numel(), int(limit_cycles),
+                                       1 if arrive else 0, _stream(stream)),
+           "lwm_attn_selftest_wait")
+    return lwm_attn_read_status(workspace, stream)
 
 
 def lwm_attn_kernel_launches() -> int:

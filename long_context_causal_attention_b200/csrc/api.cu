@@ -286,6 +286,14 @@ lwm_status lwm_rope_apply(int64_t batch, int64_t seqlen, int64_t heads, int64_t 
                                  static_cast<cudaStream_t>(stream)));
 }
 
+lwm_status lwm_attn_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_cycles, int arrive,
+                                  void* stream) {
+  if (!ws || ws_bytes < sizeof(DeviceStatus) || limit_cycles < 0) return LWM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return LWM_ERR_ALIGNMENT;
+  return cuda_status(launch_selftest_wait(static_cast<DeviceStatus*>(ws), (long long)limit_cycles,
+                                          arrive != 0, static_cast<cudaStream_t>(stream)));
+}
+
 lwm_status lwm_attn_read_status(const void* ws, void* stream) {
   if (!ws) return LWM_ERR_INVALID_ARG;
   int32_t code = 0;

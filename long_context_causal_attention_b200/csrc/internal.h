@@ -78,6 +78,11 @@ cudaError_t launch_sm100_bwd_dkdv(const Problem& p, const Workspace& ws, const v
 cudaError_t launch_sm100_bwd_dq(const Problem& p, const Workspace& ws, const void* v,
                                 const void* d_o, void* dq, cudaStream_t st);
 
+// Bounded-wait self-test: one CTA waits on an mbarrier (armed by an arrival
+// or not) for at most limit_cycles; a wait that runs out records
+// LWM_ERR_TIMEOUT in *status.
+cudaError_t launch_selftest_wait(DeviceStatus* status, long long limit_cycles, int arrive,
+                                 cudaStream_t st);
 cudaError_t launch_simt_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                             float* lse, cudaStream_t st);
 cudaError_t launch_simt_bwd(const Problem& p, const Workspace& ws, const void* v,

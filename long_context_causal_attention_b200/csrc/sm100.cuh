@@ -55,23 +55,30 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with `parity` of barrier `bar` to complete.  Returns
-// false if the CTA is aborting (this wait or another one gave up).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab,
-                                          int where) {
+// Wait for the phase with `parity` of barrier `bar` to complete, for at most
+// `limit` SM clock cycles.  Returns false if the CTA is aborting (this wait
+// or another one gave up); a wait that runs out raises the abort flag and
+// records LWM_ERR_TIMEOUT with its tag.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, const Abort& ab,
+                                                int where, long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*ab.flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *ab.flag = 1;
         report_timeout(ab.status, where);
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab,
+                                          int where) {
+  return mbar_wait_limit(bar, parity, ab, where, kWaitCycles);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
