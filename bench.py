@@ -176,6 +176,7 @@ def time_oracle_sample(w, seg, rows: int, seed: int):
     small = w.with_(batch=1, heads=1)
     t = make_tensors(small, seed=seed, device="cpu", with_grad_out=True)
     f = lambda x: x.double().numpy()
+    rows = min(rows, w.seqlen)
     r0 = w.seqlen - rows
     t0 = time.perf_counter()
     oracle.attention_backward(f(t["q"]), f(t["k"]), f(t["v"]), f(t["do"]), seg[:1],
@@ -202,7 +203,7 @@ def reference_arm(args):
         return 0
     w = WORKLOADS[args.workload]
     seg = segment_ids(w, seed=args.seed)
-    rows = args.oracle_rows
+    rows = min(args.oracle_rows, w.seqlen)
     for _ in range(args.warmup):
         time_oracle_sample(w, seg, rows, args.seed)
     times, flops, threads = [], 0.0, 1
@@ -368,9 +369,10 @@ def ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        dt, fl, threads = time_oracle_sample(w, seg, args.oracle_rows, seed)
+        rows = min(args.oracle_rows, w.seqlen)
+        dt, fl, threads = time_oracle_sample(w, seg, rows, seed)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"float64 numpy oracle, fwd+bwd of the last {args.oracle_rows} query rows "
+               "sample": f"float64 numpy oracle, fwd+bwd of the last {rows} query rows "
                          f"of one head of {w.name} ({fl / 1e9:.2f} GFLOP in {dt:.1f} s)"}
 
     if rank == 0:
