@@ -206,6 +206,33 @@ void lwm_attn_set_timing_events(void* fwd_start, void* fwd_stop, void* bwd_start
                                 void* bwd_stop, void* bwd_split);
 uint64_t lwm_attn_kernel_launches(void);
 
+/* ---- Sequence-parallel (ring) building blocks -------------------------
+ * Blockwise RingAttention (research note, "模型架构" and "Infra"; paper card,
+ * Summary): the sequence is split into equal blocks, one per device of a
+ * ring; every query block meets every key/value block once, and the results
+ * combine exactly by their log-sum-exp.  The per-block products are
+ * lwm_attn_fwd / lwm_attn_bwd on rotated inputs (rope_theta = 0); these
+ * entry points supply the rest.  All asynchronous on `stream`; device
+ * pointers; returns argument and launch errors.
+ *
+ * lwm_rope_apply_at: lwm_rope_apply with positions p = position_offset +
+ *   index in the row (a block that starts at token position_offset >= 0).
+ * lwm_attn_merge: for every row (b, s, h) of one query block, with
+ *   L = ln(e^{lse_acc} + e^{lse_part}):
+ *   o_acc <- e^{lse_acc - L} o_acc + e^{lse_part - L} o_part, lse_acc <- L.
+ *   o_acc fp32 [B,S,H,D], lse_acc fp32 [B,H,S] (start from 0 and -inf);
+ *   o_part [B,S,H,D] of `dtype`, lse_part [B,H,S].  A -inf side adds nothing.
+ * lwm_accumulate: acc[i] += x[i] for n elements (acc fp32, x of `dtype`).
+ * lwm_convert_f32: y[i] = x[i] rounded to `dtype` (nearest even). */
+lwm_status lwm_rope_apply_at(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
+                             int32_t dtype, double theta, int64_t position_offset, const void* x,
+                             void* y, int inverse, void* stream);
+lwm_status lwm_attn_merge(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
+                          int32_t dtype, float* o_acc, float* lse_acc, const void* o_part,
+                          const float* lse_part, void* stream);
+lwm_status lwm_accumulate(int64_t n, int32_t dtype, float* acc, const void* x, void* stream);
+lwm_status lwm_convert_f32(int64_t n, int32_t dtype, const float* x, void* y, void* stream);
+
 /* Failure-path self-test (no counterpart on the pages).  Clears the status
  * word at the start of ws (at least 256 bytes, 256-byte aligned) and runs one
  * CTA that waits on an mbarrier with the same bounded wait the tensor-core

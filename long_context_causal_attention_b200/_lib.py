@@ -29,7 +29,8 @@ STATUS_NAMES = {
 ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_rope_apply",
                 "lwm_attn_read_status", "lwm_status_string", "lwm_attn_set_timing_events",
                 "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc",
-                "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait")
+                "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait",
+                "lwm_rope_apply_at", "lwm_attn_merge", "lwm_accumulate", "lwm_convert_f32")
 DECODE_MAX_NEW = 16
 
 
@@ -86,6 +87,17 @@ def _load():
     lib.lwm_attn_decode.restype = ctypes.c_int
     lib.lwm_attn_selftest_wait.argtypes = [P, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int, P]
     lib.lwm_attn_selftest_wait.restype = ctypes.c_int
+    lib.lwm_rope_apply_at.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.c_int64, ctypes.c_int32, ctypes.c_double,
+                                      ctypes.c_int64, P, P, ctypes.c_int, P]
+    lib.lwm_rope_apply_at.restype = ctypes.c_int
+    lib.lwm_attn_merge.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.c_int32, P, P, P, P, P]
+    lib.lwm_attn_merge.restype = ctypes.c_int
+    lib.lwm_accumulate.argtypes = [ctypes.c_int64, ctypes.c_int32, P, P, P]
+    lib.lwm_accumulate.restype = ctypes.c_int
+    lib.lwm_convert_f32.argtypes = [ctypes.c_int64, ctypes.c_int32, P, P, P]
+    lib.lwm_convert_f32.restype = ctypes.c_int
     lib.lwm_attn_kernel_launches.argtypes = []
     lib.lwm_attn_kernel_launches.restype = ctypes.c_uint64
     return lib
@@ -288,3 +300,50 @@ def lwm_attn_selftest_wait(workspace, limit_cycles: int, arrive: bool, stream=No
 
 def lwm_attn_kernel_launches() -> int:
     return int(_lib.lwm_attn_kernel_launches())
+
+
+def lwm_rope_apply_at(x, theta, position_offset, inverse=False, out=None, stream=None):
+    """lwm_rope_apply with positions starting at ``position_offset``."""
+    _cuda(x, "x")
+    if x.dim() != 4:
+        raise ValueError("x must be [B, S, H, D]")
+    out = torch.empty_like(x) if out is None else out
+    B, S, H, D = x.shape
+    _check(_lib.lwm_rope_apply_at(B, S, H, D, _dtype_code(x), float(theta), int(position_offset),
+                                  x.data_ptr(), out.data_ptr(), 1 if inverse else 0,
+                                  _stream(stream)), "lwm_rope_apply_at")
+    return out
+
+
+def lwm_attn_merge(o_acc, lse_acc, o_part, lse_part, stream=None):
+    """In place: (o_acc, lse_acc) <- log-sum-exp merge with (o_part, lse_part)."""
+    for name, t in (("o_acc", o_acc), ("lse_acc", lse_acc), ("o_part", o_part),
+                    ("lse_part", lse_part)):
+        _cuda(t, name)
+    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32:
+        raise TypeError("o_acc and lse_acc must be float32")
+    if o_part.shape != o_acc.shape or lse_part.shape != lse_acc.shape:
+        raise ValueError("partial result must match the accumulator's shapes")
+    B, S, H, D = o_acc.shape
+    _check(_lib.lwm_attn_merge(B, S, H, D, _dtype_code(o_part), o_acc.data_ptr(),
+                               lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                               _stream(stream)), "lwm_attn_merge")
+
+
+def lwm_accumulate(acc, x, stream=None):
+    """In place: acc (float32) += x."""
+    _cuda(acc, "acc")
+    _cuda(x, "x")
+    if acc.dtype != torch.float32 or acc.shape != x.shape:
+        raise ValueError("acc must be float32 with x's shape")
+    _check(_lib.lwm_accumulate(x.numel(), _dtype_code(x), acc.data_ptr(), x.data_ptr(),
+                               _stream(stream)), "lwm_accumulate")
+
+
+def lwm_convert_f32(x, dtype, out=None, stream=None):
+    """x (float32) rounded to ``dtype`` (bfloat16 or float32)."""
+    _cuda(x, "x")
+    out = torch.empty(x.shape, dtype=dtype, device=x.device) if out is None else out
+    _check(_lib.lwm_convert_f32(x.numel(), _dtype_code(out), x.data_ptr(), out.data_ptr(),
+                                _stream(stream)), "lwm_convert_f32")
+    return out

@@ -286,6 +286,46 @@ lwm_status lwm_rope_apply(int64_t batch, int64_t seqlen, int64_t heads, int64_t 
                                  static_cast<cudaStream_t>(stream)));
 }
 
+lwm_status lwm_rope_apply_at(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
+                             int32_t dtype, double theta, int64_t position_offset, const void* x,
+                             void* y, int inverse, void* stream) {
+  if (batch < 0 || seqlen < 0 || heads < 1 || head_dim < 2 || (head_dim & 1)) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32) return LWM_ERR_INVALID_ARG;
+  if (!std::isfinite(theta) || position_offset < 0) return LWM_ERR_INVALID_ARG;
+  const int vec = dtype == LWM_DTYPE_BF16 ? 8 : 4;
+  if (head_dim % vec != 0 || head_dim > 512) return LWM_ERR_UNSUPPORTED;
+  if (batch * seqlen == 0) return LWM_OK;
+  if (!x || !y) return LWM_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return LWM_ERR_ALIGNMENT;
+  return cuda_status(launch_rope(batch, seqlen, heads, head_dim, dtype, theta, x, y, inverse,
+                                 static_cast<cudaStream_t>(stream), position_offset));
+}
+
+lwm_status lwm_attn_merge(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
+                          int32_t dtype, float* o_acc, float* lse_acc, const void* o_part,
+                          const float* lse_part, void* stream) {
+  if (batch < 0 || seqlen < 0 || heads < 1 || head_dim < 1) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32) return LWM_ERR_INVALID_ARG;
+  if (batch * seqlen == 0) return LWM_OK;
+  if (!o_acc || !lse_acc || !o_part || !lse_part) return LWM_ERR_INVALID_ARG;
+  return cuda_status(launch_attn_merge(batch, seqlen, heads, head_dim, dtype, o_acc, lse_acc,
+                                       o_part, lse_part, static_cast<cudaStream_t>(stream)));
+}
+
+lwm_status lwm_accumulate(int64_t n, int32_t dtype, float* acc, const void* x, void* stream) {
+  if (n < 0 || (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)) return LWM_ERR_INVALID_ARG;
+  if (n == 0) return LWM_OK;
+  if (!acc || !x) return LWM_ERR_INVALID_ARG;
+  return cuda_status(launch_accumulate(n, dtype, acc, x, static_cast<cudaStream_t>(stream)));
+}
+
+lwm_status lwm_convert_f32(int64_t n, int32_t dtype, const float* x, void* y, void* stream) {
+  if (n < 0 || (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)) return LWM_ERR_INVALID_ARG;
+  if (n == 0) return LWM_OK;
+  if (!x || !y) return LWM_ERR_INVALID_ARG;
+  return cuda_status(launch_convert_f32(n, dtype, x, y, static_cast<cudaStream_t>(stream)));
+}
+
 lwm_status lwm_attn_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_cycles, int arrive,
                                   void* stream) {
   if (!ws || ws_bytes < sizeof(DeviceStatus) || limit_cycles < 0) return LWM_ERR_INVALID_ARG;

@@ -54,8 +54,16 @@ void note_launches(int n);
 size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws);
 
 // Launchers (return the first CUDA error, or cudaSuccess).
+// pos0: position of token 0 of each row (p = pos0 + index in the row).
 cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, double theta,
-                        const void* x, void* y, int inverse, cudaStream_t st);
+                        const void* x, void* y, int inverse, cudaStream_t st, int64_t pos0 = 0);
+// Block results of one sequence split into key blocks (ring order):
+// o_acc/lse_acc <- exact log-sum-exp merge with (o_part, lse_part).
+cudaError_t launch_attn_merge(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, float* o_acc,
+                              float* lse_acc, const void* o_part, const float* lse_part,
+                              cudaStream_t st);
+cudaError_t launch_accumulate(int64_t n, int dtype, float* acc, const void* x, cudaStream_t st);
+cudaError_t launch_convert_f32(int64_t n, int dtype, const float* x, void* y, cudaStream_t st);
 // ranges = false computes only the per-tile bounds (no q_lo / k_hi).
 cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStream_t st,
                                   bool ranges = true);

@@ -20,7 +20,7 @@ template <> struct Vec<float> { static constexpr int N = 4; };
 template <typename T>
 __global__ void __launch_bounds__(128) rope_kernel(const T* __restrict__ x, T* __restrict__ y,
                                                    int64_t n_tok, int64_t S, int H, int D,
-                                                   double log2_theta, int inverse) {
+                                                   double log2_theta, int inverse, int64_t pos0) {
   constexpr int N = Vec<T>::N;
   constexpr int P = N / 2;
   const int per_head = D / N;
@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(128) rope_kernel(const T* __restrict__ x, T* _
   for (int u = 0; u < P; ++u) w[u] = rope_freq(c * P + u, D, log2_theta);
   const float sgn = inverse ? -1.0f : 1.0f;
   for (int64_t tok = blockIdx.x; tok < n_tok; tok += gridDim.x) {
-    const int64_t pos = tok % S;
+    const int64_t pos = pos0 + tok % S;
     float cs[P], sn[P];
 #pragma unroll
     for (int u = 0; u < P; ++u) {
@@ -121,7 +121,7 @@ int grid_for(int64_t n) {
 }  // namespace
 
 cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, double theta,
-                        const void* x, void* y, int inverse, cudaStream_t st) {
+                        const void* x, void* y, int inverse, cudaStream_t st, int64_t pos0) {
   const int64_t n_tok = B * S;
   if (n_tok == 0) return cudaSuccess;
   const size_t bytes = (size_t)n_tok * H * D * (dtype == LWM_DTYPE_BF16 ? 2 : 4);
@@ -134,10 +134,10 @@ cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, d
   if (dtype == LWM_DTYPE_BF16) {
     rope_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), n_tok, S, (int)H,
-        (int)D, l2t, inverse);
+        (int)D, l2t, inverse, pos0);
   } else {
     rope_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(x), static_cast<float*>(y),
-                                             n_tok, S, (int)H, (int)D, l2t, inverse);
+                                             n_tok, S, (int)H, (int)D, l2t, inverse, pos0);
   }
   note_launches(1);
   return cudaGetLastError();

@@ -125,6 +125,21 @@ def test_decode_workspace_and_argument_errors(lwm):
     assert lib.lwm_attn_decode(*dec(_desc(lwm, batch=0))) == 0
 
 
+def test_ring_entry_points_reject_bad_arguments(lwm):
+    lib = lwm._lib.lib()
+    P = 0x10000
+    assert lib.lwm_rope_apply_at(1, 8, 2, 64, 0, 1e4, -1, P, P, 0, None) == -1  # negative offset
+    assert lib.lwm_rope_apply_at(1, 8, 2, 64, 0, 1e4, 5, P + 4, P, 0, None) == -3
+    assert lib.lwm_rope_apply_at(0, 8, 2, 64, 0, 1e4, 5, None, None, 0, None) == 0
+    assert lib.lwm_attn_merge(1, 8, 2, 64, 5, P, P, P, P, None) == -1            # dtype
+    assert lib.lwm_attn_merge(1, 8, 2, 64, 0, None, P, P, P, None) == -1
+    assert lib.lwm_attn_merge(0, 8, 2, 64, 0, None, None, None, None, None) == 0
+    assert lib.lwm_accumulate(-1, 0, P, P, None) == -1
+    assert lib.lwm_accumulate(0, 0, None, None, None) == 0
+    assert lib.lwm_convert_f32(4, 2, P, P, None) == -1
+    assert lib.lwm_convert_f32(4, 0, None, P, None) == -1
+
+
 def test_python_binding_requires_cuda_tensors(lwm):
     import torch
     q = torch.zeros(1, 4, 1, 64)

@@ -1,0 +1,70 @@
+"""Ring (sequence-parallel) attention on one GPU: N virtual ranks in lockstep.
+
+The sequence is split into N blocks; the ring runs the library's block
+kernels (rotation at each block's offset, lwm_attn_fwd / lwm_attn_bwd on the
+rotated blocks, the log-sum-exp merge, fp32 gradient accumulation) exactly
+as N ranks would, with the shift between ranks a rotation of a list.  The
+result must match the float64 oracle on the whole sequence.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity_util import assert_close, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("n_ranks,n,theta", [(4, 256, 1e6), (3, 384, 1e7), (2, 200, 1e4)])
+def test_emulated_ring_matches_oracle(n_ranks, n, theta):
+    from long_context_causal_attention_b200 import ring
+    B, H, D = 1, 4, 128
+    S = n_ranks * n
+    g = torch.Generator(device="cuda")
+    g.manual_seed(n_ranks * 1000 + n)
+    q, k, v = ((torch.randn((B, S, H, D), generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+               for _ in range(3))
+    do = torch.randn((B, S, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    split = lambda t: [t[:, r * n:(r + 1) * n].contiguous() for r in range(n_ranks)]
+    res = ring.emulated_ring_forward(split(q), split(k), split(v), theta)
+    o = torch.cat([r[0] for r in res], dim=1)
+    lse = torch.cat([r[1] for r in res], dim=2)
+    grads = ring.emulated_ring_backward(split(q), split(k), split(v), [r[0] for r in res],
+                                        [r[1] for r in res], split(do), theta)
+    torch.cuda.synchronize()
+    dq, dk, dv = (torch.cat([gr[i] for gr in grads], dim=1) for i in range(3))
+    ref = oracle.attention_backward(to64(q), to64(k), to64(v), to64(do), None, causal=True,
+                                    theta=theta)
+    assert_close("o", to64(o), ref["o"], "bf16")
+    assert_close("lse", to64(lse), ref["lse"], "bf16")
+    assert_close("dq", to64(dq), ref["dq"], "bf16")
+    assert_close("dk", to64(dk), ref["dk"], "bf16")
+    assert_close("dv", to64(dv), ref["dv"], "bf16")
+
+
+def test_merge_kernel_equals_joint_softmax():
+    """Merging the results of two key halves equals attention over both."""
+    import long_context_causal_attention_b200 as lwm
+    B, S, H, D = 2, 300, 2, 128
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    q = (torch.randn((B, S, H, D), generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    k1, k2, v1, v2 = ((torch.randn((B, S, H, D), generator=g, device="cuda") * 0.5)
+                      .to(torch.bfloat16) for _ in range(4))
+    o1, l1 = lwm.lwm_attn_fwd(q, k1, v1, None, False, 0.0)
+    o2, l2 = lwm.lwm_attn_fwd(q, k2, v2, None, False, 0.0)
+    o_acc = torch.zeros((B, S, H, D), dtype=torch.float32, device="cuda")
+    l_acc = torch.full((B, H, S), float("-inf"), device="cuda")
+    lwm.lwm_attn_merge(o_acc, l_acc, o1, l1)
+    lwm.lwm_attn_merge(o_acc, l_acc, o2, l2)
+    torch.cuda.synchronize()
+    # joint reference: plain softmax attention of q over all 2S keys, float64
+    K, V = to64(torch.cat([k1, k2], 1)), to64(torch.cat([v1, v2], 1))
+    s = np.einsum("bshd,bthd->bhst", to64(q), K) / np.sqrt(D)
+    m = s.max(-1, keepdims=True)
+    e = np.exp(s - m)
+    ref_l = (m[..., 0] + np.log(e.sum(-1)))
+    ref_o = np.einsum("bhst,bthd->bshd", e / e.sum(-1, keepdims=True), V)
+    assert_close("o", to64(o_acc), ref_o, "bf16")
+    assert_close("lse", to64(l_acc), ref_l, "bf16")
