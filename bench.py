@@ -379,7 +379,7 @@ def ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
                        "heads": w.heads, "head_dim": w.head_dim, "theta": w.theta,
