@@ -80,8 +80,11 @@ enum : uint32_t {
   B_QD_FULL = 2,   // 2 stages
   B_QD_EMPTY = 4,  // 2 stages
   B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_DS_FULL = 9,
-  B_DKV_FULL = 10, B_DKV_EMPTY = 11, B_FIN = 12, B_S_READ = 13, B_PT_FREE = 14
+  B_DKV_FULL = 10, B_DKV_EMPTY = 11, B_FIN = 12, B_S_READ = 13, B_PT_FREE = 14,
+  B_ITEM_FULL = 15,   // 4 slots
+  B_ITEM_EMPTY = 19   // 4 slots
 };
+constexpr uint32_t kItemSlots = 4;
 constexpr uint32_t kEWWarps = kEW / 32;  // element-wise barriers take one arrival per warp
 
 struct BwdParams {
@@ -169,6 +172,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small_ptr + SOFF_MISC);
   const float* ld_smem = reinterpret_cast<const float*>(small_ptr + SOFF_LD);
   double* freq = reinterpret_cast<double*>(small_ptr + SOFF_FREQ);
+  // work items come from a global counter (greedy, in cost order): the TMA
+  // thread takes one and publishes it to the CTA through a 4-slot ring
+  volatile int* item_slot = reinterpret_cast<volatile int*>(small_ptr + SOFF_MISC + 16);
+  int* item_counter = &p.status->item_counter[0];
   const Abort ab{abort_flag, p.status};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.B * p.H * p.n_tiles;
@@ -190,6 +197,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(bar(B_FIN), 1);
     mbar_init(bar(B_S_READ), kEWWarps);
     mbar_init(bar(B_PT_FREE), 1);
+    for (uint32_t sl = 0; sl < kItemSlots; ++sl) {
+      mbar_init(bar(B_ITEM_FULL + sl), 1);
+      mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kEWWarps);
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -215,7 +226,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       int items = 0;
       bool ok = true;
       const size_t hstride = (size_t)p.n_tiles * 128;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+      for (uint32_t pub = 0; ok; ++items) {
+        const uint32_t sl = pub % kItemSlots;
+        if (pub >= kItemSlots &&
+            !mbar_wait(bar(B_ITEM_EMPTY + sl), ((pub / kItemSlots) - 1) & 1, ab, 20)) {
+          ok = false;
+          break;
+        }
+        const int idx = atomicAdd(item_counter, 1);
+        item_slot[sl] = idx;
+        mbar_arrive(bar(B_ITEM_FULL + sl));
+        ++pub;
+        if (idx >= n_items) break;
         const Item it = decode(p, idx);
         if (items > 0 && !mbar_wait(bar(B_KV_EMPTY), (items - 1) & 1, ab, 21)) { ok = false; break; }
         mbar_expect_tx(bar(B_KV_FULL), 2 * kTileBytes);
@@ -269,7 +291,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ++s_issued;
         return true;
       };
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+      for (uint32_t cons = 0; ok; ++items) {
+        const uint32_t sl = cons % kItemSlots;
+        if (!mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 18)) { ok = false; break; }
+        const int idx = item_slot[sl];
+        mbar_arrive(bar(B_ITEM_EMPTY + sl));
+        ++cons;
+        if (idx >= n_items) break;
         const Item it = decode(p, idx);
         if (!mbar_wait(bar(B_KV_FULL), items & 1, ab, 23)) { ok = false; break; }
         tc_fence_after();
@@ -319,7 +347,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t chunk0 = (uint32_t)(w & 1) * 4u, swz = (uint32_t)row & 7u;
     uint32_t steps = 0, dkv = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    for (uint32_t cons = 0; ok;) {
+      const uint32_t sl = cons % kItemSlots;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 17))) {
+        ok = false;
+        break;
+      }
+      const int idx = item_slot[sl];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + sl));
+      ++cons;
+      if (idx >= n_items) break;
       const Item it = decode(p, idx);
       const int64_t key = (int64_t)it.j * 128 + row;
       const bool key_ok = key < p.S;

@@ -16,7 +16,8 @@ struct DeviceStatus {
   int32_t code;       // lwm_status written by a kernel whose bounded wait ran out
   int32_t where;      // which wait gave up (kernel-defined tag)
   int32_t block;      // blockIdx.x of the reporting CTA
-  int32_t pad[61];
+  int32_t item_counter[4];  // work-queue heads of the persistent kernels (zeroed per call)
+  int32_t pad[57];
 };
 static_assert(sizeof(DeviceStatus) == 256, "status block is 256 bytes");
 
