@@ -67,8 +67,11 @@ enum : uint32_t {
   B_V_FULL = 6,    // kVStages
   B_V_EMPTY = 9,   // kVStages
   B_Q_READY = 12, B_S_FULL = 13, B_S_READ = 14, B_DP_FULL = 15, B_DS_FULL = 16,
-  B_DQ_FULL = 17, B_DQ_EMPTY = 18, B_FIN = 19
+  B_DQ_FULL = 17, B_DQ_EMPTY = 18, B_FIN = 19,
+  B_ITEM_FULL = 20,   // 4 slots
+  B_ITEM_EMPTY = 24   // 4 slots
 };
+constexpr uint32_t kItemSlots = 4;
 
 struct DqParams {
   const int32_t* seg;
@@ -153,6 +156,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem_raw + SOFF_MISC);
   double* freq = reinterpret_cast<double*>(smem_raw + SOFF_FREQ);
+  // work items come from a global counter (greedy, in cost order): the TMA
+  // thread takes one and publishes it to the CTA through a 4-slot ring
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem_raw + SOFF_MISC + 16);
+  int* item_counter = &p.status->item_counter[1];
   const Abort ab{abort_flag, p.status};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.B * p.H * p.n_tiles;
@@ -175,6 +182,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     mbar_init(bar(B_DQ_FULL), 1);
     mbar_init(bar(B_DQ_EMPTY), kEW / 32);
     mbar_init(bar(B_FIN), 1);
+    for (uint32_t sl = 0; sl < kItemSlots; ++sl) {
+      mbar_init(bar(B_ITEM_FULL + sl), 1);
+      mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kEW / 32);
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -196,7 +207,18 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (lane == 0) {
       uint32_t k_it = 0, v_it = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      for (uint32_t pub = 0; ok;) {
+        const uint32_t sl = pub % kItemSlots;
+        if (pub >= kItemSlots &&
+            !mbar_wait(bar(B_ITEM_EMPTY + sl), ((pub / kItemSlots) - 1) & 1, ab, 49)) {
+          ok = false;
+          break;
+        }
+        const int idx = atomicAdd(item_counter, 1);
+        item_slot[sl] = idx;
+        mbar_arrive(bar(B_ITEM_FULL + sl));
+        ++pub;
+        if (idx >= n_items) break;
         const Item it = decode(p, idx);
         auto load_k = [&](int j) -> bool {
           const uint32_t s = k_it % kKStages, n = k_it / kKStages;
@@ -258,7 +280,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         ++v_it;
         return true;
       };
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      for (uint32_t cons = 0; ok;) {
+        const uint32_t sl = cons % kItemSlots;
+        if (!mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 48)) { ok = false; break; }
+        const int idx = item_slot[sl];
+        mbar_arrive(bar(B_ITEM_EMPTY + sl));
+        ++cons;
+        if (idx >= n_items) break;
         const Item it = decode(p, idx);
         int j = first_rel(p, it);
         if (j < 0) continue;  // nothing to do: the element-wise warps write zeros
@@ -309,7 +337,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const size_t hstride = (size_t)p.n_tiles * 128;
     uint32_t steps = 0, dqc = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    for (uint32_t cons = 0; ok;) {
+      const uint32_t sl = cons % kItemSlots;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 47))) {
+        ok = false;
+        break;
+      }
+      const int idx = item_slot[sl];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + sl));
+      ++cons;
+      if (idx >= n_items) break;
       const Item it = decode(p, idx);
       const int64_t q = (int64_t)it.i * 128 + row;
       const bool q_ok = q < p.S;

@@ -66,8 +66,12 @@ enum : uint32_t {
   B_O_FULL = 14,  // per tile
   B_O_EMPTY = 16, // per tile
   B_FIN = 18,
-  B_COUNT = 19
+  B_ITEM_FULL = 19,   // 4 slots
+  B_ITEM_EMPTY = 23,  // 4 slots
+  B_COUNT = 27
 };
+constexpr uint32_t kItemSlots = 4;
+constexpr uint32_t kSoftmaxWarps = 8;
 
 struct FwdParams {
   const int32_t* seg;    // [B, S] or null
@@ -166,6 +170,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   auto bar = [&](uint32_t slot) { return bar0 + 8u * slot; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  // work items come from a global counter (greedy, in cost order): the TMA
+  // thread takes one and publishes it to the CTA through a 4-slot ring
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + OFF_MISC + 16);
+  int* item_counter = &p.status->item_counter[2];
   const Abort ab{abort_flag, p.status};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,6 +194,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(bar(B_O_EMPTY + s), 128);
     }
     mbar_init(bar(B_FIN), 1);
+    for (uint32_t sl = 0; sl < kItemSlots; ++sl) {
+      mbar_init(bar(B_ITEM_FULL + sl), 1);
+      mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kSoftmaxWarps);
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -209,7 +221,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t k_it = 0, v_it = 0;
       int items = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+      for (uint32_t pub = 0; ok; ++items) {
+        const uint32_t sl = pub % kItemSlots;
+        if (pub >= kItemSlots &&
+            !mbar_wait(bar(B_ITEM_EMPTY + sl), ((pub / kItemSlots) - 1) & 1, ab, 13)) {
+          ok = false;
+          break;
+        }
+        const int idx = atomicAdd(item_counter, 1);
+        item_slot[sl] = idx;
+        mbar_arrive(bar(B_ITEM_FULL + sl));
+        ++pub;
+        if (idx >= n_items) break;
         const Item it = decode(p, idx);
         if (items > 0 && !mbar_wait(bar(B_Q_EMPTY), (items - 1) & 1, ab, 1)) { ok = false; break; }
         const int nq = (it.qt[0] >= 0) + (it.qt[1] >= 0);
@@ -263,7 +286,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int items = 0;
       bool ok = true;
       const uint32_t sq0 = base + OFF_Q;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++items) {
+      for (uint32_t cons = 0; ok; ++items) {
+        const uint32_t sl = cons % kItemSlots;
+        if (!mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 14)) { ok = false; break; }
+        const int idx = item_slot[sl];
+        mbar_arrive(bar(B_ITEM_EMPTY + sl));
+        ++cons;
+        if (idx >= n_items) break;
         const Item it = decode(p, idx);
         if (!mbar_wait(bar(B_Q_FULL), items & 1, ab, 4)) { ok = false; break; }
         tc_fence_after();
@@ -347,7 +376,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(t * 128);
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    for (uint32_t cons = 0; ok;) {
+      const uint32_t sl = cons % kItemSlots;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 15))) {
+        ok = false;
+        break;
+      }
+      const int idx = item_slot[sl];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + sl));
+      ++cons;
+      if (idx >= n_items) break;
       const Item it = decode(p, idx);
       if (it.qt[t] < 0) continue;
       const int64_t row = (int64_t)it.qt[t] * 128 + tid;
