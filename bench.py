@@ -41,8 +41,8 @@ L2_BYTES = 126 * 2 ** 20
 # dram__bytes_write.sum, one-pass ncu capture of the full-size workload, see
 # profiles/attn_bwd_dkdv_traffic_long_128k.md); valid only for the kernel
 # source it was taken on (sha256 of the kernel file and the device headers).
-DKDV_TRAFFIC = {"bytes": {"long_128k": 32.64e9 + 2.14e9},
-                "source_sha256": "d5a5df5cf8c01584d76240667c64fb5ba0c977f72af78561b35e26af58d52586"}
+DKDV_TRAFFIC = {"bytes": {"long_128k": 6.43e9 + 2.13e9},
+                "source_sha256": "62d64d788603196261ed835b78a714d0a9f137859be95108d65117ea76d6656f"}
 
 
 def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
