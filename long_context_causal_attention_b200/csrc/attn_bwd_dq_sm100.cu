@@ -399,14 +399,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             hi = d < 0 ? 0 : (d > 32 ? 32 : (int)d);
           }
           const int64_t kv = p.S - k0;
-          if (kv < hi) hi = kv < 0 ? 0 : (int)kv;
+          const int kvalid = kv > 32 ? 32 : (kv < 0 ? 0 : (int)kv);  // columns inside the row
+          if (kvalid < hi) hi = kvalid;
           if (seg_q < 0) hi = 0;
-          const int32_t* ks = p.seg ? p.seg + (size_t)it.b * p.S + k0 : nullptr;
-          uint32_t bits = 0;
-#pragma unroll 4
-          for (int c = 0; c < 32; ++c) {
-            const bool keep = c < hi && (ks == nullptr || __ldg(ks + c) == seg_q);
-            bits |= (uint32_t)keep << c;
+          uint32_t bits = bit_range(0, hi);
+          if (p.seg) {  // lane c loads the id of key column k0 + c
+            const int32_t kseg = lane < kvalid ? __ldg(p.seg + (size_t)it.b * p.S + k0 + lane) : INT_MIN;
+            bits &= warp_segment_bits(kseg, seg_q);
           }
           mw = bits;
         }

@@ -383,13 +383,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           }
           const int64_t qv = p.S - q0;
           const int hi = qv > 32 ? 32 : (qv < 0 ? 0 : (int)qv);  // exclusive
-          const int32_t* qs = p.seg ? p.seg + (size_t)it.b * p.S + q0 : nullptr;
-          uint32_t bits = 0;
-#pragma unroll 4
-          for (int c = 0; c < 32; ++c) {
-            const bool keep = seg_k >= 0 && c >= lo && c < hi &&
-                              (qs == nullptr || __ldg(qs + c) == seg_k);
-            bits |= (uint32_t)keep << c;
+          uint32_t bits = seg_k >= 0 ? bit_range(lo, hi) : 0u;
+          if (p.seg) {  // lane c loads the id of query column q0 + c
+            const int32_t qseg = lane < hi ? __ldg(p.seg + (size_t)it.b * p.S + q0 + lane) : INT_MIN;
+            bits &= warp_segment_bits(qseg, seg_k);
           }
           mw = bits;
         }

@@ -425,17 +425,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           int lim = p.causal ? (int)(d < -1 ? -1 : (d > 127 ? 127 : d)) : 127;
           if (kvalid - 1 < lim) lim = (int)(kvalid - 1);
           if (seg_row < 0) lim = -1;
-          // 128-bit keep mask, built without touching the score registers
+          // 128-bit keep mask, built without touching the score registers:
+          // keys 32w + c <= lim, and (packing) the row's segment, one load per
+          // lane per 32 keys
           const int32_t* ks = p.seg ? p.seg + (size_t)it.b * p.S + (size_t)j * 128 : nullptr;
           uint32_t mw[4];
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            uint32_t bits = 0;
-#pragma unroll 4
-            for (int c = 0; c < 32; ++c) {
-              const int kc = w * 32 + c;
-              const bool okk = kc <= lim && (ks == nullptr || __ldg(ks + kc) == seg_row);
-              bits |= (uint32_t)okk << c;
+            const int n = lim - 32 * w + 1;
+            uint32_t bits = bit_range(0, n < 0 ? 0 : (n > 32 ? 32 : n));
+            if (ks) {
+              const int64_t kc = 32 * w + lane;
+              const int32_t kseg = kc < kvalid ? __ldg(ks + kc) : INT_MIN;
+              bits &= warp_segment_bits(kseg, seg_row);
             }
             mw[w] = bits;
           }

@@ -1,6 +1,8 @@
 // Shared device helpers for liblwm_attn (CUDA, sm_100a).
 #pragma once
 
+#include <climits>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -82,6 +84,32 @@ __device__ __forceinline__ void rope_cos_sin_fast(int64_t pos, double w, float* 
   double r = fma(-k, kTwoPiHi, a);
   r = fma(-k, kTwoPiLo, r);
   __sincosf((float)r, s, c);
+}
+
+// Packing mask of one 32 x 32 block, built by a whole warp: lane c holds the
+// segment id of column c (col_seg; a value no row holds, e.g. INT_MIN, for a
+// column past the end), every lane the id of its own row (row_seg).  Bit c of
+// the result is set iff column c belongs to this lane's segment.  One load per
+// lane instead of 32, and one pass per distinct row id in the warp (one or
+// two for contiguous packed segments).  All 32 lanes must call it.
+__device__ __forceinline__ uint32_t warp_segment_bits(int32_t col_seg, int32_t row_seg) {
+  uint32_t bits = 0, pending = 0xffffffffu;
+  while (pending) {
+    const int32_t v = __shfl_sync(0xffffffffu, row_seg, __ffs(pending) - 1);
+    const uint32_t cols = __ballot_sync(0xffffffffu, col_seg == v);
+    const uint32_t rows = __ballot_sync(0xffffffffu, row_seg == v);
+    if (row_seg == v) bits = cols;
+    pending &= ~rows;
+  }
+  return bits;
+}
+
+// Bits [lo, hi) of a 32-bit word, 0 <= lo, hi <= 32.
+__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
+  if (hi <= lo) return 0u;
+  const uint32_t upto_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  const uint32_t below_lo = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
+  return upto_hi & ~below_lo;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
