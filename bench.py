@@ -312,35 +312,71 @@ def ours(args):
     ms_step = ms / args.steps
     value = job_tflops(step_flops, ws, ms_step)
 
-    # end to end through the public API: pinned host inputs in, gradients out
+    # end to end through the public API: every step copies its inputs in from
+    # pinned host memory and its gradients out to pinned host memory.  Two
+    # device buffer sets alternate, so the copies of step s+1's inputs (copy-in
+    # stream) and of step s-1's gradients (copy-out stream) run while step s
+    # computes, as a training loop streaming its batches would.
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
-        hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3))
-        n_e2e = max(1, min(args.steps, 3))
+        n_e2e = max(2, args.steps)
+        host_in = [x.cpu().pin_memory() for x in (q, k, v, do)]
+        host_out = [[torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3)]
+                    for _ in range(2)]
+        sets = [(q, k, v, do, o, lse, dq, dk, dv)]
+        sets.append(tuple(torch.empty_like(x) for x in sets[0]))
+        copy_in = torch.cuda.Stream(device=dev)
+        copy_out = torch.cuda.Stream(device=dev)
 
-        def e2e_step():
-            for hsrc, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
-                dst.copy_(hsrc, non_blocking=True)
-            step()
-            for src, hdst in ((dq, hdq), (dk, hdk), (dv, hdv)):
-                hdst.copy_(src, non_blocking=True)
+        def run_step(bufs):
+            q_, k_, v_, do_, o_, lse_, dq_, dk_, dv_ = bufs
+            lwm.lwm_attn_fwd(q_, k_, v_, seg_d, w.causal, w.theta, w.scale, o=o_, lse=lse_,
+                             workspace=ws_f, stream=stream)
+            lwm.lwm_attn_bwd(q_, k_, v_, o_, lse_, do_, seg_d, w.causal, w.theta, w.scale,
+                             dq=dq_, dk=dk_, dv=dv_, workspace=ws_b, stream=stream)
 
-        e2e_step()
-        torch.cuda.synchronize()
+        def e2e_run(n):
+            ev = lambda: torch.cuda.Event(enable_timing=False)
+            start_ev = torch.cuda.Event(enable_timing=True)
+            stop_ev = torch.cuda.Event(enable_timing=True)
+            start_ev.record(stream)
+            copy_in.wait_event(start_ev)
+            in_done, comp_done, out_done = [], [], []
+            for s_ in range(n):
+                bufs = sets[s_ % 2]
+                with torch.cuda.stream(copy_in):
+                    if s_ >= 2:
+                        copy_in.wait_event(comp_done[s_ - 2])  # step s-2 is done with the set
+                    for hsrc, dst in zip(host_in, bufs[:4]):
+                        dst.copy_(hsrc, non_blocking=True)
+                    in_done.append(ev())
+                    in_done[-1].record(copy_in)
+                stream.wait_event(in_done[s_])
+                if s_ >= 2:
+                    stream.wait_event(out_done[s_ - 2])   # its gradients have left the set
+                run_step(bufs)
+                comp_done.append(ev())
+                comp_done[-1].record(stream)
+                with torch.cuda.stream(copy_out):
+                    copy_out.wait_event(comp_done[s_])
+                    for src, hdst in zip(bufs[6:], host_out[s_ % 2]):
+                        hdst.copy_(src, non_blocking=True)
+                    out_done.append(ev())
+                    out_done[-1].record(copy_out)
+            stream.wait_event(out_done[-1])
+            stop_ev.record(stream)
+            torch.cuda.synchronize()
+            return start_ev.elapsed_time(stop_ev)
+
+        e2e_run(2)
         barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        ems = e2e_run(n_e2e)
         barrier()
-        ems, = max_over_ranks([e0.elapsed_time(e1)], ws, dev)
+        ems, = max_over_ranks([ems], ws, dev)
         nb = q.numel() * q.element_size()
         e2e = {"value": job_tflops(step_flops, ws, ems / n_e2e), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 3 * nb, "steps": n_e2e}
+               "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 3 * nb, "steps": n_e2e,
+               "overlap": "double-buffered: copies of neighbouring steps run during compute"}
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
