@@ -42,7 +42,7 @@ L2_BYTES = 126 * 2 ** 20
 # profiles/attn_bwd_dkdv_traffic_long_128k.md); valid only for the kernel
 # source it was taken on (sha256 of the kernel file and the device headers).
 DKDV_TRAFFIC = {"bytes": {"long_128k": 6.43e9 + 2.13e9},
-                "source_sha256": "62d64d788603196261ed835b78a714d0a9f137859be95108d65117ea76d6656f"}
+                "source_sha256": "dd20546d0968e6e8239479b5e3e266cb7dbf6cb462389eeadb9424348f61cb6a"}
 
 
 def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
@@ -383,7 +383,7 @@ def ours(args):
     # dominant kernel: dK/dV, whose four GEMMs per kept pair (S^T, dP^T, dV,
     # dK) are all algorithmic work: 8*D flops per pair and head
     dkdv_flops = 8.0 * w.head_dim * w.heads * pairs
-    achieved = dkdv_flops / (dkdv_k * 1e-3) / 1e12
+    achieved = dkdv_flops / (dkdv_k * 1e-3) / 1e12 if dkdv_k > 0.0 else None
     traffic = None
     units = tile_pairs(seg, w.heads, w.causal)
     if (w.name in DKDV_TRAFFIC["bytes"] and
@@ -391,8 +391,10 @@ def ours(args):
         traffic = DKDV_TRAFFIC["bytes"][w.name]
     bwd_flops = 2.5 * fwd_flops
     dq_k = bwd_k - dkdv_k
+    if achieved is None:  # the CUDA-core backward (fp32, head_dim 64) is one launch
+        dq_k, dkdv_k = None, None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
+                "frac": achieved / peak if achieved else None, "traffic": traffic,
                 "kernel": "attn_bwd_dkdv_kernel",
                 "algorithmic": "8*D*H flops per kept (query, key) pair: S^T, dP^T, dV, dK",
                 "tile_pairs": units,
@@ -400,8 +402,8 @@ def ours(args):
                 "dkdv_kernel_ms": dkdv_k, "dq_kernel_ms": dq_k, "fwd_kernel_ms": fwd_k,
                 "fwd_kernel_tflops": fwd_flops / (fwd_k * 1e-3) / 1e12,
                 "bwd_kernels_tflops": bwd_flops / (bwd_k * 1e-3) / 1e12,
-                "dq_kernel_tflops_incl_recompute": 6.0 * w.head_dim * w.heads * pairs
-                / (dq_k * 1e-3) / 1e12}
+                "dq_kernel_tflops_incl_recompute": (6.0 * w.head_dim * w.heads * pairs
+                                                    / (dq_k * 1e-3) / 1e12) if dq_k else None}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
