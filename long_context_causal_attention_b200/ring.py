@@ -19,7 +19,7 @@ and are home after N shifts.
 Each step of the arithmetic runs in the library's CUDA kernels
 (lwm_rope_apply_at, lwm_attn_fwd / lwm_attn_bwd on rotated inputs,
 lwm_attn_merge, lwm_accumulate, lwm_convert_f32); this module only orders
-them and moves blocks.  Two drivers run the same per-rank algorithm:
+them and moves blocks.  Two stepping loops run the same per-rank algorithm:
 ``ring_forward`` / ``ring_backward`` for one rank of a torch.distributed
 process group (NCCL point-to-point over NVLink; block i+1 is in flight while
 block i is computed), and ``emulated_ring_forward`` / ``..._backward`` for
@@ -64,9 +64,9 @@ class GpuBlockOps:
 
 
 # ----------------------------------------------------------------------------
-# the per-rank algorithm, as generators: ("start", tensors) hands the driver
-# the tensors to pass on to the next rank and gets back a handle; ("wait",
-# handle) returns the tensors received from the previous rank.
+# the per-rank algorithm, as generators: ("start", tensors) hands the
+# stepping loop the tensors to pass on to the next rank and gets back a
+# handle; ("wait", handle) returns the tensors received from the previous rank.
 # ----------------------------------------------------------------------------
 def _forward_steps(rank, size, q, k, v, theta, scale, ops):
     B, n, H, D = q.shape
@@ -111,7 +111,7 @@ def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops):
 
 
 # ----------------------------------------------------------------------------
-# drivers
+# stepping loops
 # ----------------------------------------------------------------------------
 def _run_distributed(gen, group):
     import torch.distributed as dist
