@@ -1,6 +1,6 @@
 """Ring attention's exchange schedule on world-size 2 and 3 gloo ranks (CPU).
 
-The ring driver for torch.distributed (NCCL on GPUs) is run here on gloo
+The ring stepping loop for torch.distributed (NCCL on GPUs) runs here on gloo
 ranks with a CPU stand-in for the block operations (float64 torch math, the
 oracle's rotation), so the point-to-point schedule, the causal skipping of
 later blocks, the log-sum-exp merge order and the final shift that brings
