@@ -405,6 +405,26 @@ def ours(args):
                 "dq_kernel_tflops_incl_recompute": (6.0 * w.head_dim * w.heads * pairs
                                                     / (dq_k * 1e-3) / 1e12) if dq_k else None}
 
+    # the HBM-bound pre-pass on its own (step A2): lwm_rope_apply over q,
+    # reading and writing every element once, against the copy bandwidth
+    rope_out = torch.empty_like(q)
+    lwm.lwm_rope_apply(q, w.theta, out=rope_out, stream=stream)
+    r0 = torch.cuda.Event(enable_timing=True)
+    r1 = torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    n_rope = 5
+    for _ in range(n_rope):
+        lwm.lwm_rope_apply(q, w.theta, out=rope_out, stream=stream)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    rope_ms = r0.elapsed_time(r1) / n_rope
+    rope_bytes = 2 * q.numel() * q.element_size()
+    del rope_out
+    hbm_kernels = {"rope_apply": {"bytes": rope_bytes, "ms": rope_ms,
+                                  "GB/s": rope_bytes / (rope_ms * 1e-3) / 1e9,
+                                  "frac_of_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9
+                                  / float(peaks["hbm_gbs"])}}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rows = min(args.oracle_rows, w.seqlen)
@@ -432,6 +452,7 @@ def ours(args):
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
+            "hbm_kernels": hbm_kernels,
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

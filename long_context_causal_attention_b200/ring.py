@@ -6,9 +6,12 @@ row is split into N equal blocks, block r held by rank r of a ring.  Every
 rank keeps its query block and passes its key/value block to the next rank N
 times over, so each query block meets every key/value block once; the
 per-block results combine exactly by their log-sum-exp, so the result equals
-attention over the whole sequence.  With a causal mask, block pairs whose
-keys all come after the queries (source rank > own rank) are skipped, the
-diagonal pair is causal inside and earlier blocks are attended in full.
+attention over the whole sequence.  With a causal mask, chunk pairs whose
+keys all come after the queries are skipped, the diagonal pair is causal
+inside and earlier chunks are attended in full.  Token layout: "contiguous"
+(rank r holds chunk r of N, so late ranks do most of the causal work) or
+"zigzag" (the default: 2N chunks, rank r holds chunks r and 2N-1-r, the
+same work on every rank).
 
 Backward: every rank computes, for each visiting key/value block, the
 contributions to its own dq and to the visitor's dk and dv (FlashAttention
@@ -64,49 +67,108 @@ class GpuBlockOps:
 
 
 # ----------------------------------------------------------------------------
+# token layout: which global chunks of the sequence each rank holds
+# ----------------------------------------------------------------------------
+def chunk_ids(rank: int, size: int, layout: str):
+    """Global chunk indices held by ``rank``, in the order they sit in its
+    local tensors.  "contiguous": N chunks, rank r holds chunk r.  "zigzag":
+    2N chunks, rank r holds chunks r and 2N-1-r, so every rank has the same
+    causal work (an early chunk with few keys and a late one with many)."""
+    if layout == "contiguous":
+        return [rank]
+    if layout == "zigzag":
+        return [rank, 2 * size - 1 - rank]
+    raise ValueError(f"unknown layout {layout!r}")
+
+
+def split_for_ranks(x, size: int, layout: str = "zigzag", dim: int = 1):
+    """The local tensor of every rank, cut from a whole-sequence tensor."""
+    n_chunks = size * len(chunk_ids(0, size, layout))
+    chunks = torch.chunk(x, n_chunks, dim=dim)
+    if len({c.shape[dim] for c in chunks}) != 1 or len(chunks) != n_chunks:
+        raise ValueError("sequence length must split into equal chunks")
+    return [torch.cat([chunks[g] for g in chunk_ids(r, size, layout)], dim=dim).contiguous()
+            for r in range(size)]
+
+
+def merge_from_ranks(parts, layout: str = "zigzag", dim: int = 1):
+    """Inverse of split_for_ranks: the whole-sequence tensor."""
+    size = len(parts)
+    per = len(chunk_ids(0, size, layout))
+    chunks = [None] * (size * per)
+    for r, t in enumerate(parts):
+        for c, piece in zip(chunk_ids(r, size, layout), torch.chunk(t, per, dim=dim)):
+            chunks[c] = piece
+    return torch.cat(chunks, dim=dim)
+
+
+def _pairs(q_ids, k_ids):
+    """(local query chunk, visiting key chunk, causal) for every pair with
+    allowed keys: earlier key chunks in full, the same chunk causally."""
+    out = []
+    for a, qa in enumerate(q_ids):
+        for b, kb in enumerate(k_ids):
+            if kb <= qa:
+                out.append((a, b, kb == qa))
+    return out
+
+
+# ----------------------------------------------------------------------------
 # the per-rank algorithm, as generators: ("start", tensors) hands the
 # stepping loop the tensors to pass on to the next rank and gets back a
 # handle; ("wait", handle) returns the tensors received from the previous rank.
 # ----------------------------------------------------------------------------
-def _forward_steps(rank, size, q, k, v, theta, scale, ops):
-    B, n, H, D = q.shape
-    pos0 = rank * n
-    qr = ops.rotate(q, theta, pos0)
-    blk = [ops.rotate(k, theta, pos0), v]
-    o_acc = ops.zeros_f32((B, n, H, D), q.device)
-    lse_acc = ops.full_f32((B, H, n), float("-inf"), q.device)
+def _forward_steps(rank, size, q, k, v, theta, scale, ops, layout):
+    ids = chunk_ids(rank, size, layout)
+    qs = torch.chunk(q, len(ids), dim=1)
+    n = qs[0].shape[1]
+    B, _, H, D = q.shape
+    qr = [ops.rotate(x.contiguous(), theta, g * n) for x, g in zip(qs, ids)]
+    blk = [ops.rotate(x.contiguous(), theta, g * n) for x, g in zip(torch.chunk(k, len(ids), 1), ids)]
+    blk += [x.contiguous() for x in torch.chunk(v, len(ids), dim=1)]
+    o_acc = [ops.zeros_f32((B, n, H, D), q.device) for _ in ids]
+    lse_acc = [ops.full_f32((B, H, n), float("-inf"), q.device) for _ in ids]
+    c = len(ids)
     for s in range(size):
         src = (rank - s) % size
         h = (yield ("start", blk)) if s < size - 1 else None
-        if src <= rank:
-            o_p, lse_p = ops.block_fwd(qr, blk[0], blk[1], src == rank, scale)
-            ops.merge(o_acc, lse_acc, o_p, lse_p)
+        for a, b, causal in _pairs(ids, chunk_ids(src, size, layout)):
+            o_p, lse_p = ops.block_fwd(qr[a], blk[b], blk[c + b], causal, scale)
+            ops.merge(o_acc[a], lse_acc[a], o_p, lse_p)
         if s < size - 1:
             blk = yield ("wait", h)
-    return ops.convert(o_acc, q.dtype), lse_acc
+    o = torch.cat([ops.convert(x, q.dtype) for x in o_acc], dim=1)
+    return o, torch.cat(lse_acc, dim=2)
 
 
-def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops):
-    B, n, H, D = q.shape
-    pos0 = rank * n
-    qr = ops.rotate(q, theta, pos0)
-    dq_acc = ops.zeros_f32((B, n, H, D), q.device)
-    # the visiting block: rotated keys, values and their gradient accumulators
-    blk = [ops.rotate(k, theta, pos0), v, ops.zeros_f32((B, n, H, D), q.device),
-           ops.zeros_f32((B, n, H, D), q.device)]
+def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops, layout):
+    ids = chunk_ids(rank, size, layout)
+    c = len(ids)
+    n = q.shape[1] // c
+    B, _, H, D = q.shape
+    cut = lambda t, dim=1: [x.contiguous() for x in torch.chunk(t, c, dim=dim)]
+    qr = [ops.rotate(x, theta, g * n) for x, g in zip(cut(q), ids)]
+    os_, dos, lses = cut(o), cut(d_o), cut(lse, 2)
+    dq_acc = [ops.zeros_f32((B, n, H, D), q.device) for _ in ids]
+    # the visiting blocks: rotated keys, values and their gradient accumulators
+    blk = [ops.rotate(x, theta, g * n) for x, g in zip(cut(k), ids)] + cut(v)
+    blk += [ops.zeros_f32((B, n, H, D), q.device) for _ in range(2 * c)]
     for s in range(size):
         src = (rank - s) % size
-        if src <= rank:
-            dq_p, dk_p, dv_p = ops.block_bwd(qr, blk[0], blk[1], o, lse, d_o, src == rank, scale)
-            ops.accumulate(dq_acc, dq_p)
-            ops.accumulate(blk[2], dk_p)
-            ops.accumulate(blk[3], dv_p)
+        for a, b, causal in _pairs(ids, chunk_ids(src, size, layout)):
+            dq_p, dk_p, dv_p = ops.block_bwd(qr[a], blk[b], blk[c + b], os_[a], lses[a], dos[a],
+                                             causal, scale)
+            ops.accumulate(dq_acc[a], dq_p)
+            ops.accumulate(blk[2 * c + b], dk_p)
+            ops.accumulate(blk[3 * c + b], dv_p)
         # N shifts in all: after the last one every block is home with its sums
         h = yield ("start", blk)
         blk = yield ("wait", h)
-    dq = ops.convert(ops.rotate(dq_acc, theta, pos0, inverse=True), q.dtype)
-    dk = ops.convert(ops.rotate(blk[2], theta, pos0, inverse=True), k.dtype)
-    dv = ops.convert(blk[3], v.dtype)
+    dq = torch.cat([ops.convert(ops.rotate(x, theta, g * n, inverse=True), q.dtype)
+                    for x, g in zip(dq_acc, ids)], dim=1)
+    dk = torch.cat([ops.convert(ops.rotate(blk[2 * c + b], theta, g * n, inverse=True), k.dtype)
+                    for b, g in enumerate(ids)], dim=1)
+    dv = torch.cat([ops.convert(blk[3 * c + b], v.dtype) for b in range(c)], dim=1)
     return dq, dk, dv
 
 
@@ -166,40 +228,44 @@ def _run_emulated(gens):
         msgs = [outgoing[(r - 1) % size] for r in range(size)]
 
 
-def ring_forward(q, k, v, rope_theta=1e4, softmax_scale=0.0, group=None, ops=None):
-    """This rank's block of O (dtype of q) and LSE [B, H, n] (fp32) for causal
-    attention over the sequence formed by all ranks' blocks in rank order."""
+def ring_forward(q, k, v, rope_theta=1e4, softmax_scale=0.0, group=None, ops=None,
+                 layout="zigzag"):
+    """This rank's part of O (dtype of q) and LSE [B, H, n] (fp32) for causal
+    attention over the whole sequence; the rank holds the chunks
+    ``chunk_ids(rank, size, layout)`` (see split_for_ranks)."""
     import torch.distributed as dist
     ops = ops or GpuBlockOps()
     gen = _forward_steps(dist.get_rank(group), dist.get_world_size(group), q, k, v,
-                         rope_theta, softmax_scale, ops)
+                         rope_theta, softmax_scale, ops, layout)
     return _run_distributed(gen, group)
 
 
-def ring_backward(q, k, v, o, lse, d_o, rope_theta=1e4, softmax_scale=0.0, group=None, ops=None):
-    """This rank's blocks of dq, dk, dv (gradients w.r.t. the un-rotated inputs)."""
+def ring_backward(q, k, v, o, lse, d_o, rope_theta=1e4, softmax_scale=0.0, group=None,
+                  ops=None, layout="zigzag"):
+    """This rank's parts of dq, dk, dv (gradients w.r.t. the un-rotated inputs)."""
     import torch.distributed as dist
     ops = ops or GpuBlockOps()
     gen = _backward_steps(dist.get_rank(group), dist.get_world_size(group), q, k, v, o, lse, d_o,
-                          rope_theta, softmax_scale, ops)
+                          rope_theta, softmax_scale, ops, layout)
     return _run_distributed(gen, group)
 
 
 def emulated_ring_forward(q_blocks, k_blocks, v_blocks, rope_theta=1e4, softmax_scale=0.0,
-                          ops=None):
-    """The ring forward for N virtual ranks on one device (lists of blocks)."""
+                          ops=None, layout="zigzag"):
+    """The ring forward for N virtual ranks on one device (lists of the ranks'
+    local tensors, as split_for_ranks cuts them)."""
     ops = ops or GpuBlockOps()
     n = len(q_blocks)
     gens = [_forward_steps(r, n, q_blocks[r], k_blocks[r], v_blocks[r], rope_theta,
-                           softmax_scale, ops) for r in range(n)]
+                           softmax_scale, ops, layout) for r in range(n)]
     return _run_emulated(gens)
 
 
 def emulated_ring_backward(q_blocks, k_blocks, v_blocks, o_blocks, lse_blocks, do_blocks,
-                           rope_theta=1e4, softmax_scale=0.0, ops=None):
+                           rope_theta=1e4, softmax_scale=0.0, ops=None, layout="zigzag"):
     ops = ops or GpuBlockOps()
     n = len(q_blocks)
     gens = [_backward_steps(r, n, q_blocks[r], k_blocks[r], v_blocks[r], o_blocks[r],
-                            lse_blocks[r], do_blocks[r], rope_theta, softmax_scale, ops)
+                            lse_blocks[r], do_blocks[r], rope_theta, softmax_scale, ops, layout)
             for r in range(n)]
     return _run_emulated(gens)

@@ -1,7 +1,8 @@
 """Ring (sequence-parallel) attention on one GPU: N virtual ranks in lockstep.
 
-The sequence is split into N blocks; the ring runs the library's block
-kernels (rotation at each block's offset, lwm_attn_fwd / lwm_attn_bwd on the
+The sequence is split into N blocks (contiguous layout) or 2N chunks
+(zigzag layout, two per rank); the ring runs the library's block kernels
+(rotation at each chunk's offset, lwm_attn_fwd / lwm_attn_bwd on the
 rotated blocks, the log-sum-exp merge, fp32 gradient accumulation) exactly
 as N ranks would, with the shift between ranks a rotation of a list.  The
 result must match the float64 oracle on the whole sequence.
@@ -16,8 +17,9 @@ from tests.parity_util import assert_close, to64
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("n_ranks,n,theta", [(4, 256, 1e6), (3, 384, 1e7), (2, 200, 1e4)])
-def test_emulated_ring_matches_oracle(n_ranks, n, theta):
+@pytest.mark.parametrize("n_ranks,n,theta,layout", [(4, 256, 1e6, "zigzag"), (3, 384, 1e7, "contiguous"),
+                                                   (2, 200, 1e4, "zigzag"), (4, 128, 1e6, "contiguous")])
+def test_emulated_ring_matches_oracle(n_ranks, n, theta, layout):
     from long_context_causal_attention_b200 import ring
     B, H, D = 1, 4, 128
     S = n_ranks * n
@@ -26,14 +28,14 @@ def test_emulated_ring_matches_oracle(n_ranks, n, theta):
     q, k, v = ((torch.randn((B, S, H, D), generator=g, device="cuda") * 0.5).to(torch.bfloat16)
                for _ in range(3))
     do = torch.randn((B, S, H, D), generator=g, device="cuda").to(torch.bfloat16)
-    split = lambda t: [t[:, r * n:(r + 1) * n].contiguous() for r in range(n_ranks)]
-    res = ring.emulated_ring_forward(split(q), split(k), split(v), theta)
-    o = torch.cat([r[0] for r in res], dim=1)
-    lse = torch.cat([r[1] for r in res], dim=2)
+    split = lambda t, dim=1: ring.split_for_ranks(t, n_ranks, layout, dim)
+    res = ring.emulated_ring_forward(split(q), split(k), split(v), theta, layout=layout)
+    o = ring.merge_from_ranks([r[0] for r in res], layout)
+    lse = ring.merge_from_ranks([r[1] for r in res], layout, dim=2)
     grads = ring.emulated_ring_backward(split(q), split(k), split(v), [r[0] for r in res],
-                                        [r[1] for r in res], split(do), theta)
+                                        [r[1] for r in res], split(do), theta, layout=layout)
     torch.cuda.synchronize()
-    dq, dk, dv = (torch.cat([gr[i] for gr in grads], dim=1) for i in range(3))
+    dq, dk, dv = (ring.merge_from_ranks([gr[i] for gr in grads], layout) for i in range(3))
     ref = oracle.attention_backward(to64(q), to64(k), to64(v), to64(do), None, causal=True,
                                     theta=theta)
     assert_close("o", to64(o), ref["o"], "bf16")

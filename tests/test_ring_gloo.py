@@ -81,32 +81,36 @@ def _inputs(S, seed=7):
     return [rng.standard_normal((1, S, 2, 8)) for _ in range(4)]  # q, k, v, dO
 
 
-def _worker(rank, size, port, n, theta, out):
+def _worker(rank, size, port, n, theta, layout, out):
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=size,
                             timeout=datetime.timedelta(seconds=60))
     try:
         from long_context_causal_attention_b200 import ring as mod
-        q, k, v, do = (torch.from_numpy(a[:, rank * n:(rank + 1) * n].copy()) for a in _inputs(size * n))
+        q, k, v, do = (mod.split_for_ranks(torch.from_numpy(a), size, layout)[rank]
+                       for a in _inputs(size * n))
         ops = CpuBlockOps()
-        o, lse = mod.ring_forward(q, k, v, theta, ops=ops)
-        dq, dk, dv = mod.ring_backward(q, k, v, o, lse, do, theta, ops=ops)
+        o, lse = mod.ring_forward(q, k, v, theta, ops=ops, layout=layout)
+        dq, dk, dv = mod.ring_backward(q, k, v, o, lse, do, theta, ops=ops, layout=layout)
         out.put((rank, o.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("size,n", [(2, 24), (3, 16)])
-def test_ring_on_gloo_ranks_matches_oracle(size, n):
+@pytest.mark.parametrize("size,n,layout", [(2, 24, "contiguous"), (3, 16, "contiguous"),
+                                           (2, 24, "zigzag"), (3, 18, "zigzag")])
+def test_ring_on_gloo_ranks_matches_oracle(size, n, layout):
     import oracle
+    from long_context_causal_attention_b200 import ring
     theta = 300.0
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
-    procs = [ctx.Process(target=_worker, args=(r, size, port, n, theta, out)) for r in range(size)]
+    procs = [ctx.Process(target=_worker, args=(r, size, port, n, theta, layout, out))
+             for r in range(size)]
     for p in procs:
         p.start()
     res = sorted((out.get(timeout=120) for _ in range(size)), key=lambda t: t[0])
@@ -115,7 +119,8 @@ def test_ring_on_gloo_ranks_matches_oracle(size, n):
     assert all(p.exitcode == 0 for p in procs)
     q, k, v, do = _inputs(size * n)
     ref = oracle.attention_backward(q, k, v, do, None, causal=True, theta=theta)
-    cat = lambda i, ax: np.concatenate([r[i] for r in res], axis=ax)
+    cat = lambda i, ax: ring.merge_from_ranks([torch.from_numpy(r[i]) for r in res], layout,
+                                              dim=ax).numpy()
     np.testing.assert_allclose(cat(1, 1), ref["o"], atol=1e-10)
     np.testing.assert_allclose(cat(2, 2), ref["lse"], atol=1e-10)
     np.testing.assert_allclose(cat(3, 1), ref["dq"], atol=1e-10)
