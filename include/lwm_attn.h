@@ -224,6 +224,22 @@ uint64_t lwm_attn_kernel_launches(void);
  *   o_part [B,S,H,D] of `dtype`, lse_part [B,H,S].  A -inf side adds nothing.
  * lwm_accumulate: acc[i] += x[i] for n elements (acc fp32, x of `dtype`).
  * lwm_convert_f32: y[i] = x[i] rounded to `dtype` (nearest even). */
+/* lwm_attn_fwd_pair / lwm_attn_bwd_pair: lwm_attn_fwd / lwm_attn_bwd for a
+ *   block pair of a packed ring: queries of one block (segment ids
+ *   desc->segment_ids) against the keys and values of another block of the
+ *   same length (segment ids k_segment_ids), row i attending key j when their
+ *   ids match (and j <= i if causal, for the diagonal pair).  Both id arrays
+ *   or neither (LWM_ERR_INVALID_ARG otherwise); k_segment_ids [B, S], device,
+ *   4-byte aligned.  Same workspace size, buffers, errors and outputs as the
+ *   single-block calls, which are the case k_segment_ids = segment_ids. */
+lwm_status lwm_attn_fwd_pair(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                             const void* q, const void* k, const void* v, void* o, float* lse,
+                             void* ws, size_t ws_bytes, void* stream);
+lwm_status lwm_attn_bwd_pair(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                             const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* d_o, void* dq, void* dk, void* dv,
+                             void* ws, size_t ws_bytes, void* stream);
+
 lwm_status lwm_rope_apply_at(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
                              int32_t dtype, double theta, int64_t position_offset, const void* x,
                              void* y, int inverse, void* stream);

@@ -30,7 +30,8 @@ ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_
                 "lwm_attn_read_status", "lwm_status_string", "lwm_attn_set_timing_events",
                 "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc",
                 "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait",
-                "lwm_rope_apply_at", "lwm_attn_merge", "lwm_accumulate", "lwm_convert_f32")
+                "lwm_rope_apply_at", "lwm_attn_merge", "lwm_accumulate", "lwm_convert_f32",
+                "lwm_attn_fwd_pair", "lwm_attn_bwd_pair")
 DECODE_MAX_NEW = 16
 
 
@@ -87,6 +88,12 @@ def _load():
     lib.lwm_attn_decode.restype = ctypes.c_int
     lib.lwm_attn_selftest_wait.argtypes = [P, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int, P]
     lib.lwm_attn_selftest_wait.restype = ctypes.c_int
+    lib.lwm_attn_fwd_pair.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P, P,
+                                      ctypes.c_size_t, P]
+    lib.lwm_attn_fwd_pair.restype = ctypes.c_int
+    lib.lwm_attn_bwd_pair.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P, P, P, P, P,
+                                      P, ctypes.c_size_t, P]
+    lib.lwm_attn_bwd_pair.restype = ctypes.c_int
     lib.lwm_rope_apply_at.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int32, ctypes.c_double,
                                       ctypes.c_int64, P, P, ctypes.c_int, P]
@@ -256,6 +263,57 @@ def lwm_attn_decode(q_new, k_cache, v_cache, segment_ids=None, causal=True, rope
     if check_status:
         _check(lwm_attn_read_status(workspace, stream), "lwm_attn_decode (device status)")
     return o, lse
+
+
+def _kseg_ptr(k_segment_ids, q):
+    if k_segment_ids is None:
+        return None
+    _cuda(k_segment_ids, "k_segment_ids")
+    if k_segment_ids.dtype != torch.int32 or tuple(k_segment_ids.shape) != tuple(q.shape[:2]):
+        raise ValueError("k_segment_ids must be int32 [B, S]")
+    return k_segment_ids.data_ptr()
+
+
+def lwm_attn_fwd_pair(q, k, v, segment_ids, k_segment_ids, causal=True, rope_theta=1e4,
+                      softmax_scale=0.0, o=None, lse=None, workspace=None, stream=None):
+    """lwm_attn_fwd for a block pair: query ids ``segment_ids``, key ids
+    ``k_segment_ids`` (both or neither)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, name)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    desc = make_desc(q, segment_ids, causal, rope_theta, softmax_scale)
+    B, S, H, D = q.shape
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    workspace = alloc_workspace(desc, False, q.device) if workspace is None else workspace
+    _check(_lib.lwm_attn_fwd_pair(ctypes.byref(desc), _kseg_ptr(k_segment_ids, q), q.data_ptr(),
+                                  k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "lwm_attn_fwd_pair")
+    return o, lse
+
+
+def lwm_attn_bwd_pair(q, k, v, o, lse, d_o, segment_ids, k_segment_ids, causal=True,
+                      rope_theta=1e4, softmax_scale=0.0, dq=None, dk=None, dv=None,
+                      workspace=None, stream=None):
+    """lwm_attn_bwd for a block pair (see lwm_attn_fwd_pair)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("d_o", d_o)):
+        _cuda(t, name)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    _cuda(lse, "lse")
+    desc = make_desc(q, segment_ids, causal, rope_theta, softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    workspace = alloc_workspace(desc, True, q.device) if workspace is None else workspace
+    _check(_lib.lwm_attn_bwd_pair(ctypes.byref(desc), _kseg_ptr(k_segment_ids, q), q.data_ptr(),
+                                  k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  d_o.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "lwm_attn_bwd_pair")
+    return dq, dk, dv
 
 
 def lwm_rope_apply(x, theta, inverse=False, out=None, stream=None):

@@ -64,6 +64,12 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
   const size_t tiles = (size_t)p.B * (size_t)p.n_tiles * sizeof(int32_t);
   w.tile_min = static_cast<int32_t*>(take(tiles));
   w.tile_max = static_cast<int32_t*>(take(tiles));
+  w.ktile_min = static_cast<int32_t*>(take(tiles));
+  w.ktile_max = static_cast<int32_t*>(take(tiles));
+  if (p.kseg == p.seg) {
+    w.ktile_min = w.tile_min;
+    w.ktile_max = w.tile_max;
+  }
   w.q_lo = static_cast<int32_t*>(take(tiles));
   w.k_hi = static_cast<int32_t*>(take(tiles));
   const size_t nel = (size_t)p.B * p.S * p.H * p.D;
@@ -98,6 +104,8 @@ size_t layout_decode_workspace(const Problem& p, int64_t n_new, void* base, Work
   const size_t tiles = (size_t)p.B * (size_t)p.n_tiles * sizeof(int32_t);
   w.tile_min = static_cast<int32_t*>(take(tiles));
   w.tile_max = static_cast<int32_t*>(take(tiles));
+  w.ktile_min = w.tile_min;
+  w.ktile_max = w.tile_max;
   const size_t parts = (size_t)p.B * p.H * (size_t)n_new *
                        (size_t)((p.S + kDecodeChunk - 1) / kDecodeChunk);
   w.dec_ml = static_cast<float*>(take(parts * 2 * sizeof(float)));
@@ -130,6 +138,7 @@ lwm_status make_problem(const lwm_attn_desc* d, Problem* p) {
   p->theta = d->rope_theta;
   p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / std::sqrt((double)d->head_dim));
   p->seg = d->segment_ids;
+  p->kseg = d->segment_ids;
   p->n_tiles = (d->seqlen + kTile - 1) / kTile;
   p->elt = d->dtype == LWM_DTYPE_BF16 ? 2 : 4;
   return LWM_OK;
@@ -166,21 +175,23 @@ cudaError_t prologue(const Problem& p, Workspace& w, const void* q, const void* 
 }  // namespace
 }  // namespace lwm
 
-using namespace lwm;
-
-extern "C" {
-
-size_t lwm_attn_workspace_size(const lwm_attn_desc* desc, int is_bwd) {
-  Problem p{};
-  if (make_problem(desc, &p) != LWM_OK) return 0;
-  return layout_workspace(p, is_bwd != 0, nullptr, nullptr);
+namespace lwm {
+namespace {
+// Key segment ids of a block pair: both id arrays or neither.
+lwm_status set_key_segments(Problem* p, const int32_t* k_segment_ids) {
+  if ((p->seg == nullptr) != (k_segment_ids == nullptr)) return LWM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(k_segment_ids) & 3u) return LWM_ERR_ALIGNMENT;
+  p->kseg = k_segment_ids;
+  return LWM_OK;
 }
 
-lwm_status lwm_attn_fwd(const lwm_attn_desc* desc, const void* q, const void* k, const void* v,
-                        void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_ids,
+                    const void* q, const void* k, const void* v, void* o, float* lse, void* ws,
+                    size_t ws_bytes, void* stream) {
   Problem p{};
   lwm_status s = make_problem(desc, &p);
   if (s != LWM_OK) return s;
+  if (k_segment_ids && (s = set_key_segments(&p, *k_segment_ids)) != LWM_OK) return s;
   if (p.B * p.S == 0) return LWM_OK;
   if (!q || !k || !v || !o || !lse) return LWM_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -200,12 +211,14 @@ lwm_status lwm_attn_fwd(const lwm_attn_desc* desc, const void* q, const void* k,
   return cuda_status(e);
 }
 
-lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k, const void* v,
-                        const void* o, const float* lse, const void* d_o, void* dq, void* dk,
-                        void* dv, void* ws, size_t ws_bytes, void* stream) {
+lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_ids,
+                    const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* d_o, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                    void* stream) {
   Problem p{};
   lwm_status s = make_problem(desc, &p);
   if (s != LWM_OK) return s;
+  if (k_segment_ids && (s = set_key_segments(&p, *k_segment_ids)) != LWM_OK) return s;
   if (p.B * p.S == 0) return LWM_OK;
   if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv) return LWM_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
@@ -233,6 +246,44 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
   e = launch_simt_bwd(p, w, v, lse, d_o, dq, dk, dv, st);
   record_event(3, st);
   return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace lwm
+
+using namespace lwm;
+
+extern "C" {
+
+size_t lwm_attn_workspace_size(const lwm_attn_desc* desc, int is_bwd) {
+  Problem p{};
+  if (make_problem(desc, &p) != LWM_OK) return 0;
+  return layout_workspace(p, is_bwd != 0, nullptr, nullptr);
+}
+
+
+lwm_status lwm_attn_fwd(const lwm_attn_desc* desc, const void* q, const void* k, const void* v,
+                        void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return attn_fwd(desc, nullptr, q, k, v, o, lse, ws, ws_bytes, stream);
+}
+
+lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* d_o, void* dq, void* dk,
+                        void* dv, void* ws, size_t ws_bytes, void* stream) {
+  return attn_bwd(desc, nullptr, q, k, v, o, lse, d_o, dq, dk, dv, ws, ws_bytes, stream);
+}
+
+lwm_status lwm_attn_fwd_pair(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                             const void* q, const void* k, const void* v, void* o, float* lse,
+                             void* ws, size_t ws_bytes, void* stream) {
+  return attn_fwd(desc, &k_segment_ids, q, k, v, o, lse, ws, ws_bytes, stream);
+}
+
+lwm_status lwm_attn_bwd_pair(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                             const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* d_o, void* dq, void* dk, void* dv,
+                             void* ws, size_t ws_bytes, void* stream) {
+  return attn_bwd(desc, &k_segment_ids, q, k, v, o, lse, d_o, dq, dk, dv, ws, ws_bytes, stream);
 }
 
 size_t lwm_attn_decode_workspace_size(const lwm_attn_desc* desc, int64_t n_new) {

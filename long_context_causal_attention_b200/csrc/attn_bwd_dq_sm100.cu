@@ -74,9 +74,12 @@ enum : uint32_t {
 constexpr uint32_t kItemSlots = 4;
 
 struct DqParams {
-  const int32_t* seg;
-  const int32_t* tmin;
+  const int32_t* seg;    // query segment ids [B, S] or null
+  const int32_t* kseg;   // key segment ids (seg unless a block pair)
+  const int32_t* tmin;   // query tile bounds
   const int32_t* tmax;
+  const int32_t* ktmin;  // key tile bounds
+  const int32_t* ktmax;
   const int32_t* q_lo;
   const float* lse2;   // [B, H, nT*128]: LSE * log2(e), +inf where the row has no keys
   const float* dpad;   // [B, H, nT*128]: dot(dO, O), 0 past the end
@@ -124,7 +127,7 @@ __device__ __forceinline__ bool rel(const DqParams& p, const Item& it, int j) {
   if (j < it.lo || j > it.hi) return false;
   if (!p.seg) return true;
   const size_t kj = (size_t)it.b * p.n_tiles + j;
-  return meet(it.qmin, it.qmax, p.tmin[kj], p.tmax[kj]);
+  return meet(it.qmin, it.qmax, p.ktmin[kj], p.ktmax[kj]);
 }
 
 __device__ __forceinline__ int next_rel(const DqParams& p, const Item& it, int j) {
@@ -387,7 +390,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                        ((int64_t)(it.i + 1) * 128 > p.S);
         if (p.seg) {
           const size_t kj = (size_t)it.b * p.n_tiles + j;
-          const int32_t a0 = p.tmin[kj], a1 = p.tmax[kj];
+          const int32_t a0 = p.ktmin[kj], a1 = p.ktmax[kj];
           partial |= !(it.qmin >= 0 && it.qmin == it.qmax && a0 == it.qmin && a1 == it.qmin);
         }
         uint32_t mw = 0xffffffffu;
@@ -404,8 +407,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           if (seg_q < 0) hi = 0;
           uint32_t bits = bit_range(0, hi);
           if (p.seg) {  // lane c loads the id of key column k0 + c
-            const int32_t kseg = lane < kvalid ? __ldg(p.seg + (size_t)it.b * p.S + k0 + lane) : INT_MIN;
-            bits &= warp_segment_bits(kseg, seg_q);
+            const int32_t kid = lane < kvalid ? __ldg(p.kseg + (size_t)it.b * p.S + k0 + lane) : INT_MIN;
+            bits &= warp_segment_bits(kid, seg_q);
           }
           mw = bits;
         }
@@ -523,8 +526,11 @@ cudaError_t launch_sm100_bwd_dq(const Problem& pb, const Workspace& ws, const vo
   p.q_rot = static_cast<const __nv_bfloat16*>(ws.q_rot);
   p.d_o = static_cast<const __nv_bfloat16*>(d_o);
   p.seg = pb.seg;
+  p.kseg = pb.kseg;
   p.tmin = ws.tile_min;
   p.tmax = ws.tile_max;
+  p.ktmin = ws.ktile_min;
+  p.ktmax = ws.ktile_max;
   p.q_lo = ws.q_lo;
   p.lse2 = ws.lse2_pad;
   p.dpad = ws.delta_pad;

@@ -88,9 +88,12 @@ constexpr uint32_t kItemSlots = 4;
 constexpr uint32_t kEWWarps = kEW / 32;  // element-wise barriers take one arrival per warp
 
 struct BwdParams {
-  const int32_t* seg;
-  const int32_t* tmin;
+  const int32_t* seg;    // query segment ids [B, S] or null
+  const int32_t* kseg;   // key segment ids (seg unless a block pair)
+  const int32_t* tmin;   // query tile bounds
   const int32_t* tmax;
+  const int32_t* ktmin;  // key tile bounds
+  const int32_t* ktmax;
   const int32_t* k_hi;
   const float* lse2;   // [B, H, nT*128]: LSE * log2(e), +inf where the row has no keys
   const float* dpad;   // [B, H, nT*128]: dot(dO, O), 0 past the end
@@ -127,8 +130,8 @@ __device__ __forceinline__ Item decode(const BwdParams& p, int idx) {
   if (p.seg) {
     const size_t kj = (size_t)it.b * p.n_tiles + it.j;
     it.hi = p.k_hi[kj];
-    it.kmin = p.tmin[kj];
-    it.kmax = p.tmax[kj];
+    it.kmin = p.ktmin[kj];
+    it.kmax = p.ktmax[kj];
   }
   return it;
 }
@@ -361,7 +364,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const Item it = decode(p, idx);
       const int64_t key = (int64_t)it.j * 128 + row;
       const bool key_ok = key < p.S;
-      const int32_t seg_k = key_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + key] : 0) : -1;
+      const int32_t seg_k = key_ok ? (p.seg ? p.kseg[(size_t)it.b * p.S + key] : 0) : -1;
       int n = 0;
       for (int i = it.lo; i <= it.hi; ++i) {
         if (!rel(p, it, i)) continue;
@@ -575,8 +578,11 @@ cudaError_t launch_sm100_bwd_dkdv(const Problem& pb, const Workspace& ws, const 
     return cudaErrorInvalidValue;
   BwdParams p{};
   p.seg = pb.seg;
+  p.kseg = pb.kseg;
   p.tmin = ws.tile_min;
   p.tmax = ws.tile_max;
+  p.ktmin = ws.ktile_min;
+  p.ktmax = ws.ktile_max;
   p.k_hi = ws.k_hi;
   p.lse2 = ws.lse2_pad;
   p.dpad = ws.delta_pad;

@@ -74,9 +74,12 @@ constexpr uint32_t kItemSlots = 4;
 constexpr uint32_t kSoftmaxWarps = 8;
 
 struct FwdParams {
-  const int32_t* seg;    // [B, S] or null
-  const int32_t* tmin;   // [B, nT] (valid when seg != null)
+  const int32_t* seg;    // [B, S] query segment ids, or null
+  const int32_t* kseg;   // [B, S] key segment ids (seg unless a block pair)
+  const int32_t* tmin;   // [B, nT] query tile bounds (valid when seg != null)
   const int32_t* tmax;
+  const int32_t* ktmin;  // [B, nT] key tile bounds
+  const int32_t* ktmax;
   const int32_t* q_lo;
   __nv_bfloat16* o;
   float* lse;
@@ -127,7 +130,7 @@ __device__ __forceinline__ bool rel(const FwdParams& p, const Item& it, int t, i
   if (it.qt[t] < 0 || j < it.lo[t] || j > it.hi[t]) return false;
   if (!p.seg) return true;
   const size_t kj = (size_t)it.b * p.n_tiles + j;
-  return meet(it.qmin[t], it.qmax[t], p.tmin[kj], p.tmax[kj]);
+  return meet(it.qmin[t], it.qmax[t], p.ktmin[kj], p.ktmax[kj]);
 }
 
 __device__ __forceinline__ bool rel_any(const FwdParams& p, const Item& it, int j) {
@@ -401,7 +404,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool partial = (p.causal && j == it.qt[t]) || ((int64_t)(j + 1) * 128 > p.S);
         if (p.seg) {
           const size_t kj = (size_t)it.b * p.n_tiles + j;
-          const int32_t a0 = p.tmin[kj], a1 = p.tmax[kj];
+          const int32_t a0 = p.ktmin[kj], a1 = p.ktmax[kj];
           partial |= !(it.qmin[t] >= 0 && it.qmin[t] == it.qmax[t] && a0 == it.qmin[t] &&
                        a1 == it.qmin[t]);
         }
@@ -428,7 +431,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // 128-bit keep mask, built without touching the score registers:
           // keys 32w + c <= lim, and (packing) the row's segment, one load per
           // lane per 32 keys
-          const int32_t* ks = p.seg ? p.seg + (size_t)it.b * p.S + (size_t)j * 128 : nullptr;
+          const int32_t* ks = p.seg ? p.kseg + (size_t)it.b * p.S + (size_t)j * 128 : nullptr;
           uint32_t mw[4];
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
@@ -613,8 +616,11 @@ cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void*
     return cudaErrorInvalidValue;
   FwdParams p{};
   p.seg = pb.seg;
+  p.kseg = pb.kseg;
   p.tmin = ws.tile_min;
   p.tmax = ws.tile_max;
+  p.ktmin = ws.ktile_min;
+  p.ktmax = ws.ktile_max;
   p.q_lo = ws.q_lo;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;

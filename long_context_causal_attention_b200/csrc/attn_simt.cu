@@ -77,8 +77,9 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128)
 simt_fwd_kernel(const T* __restrict__ qr, const T* __restrict__ kr, const T* __restrict__ v,
                 T* __restrict__ o, float* __restrict__ lse, const int32_t* __restrict__ seg,
-                const int32_t* __restrict__ tmin, const int32_t* __restrict__ tmax, int64_t S,
-                int H, int64_t n_tiles, float scale_log2, int causal) {
+                const int32_t* __restrict__ kseg, const int32_t* __restrict__ ktmin,
+                const int32_t* __restrict__ ktmax, int64_t S, int H, int64_t n_tiles,
+                float scale_log2, int causal) {
   constexpr int DPL = D / 32;
   __shared__ float qs[4][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,12 +99,12 @@ simt_fwd_kernel(const T* __restrict__ qr, const T* __restrict__ kr, const T* __r
   if (si >= 0) {
     const int64_t kend = causal ? i + 1 : S;
     for (int64_t t0 = 0; t0 < kend; t0 += kTile) {
-      if (seg && !tile_may_hold(tmin, tmax, b * n_tiles + t0 / kTile, si)) continue;
+      if (seg && !tile_may_hold(ktmin, ktmax, b * n_tiles + t0 / kTile, si)) continue;
       const int64_t t1 = min(t0 + (int64_t)kTile, kend);
       for (int64_t j0 = t0; j0 < t1; j0 += 32) {
         const int64_t j = j0 + lane;
         float s = -INFINITY;
-        if (j < t1 && (!seg || seg[(size_t)b * S + j] == si))
+        if (j < t1 && (!seg || kseg[(size_t)b * S + j] == si))
           s = dot_row<T, D>(qs[warp], kr + ((size_t)b * S + j) * rs + (size_t)h * D) * scale_log2;
         const float mnew = fmaxf(m, warp_max(s));
         if (mnew == -INFINITY) continue;
@@ -137,7 +138,8 @@ __global__ void __launch_bounds__(128)
 simt_bwd_dq_kernel(const T* __restrict__ qr, const T* __restrict__ kr, const T* __restrict__ v,
                    const T* __restrict__ d_o, const float* __restrict__ lse,
                    const float* __restrict__ delta, const int32_t* __restrict__ seg,
-                   const int32_t* __restrict__ tmin, const int32_t* __restrict__ tmax,
+                   const int32_t* __restrict__ kseg, const int32_t* __restrict__ ktmin,
+                   const int32_t* __restrict__ ktmax,
                    T* __restrict__ dq, int64_t S, int H, int64_t n_tiles, float scale,
                    float scale_log2, int causal, double log2_theta, int rotate) {
   constexpr int DPL = D / 32;
@@ -166,12 +168,12 @@ simt_bwd_dq_kernel(const T* __restrict__ qr, const T* __restrict__ kr, const T* 
     const float Di = delta[srow];
     const int64_t kend = causal ? i + 1 : S;
     for (int64_t t0 = 0; t0 < kend; t0 += kTile) {
-      if (seg && !tile_may_hold(tmin, tmax, b * n_tiles + t0 / kTile, si)) continue;
+      if (seg && !tile_may_hold(ktmin, ktmax, b * n_tiles + t0 / kTile, si)) continue;
       const int64_t t1 = min(t0 + (int64_t)kTile, kend);
       for (int64_t j0 = t0; j0 < t1; j0 += 32) {
         const int64_t j = j0 + lane;
         float ds = 0.f;
-        if (j < t1 && (!seg || seg[(size_t)b * S + j] == si)) {
+        if (j < t1 && (!seg || kseg[(size_t)b * S + j] == si)) {
           const size_t kro = ((size_t)b * S + j) * rs + hoff;
           const float p = exp2f(dot_row<T, D>(qs[warp], kr + kro) * scale_log2 - lse2);
           const float dp = dot_row<T, D>(gs[warp], v + kro);
@@ -202,7 +204,8 @@ __global__ void __launch_bounds__(128)
 simt_bwd_dkdv_kernel(const T* __restrict__ qr, const T* __restrict__ kr, const T* __restrict__ v,
                      const T* __restrict__ d_o, const float* __restrict__ lse,
                      const float* __restrict__ delta, const int32_t* __restrict__ seg,
-                     const int32_t* __restrict__ tmin, const int32_t* __restrict__ tmax,
+                     const int32_t* __restrict__ kseg, const int32_t* __restrict__ tmin,
+                     const int32_t* __restrict__ tmax,
                      T* __restrict__ dk, T* __restrict__ dv, int64_t S, int H, int64_t n_tiles,
                      float scale, float scale_log2, int causal, double log2_theta, int rotate) {
   constexpr int DPL = D / 32;
@@ -220,7 +223,7 @@ simt_bwd_dkdv_kernel(const T* __restrict__ qr, const T* __restrict__ kr, const T
     vs[warp][d] = to_f32(v[tok * rs + hoff + d]);
   }
   __syncwarp();
-  const int32_t sj = seg ? seg[tok] : 0;
+  const int32_t sj = seg ? kseg[tok] : 0;
   float ak[DPL], av[DPL];
 #pragma unroll
   for (int u = 0; u < DPL; ++u) ak[u] = av[u] = 0.f;
@@ -276,8 +279,8 @@ cudaError_t fwd_impl(const Problem& p, const Workspace& ws, const void* v, void*
   dim3 grid((unsigned)((p.S + 3) / 4), (unsigned)p.H, (unsigned)p.B);
   simt_fwd_kernel<T, D><<<grid, 128, 0, st>>>(
       static_cast<const T*>(ws.q_rot), static_cast<const T*>(ws.k_rot), static_cast<const T*>(v),
-      static_cast<T*>(o), lse, p.seg, ws.tile_min, ws.tile_max, p.S, (int)p.H, p.n_tiles,
-      p.scale * kLog2e, p.causal);
+      static_cast<T*>(o), lse, p.seg, p.kseg, ws.ktile_min, ws.ktile_max, p.S, (int)p.H,
+      p.n_tiles, p.scale * kLog2e, p.causal);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -290,14 +293,14 @@ cudaError_t bwd_impl(const Problem& p, const Workspace& ws, const void* v, const
   const double l2t = rotate ? log2(p.theta) : 0.0;
   simt_bwd_dq_kernel<T, D><<<grid, 128, 0, st>>>(
       static_cast<const T*>(ws.q_rot), static_cast<const T*>(ws.k_rot), static_cast<const T*>(v),
-      static_cast<const T*>(d_o), lse, ws.delta, p.seg, ws.tile_min, ws.tile_max,
+      static_cast<const T*>(d_o), lse, ws.delta, p.seg, p.kseg, ws.ktile_min, ws.ktile_max,
       static_cast<T*>(dq), p.S, (int)p.H, p.n_tiles, p.scale, p.scale * kLog2e, p.causal, l2t,
       rotate);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   simt_bwd_dkdv_kernel<T, D><<<grid, 128, 0, st>>>(
       static_cast<const T*>(ws.q_rot), static_cast<const T*>(ws.k_rot), static_cast<const T*>(v),
-      static_cast<const T*>(d_o), lse, ws.delta, p.seg, ws.tile_min, ws.tile_max,
+      static_cast<const T*>(d_o), lse, ws.delta, p.seg, p.kseg, ws.tile_min, ws.tile_max,
       static_cast<T*>(dk), static_cast<T*>(dv), p.S, (int)p.H, p.n_tiles, p.scale,
       p.scale * kLog2e, p.causal, l2t, rotate);
   note_launches(2);

@@ -18,7 +18,8 @@ struct Problem {
   int causal;
   double theta;       // <= 0: no rotation
   float scale;        // resolved softmax scale (> 0)
-  const int32_t* seg; // may be null
+  const int32_t* seg; // may be null; segment ids of the queries
+  const int32_t* kseg; // segment ids of the keys: seg itself, except for a block pair
   int64_t n_tiles;    // ceil(S / 128)
   size_t elt;         // bytes per element of dtype
 };
@@ -28,6 +29,8 @@ struct Workspace {
   DeviceStatus* status;
   int32_t* tile_min;   // [B, n_tiles] smallest non-negative id in the tile (INT32_MAX if none)
   int32_t* tile_max;   // [B, n_tiles] largest id in the tile (-1 if none)
+  int32_t* ktile_min;  // the same bounds for the key ids (alias of tile_min/max
+  int32_t* ktile_max;  //   unless the keys carry their own ids)
   int32_t* q_lo;       // [B, n_tiles] first key tile a query tile may need
   int32_t* k_hi;       // [B, n_tiles] last query tile a key tile may feed
   void* q_rot;         // [B, S, H, D] rotated q (dtype)

@@ -46,27 +46,32 @@ __device__ __forceinline__ bool meet(int32_t a0, int32_t a1, int32_t b0, int32_t
   return a1 >= 0 && b1 >= 0 && a0 <= b1 && b0 <= a1;
 }
 
+// q bounds (tmin, tmax) describe the query tiles, k bounds the key tiles
+// (the same arrays unless the keys carry their own segment ids).
 __global__ void tile_ranges_kernel(const int32_t* __restrict__ tmin, const int32_t* __restrict__ tmax,
-                                   int64_t B, int64_t n_tiles, int causal,
-                                   int32_t* __restrict__ q_lo, int32_t* __restrict__ k_hi) {
+                                   const int32_t* __restrict__ ktmin,
+                                   const int32_t* __restrict__ ktmax, int64_t B, int64_t n_tiles,
+                                   int causal, int32_t* __restrict__ q_lo,
+                                   int32_t* __restrict__ k_hi) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * n_tiles) return;
   const int64_t b = idx / n_tiles, t = idx % n_tiles;
   const int32_t* mn = tmin + b * n_tiles;
   const int32_t* mx = tmax + b * n_tiles;
-  const int32_t a0 = mn[t], a1 = mx[t];
+  const int32_t* kmn = ktmin + b * n_tiles;
+  const int32_t* kmx = ktmax + b * n_tiles;
   // first key tile for query tile t
   const int64_t jmax = causal ? t : n_tiles - 1;
   int64_t lo = jmax + 1;
   for (int64_t j = 0; j <= jmax; ++j) {
-    if (meet(a0, a1, mn[j], mx[j])) { lo = j; break; }
+    if (meet(mn[t], mx[t], kmn[j], kmx[j])) { lo = j; break; }
   }
   q_lo[idx] = (int32_t)lo;
   // last query tile for key tile t
   const int64_t imin = causal ? t : 0;
   int64_t hi = imin - 1;
   for (int64_t i = n_tiles - 1; i >= imin; --i) {
-    if (meet(a0, a1, mn[i], mx[i])) { hi = i; break; }
+    if (meet(kmn[t], kmx[t], mn[i], mx[i])) { hi = i; break; }
   }
   k_hi[idx] = (int32_t)hi;
 }
@@ -81,13 +86,19 @@ cudaError_t launch_segment_bounds(const Problem& p, const Workspace& ws, cudaStr
   const int threads = 128;
   const unsigned grid = (unsigned)((n + threads - 1) / threads);
   tile_bounds_kernel<<<grid, threads, 0, st>>>(p.seg, p.B, p.S, p.n_tiles, ws.tile_min, ws.tile_max);
-  if (!ranges) {
-    note_launches(1);
-    return cudaGetLastError();
+  int launched = 1;
+  if (p.kseg != p.seg) {
+    tile_bounds_kernel<<<grid, threads, 0, st>>>(p.kseg, p.B, p.S, p.n_tiles, ws.ktile_min,
+                                                 ws.ktile_max);
+    ++launched;
   }
-  tile_ranges_kernel<<<grid, threads, 0, st>>>(ws.tile_min, ws.tile_max, p.B, p.n_tiles, p.causal,
-                                               ws.q_lo, ws.k_hi);
-  note_launches(2);
+  if (ranges) {
+    tile_ranges_kernel<<<grid, threads, 0, st>>>(ws.tile_min, ws.tile_max, ws.ktile_min,
+                                                 ws.ktile_max, p.B, p.n_tiles, p.causal, ws.q_lo,
+                                                 ws.k_hi);
+    ++launched;
+  }
+  note_launches(launched);
   return cudaGetLastError();
 }
 

@@ -27,8 +27,9 @@ them and moves blocks.  Two stepping loops run the same per-rank algorithm:
 process group (NCCL point-to-point over NVLink; block i+1 is in flight while
 block i is computed), and ``emulated_ring_forward`` / ``..._backward`` for
 N virtual ranks stepped in lockstep on one device (same kernels, the shift
-is a rotation of a list).  Segment ids (packing) are not supported across
-blocks yet.
+is a rotation of a list).  Packed rows: the segment ids of each rank's
+chunks (cut like q) travel with the key blocks, and every block pair is
+masked by query ids against key ids (lwm_attn_fwd_pair / lwm_attn_bwd_pair).
 """
 from __future__ import annotations
 
@@ -43,12 +44,12 @@ class GpuBlockOps:
     def rotate(self, x, theta, pos0, inverse=False):
         return L.lwm_rope_apply_at(x, theta, pos0, inverse)
 
-    def block_fwd(self, q, k, v, causal, scale):
+    def block_fwd(self, q, k, v, causal, scale, q_seg=None, k_seg=None):
         # inputs are rotated already: rope_theta = 0
-        return L.lwm_attn_fwd(q, k, v, None, causal, 0.0, scale)
+        return L.lwm_attn_fwd_pair(q, k, v, q_seg, k_seg, causal, 0.0, scale)
 
-    def block_bwd(self, q, k, v, o, lse, d_o, causal, scale):
-        return L.lwm_attn_bwd(q, k, v, o, lse, d_o, None, causal, 0.0, scale)
+    def block_bwd(self, q, k, v, o, lse, d_o, causal, scale, q_seg=None, k_seg=None):
+        return L.lwm_attn_bwd_pair(q, k, v, o, lse, d_o, q_seg, k_seg, causal, 0.0, scale)
 
     def merge(self, o_acc, lse_acc, o_part, lse_part):
         L.lwm_attn_merge(o_acc, lse_acc, o_part, lse_part)
@@ -118,22 +119,27 @@ def _pairs(q_ids, k_ids):
 # stepping loop the tensors to pass on to the next rank and gets back a
 # handle; ("wait", handle) returns the tensors received from the previous rank.
 # ----------------------------------------------------------------------------
-def _forward_steps(rank, size, q, k, v, theta, scale, ops, layout):
+def _forward_steps(rank, size, q, k, v, theta, scale, ops, layout, seg=None):
     ids = chunk_ids(rank, size, layout)
-    qs = torch.chunk(q, len(ids), dim=1)
+    c = len(ids)
+    qs = torch.chunk(q, c, dim=1)
     n = qs[0].shape[1]
     B, _, H, D = q.shape
     qr = [ops.rotate(x.contiguous(), theta, g * n) for x, g in zip(qs, ids)]
-    blk = [ops.rotate(x.contiguous(), theta, g * n) for x, g in zip(torch.chunk(k, len(ids), 1), ids)]
-    blk += [x.contiguous() for x in torch.chunk(v, len(ids), dim=1)]
+    qseg = [x.contiguous() for x in torch.chunk(seg, c, dim=1)] if seg is not None else [None] * c
+    # the travelling block: rotated keys, values (and the keys' segment ids)
+    blk = [ops.rotate(x.contiguous(), theta, g * n) for x, g in zip(torch.chunk(k, c, 1), ids)]
+    blk += [x.contiguous() for x in torch.chunk(v, c, dim=1)]
+    if seg is not None:
+        blk += qseg
     o_acc = [ops.zeros_f32((B, n, H, D), q.device) for _ in ids]
     lse_acc = [ops.full_f32((B, H, n), float("-inf"), q.device) for _ in ids]
-    c = len(ids)
     for s in range(size):
         src = (rank - s) % size
         h = (yield ("start", blk)) if s < size - 1 else None
         for a, b, causal in _pairs(ids, chunk_ids(src, size, layout)):
-            o_p, lse_p = ops.block_fwd(qr[a], blk[b], blk[c + b], causal, scale)
+            kseg = blk[2 * c + b] if seg is not None else None
+            o_p, lse_p = ops.block_fwd(qr[a], blk[b], blk[c + b], causal, scale, qseg[a], kseg)
             ops.merge(o_acc[a], lse_acc[a], o_p, lse_p)
         if s < size - 1:
             blk = yield ("wait", h)
@@ -141,7 +147,7 @@ def _forward_steps(rank, size, q, k, v, theta, scale, ops, layout):
     return o, torch.cat(lse_acc, dim=2)
 
 
-def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops, layout):
+def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops, layout, seg=None):
     ids = chunk_ids(rank, size, layout)
     c = len(ids)
     n = q.shape[1] // c
@@ -149,15 +155,20 @@ def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops, layout)
     cut = lambda t, dim=1: [x.contiguous() for x in torch.chunk(t, c, dim=dim)]
     qr = [ops.rotate(x, theta, g * n) for x, g in zip(cut(q), ids)]
     os_, dos, lses = cut(o), cut(d_o), cut(lse, 2)
+    qseg = cut(seg) if seg is not None else [None] * c
     dq_acc = [ops.zeros_f32((B, n, H, D), q.device) for _ in ids]
-    # the visiting blocks: rotated keys, values and their gradient accumulators
+    # the travelling block: rotated keys, values, their gradient sums (and the
+    # keys' segment ids)
     blk = [ops.rotate(x, theta, g * n) for x, g in zip(cut(k), ids)] + cut(v)
     blk += [ops.zeros_f32((B, n, H, D), q.device) for _ in range(2 * c)]
+    if seg is not None:
+        blk += qseg
     for s in range(size):
         src = (rank - s) % size
         for a, b, causal in _pairs(ids, chunk_ids(src, size, layout)):
+            kseg = blk[4 * c + b] if seg is not None else None
             dq_p, dk_p, dv_p = ops.block_bwd(qr[a], blk[b], blk[c + b], os_[a], lses[a], dos[a],
-                                             causal, scale)
+                                             causal, scale, qseg[a], kseg)
             ops.accumulate(dq_acc[a], dq_p)
             ops.accumulate(blk[2 * c + b], dk_p)
             ops.accumulate(blk[3 * c + b], dv_p)
@@ -229,43 +240,46 @@ def _run_emulated(gens):
 
 
 def ring_forward(q, k, v, rope_theta=1e4, softmax_scale=0.0, group=None, ops=None,
-                 layout="zigzag"):
+                 layout="zigzag", segment_ids=None):
     """This rank's part of O (dtype of q) and LSE [B, H, n] (fp32) for causal
     attention over the whole sequence; the rank holds the chunks
     ``chunk_ids(rank, size, layout)`` (see split_for_ranks)."""
     import torch.distributed as dist
     ops = ops or GpuBlockOps()
     gen = _forward_steps(dist.get_rank(group), dist.get_world_size(group), q, k, v,
-                         rope_theta, softmax_scale, ops, layout)
+                         rope_theta, softmax_scale, ops, layout, segment_ids)
     return _run_distributed(gen, group)
 
 
 def ring_backward(q, k, v, o, lse, d_o, rope_theta=1e4, softmax_scale=0.0, group=None,
-                  ops=None, layout="zigzag"):
+                  ops=None, layout="zigzag", segment_ids=None):
     """This rank's parts of dq, dk, dv (gradients w.r.t. the un-rotated inputs)."""
     import torch.distributed as dist
     ops = ops or GpuBlockOps()
     gen = _backward_steps(dist.get_rank(group), dist.get_world_size(group), q, k, v, o, lse, d_o,
-                          rope_theta, softmax_scale, ops, layout)
+                          rope_theta, softmax_scale, ops, layout, segment_ids)
     return _run_distributed(gen, group)
 
 
 def emulated_ring_forward(q_blocks, k_blocks, v_blocks, rope_theta=1e4, softmax_scale=0.0,
-                          ops=None, layout="zigzag"):
+                          ops=None, layout="zigzag", seg_blocks=None):
     """The ring forward for N virtual ranks on one device (lists of the ranks'
     local tensors, as split_for_ranks cuts them)."""
     ops = ops or GpuBlockOps()
     n = len(q_blocks)
     gens = [_forward_steps(r, n, q_blocks[r], k_blocks[r], v_blocks[r], rope_theta,
-                           softmax_scale, ops, layout) for r in range(n)]
+                           softmax_scale, ops, layout,
+                           seg_blocks[r] if seg_blocks is not None else None) for r in range(n)]
     return _run_emulated(gens)
 
 
 def emulated_ring_backward(q_blocks, k_blocks, v_blocks, o_blocks, lse_blocks, do_blocks,
-                           rope_theta=1e4, softmax_scale=0.0, ops=None, layout="zigzag"):
+                           rope_theta=1e4, softmax_scale=0.0, ops=None, layout="zigzag",
+                           seg_blocks=None):
     ops = ops or GpuBlockOps()
     n = len(q_blocks)
     gens = [_backward_steps(r, n, q_blocks[r], k_blocks[r], v_blocks[r], o_blocks[r],
-                            lse_blocks[r], do_blocks[r], rope_theta, softmax_scale, ops, layout)
+                            lse_blocks[r], do_blocks[r], rope_theta, softmax_scale, ops, layout,
+                            seg_blocks[r] if seg_blocks is not None else None)
             for r in range(n)]
     return _run_emulated(gens)

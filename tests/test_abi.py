@@ -140,6 +140,22 @@ def test_ring_entry_points_reject_bad_arguments(lwm):
     assert lib.lwm_convert_f32(4, 0, None, P, None) == -1
 
 
+def test_pair_entry_points_need_both_or_neither_segment_arrays(lwm):
+    lib = lwm._lib.lib()
+    P = 0x10000
+    big = 1 << 40
+    with_ids = _desc(lwm, segment_ids=P)
+    no_ids = _desc(lwm)
+    fwd = lambda d, kseg: lib.lwm_attn_fwd_pair(ctypes.byref(d), kseg, P, P, P, P, P, P, big, None)
+    assert fwd(with_ids, None) == -1
+    assert fwd(no_ids, P) == -1
+    assert fwd(with_ids, P + 2) == -3
+    bwd = lambda d, kseg: lib.lwm_attn_bwd_pair(ctypes.byref(d), kseg, P, P, P, P, P, P, P, P, P,
+                                                P, big, None)
+    assert bwd(with_ids, None) == -1
+    assert bwd(_desc(lwm, head_dim=32, segment_ids=P), P) == -2
+
+
 def test_python_binding_requires_cuda_tensors(lwm):
     import torch
     q = torch.zeros(1, 4, 1, 64)

@@ -45,6 +45,42 @@ def test_emulated_ring_matches_oracle(n_ranks, n, theta, layout):
     assert_close("dv", to64(dv), ref["dv"], "bf16")
 
 
+@pytest.mark.parametrize("n_ranks,n,layout", [(4, 256, "zigzag"), (3, 300, "contiguous")])
+def test_emulated_ring_packed_matches_oracle(n_ranks, n, layout):
+    """Packed rows with padding: the segment ids travel with the key blocks and
+    every block pair is masked query ids against key ids."""
+    import numpy as np
+    from long_context_causal_attention_b200 import ring
+    from workloads import random_segments
+    B, H, D, theta = 2, 2, 128, 1e6
+    S = n_ranks * n
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77 + n)
+    q, k, v = ((torch.randn((B, S, H, D), generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+               for _ in range(3))
+    do = torch.randn((B, S, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    seg = random_segments(np.random.default_rng(n), B, S, 40, 500, pad_tail=3)
+    seg_d = torch.as_tensor(seg, dtype=torch.int32, device="cuda")
+    split = lambda t: ring.split_for_ranks(t, n_ranks, layout)
+    segs = split(seg_d)
+    res = ring.emulated_ring_forward(split(q), split(k), split(v), theta, layout=layout,
+                                     seg_blocks=segs)
+    o = ring.merge_from_ranks([r[0] for r in res], layout)
+    lse = ring.merge_from_ranks([r[1] for r in res], layout, dim=2)
+    grads = ring.emulated_ring_backward(split(q), split(k), split(v), [r[0] for r in res],
+                                        [r[1] for r in res], split(do), theta, layout=layout,
+                                        seg_blocks=segs)
+    torch.cuda.synchronize()
+    dq, dk, dv = (ring.merge_from_ranks([gr[i] for gr in grads], layout) for i in range(3))
+    ref = oracle.attention_backward(to64(q), to64(k), to64(v), to64(do), seg, causal=True,
+                                    theta=theta)
+    assert_close("o", to64(o), ref["o"], "bf16")
+    assert_close("lse", to64(lse), ref["lse"], "bf16")
+    assert_close("dq", to64(dq), ref["dq"], "bf16")
+    assert_close("dk", to64(dk), ref["dk"], "bf16")
+    assert_close("dv", to64(dv), ref["dv"], "bf16")
+
+
 def test_merge_kernel_equals_joint_softmax():
     """Merging the results of two key halves equals attention over both."""
     import long_context_causal_attention_b200 as lwm
