@@ -38,6 +38,9 @@ from .attention import (  # noqa: F401
     attention_backward,
     attention_rows,
     attention_decode,
+    sample_runs,
+    packed_loss_weights,
+    packed_cross_entropy,
     kept_pairs,
     attention_flops,
 )

@@ -28,6 +28,14 @@ What it computes, step by step, and where each step comes from:
 
 Scores are materialised one block of query rows at a time so memory stays
 bounded; there is no other blocking, fusion or reordering.
+
+7. Packed loss re-weighting (same section, Masked Sequence Packing: packed
+   training made numerically equal to unpacked training with padding): a
+   sample is a contiguous run of one segment id; each loss token of a sample
+   with n loss tokens weighs 1 / (n * number of samples with a loss token),
+   so the packed loss is the mean over samples of each sample's mean token
+   cross-entropy.  packed_cross_entropy returns that loss and d loss / d
+   logits.
 """
 
 from __future__ import annotations
@@ -317,3 +325,60 @@ def attention_flops(seg, heads: int, head_dim: int, causal=True) -> dict:
     pi = kept_pairs(seg, causal)
     fwd = 4.0 * head_dim * heads * pi
     return {"pairs": pi, "fwd": fwd, "bwd": 2.5 * fwd, "fwd_bwd": 3.5 * fwd}
+
+
+def sample_runs(seg_row):
+    """Samples of one packed row: maximal runs of equal non-negative segment
+    id, as (start, end) index pairs (research note, "训练方法": each packed
+    sample is a contiguous piece of the row)."""
+    seg_row = np.asarray(seg_row)
+    runs, start = [], 0
+    for t in range(1, len(seg_row) + 1):
+        if t == len(seg_row) or seg_row[t] != seg_row[t - 1]:
+            if seg_row[start] >= 0:
+                runs.append((start, t))
+            start = t
+    return runs
+
+
+def packed_loss_weights(seg, targets):
+    """Per-token loss weights that make packed training equal to unpacked
+    training with padding (research note, "训练方法", Masked Sequence
+    Packing, and the ablation of section "评测": naive packing down-weights
+    short samples).  Unpacked training averages each sample's loss over its
+    own loss tokens, then averages over the samples of the batch; so a loss
+    token of a sample with n loss tokens weighs 1 / (n * number of samples
+    that have a loss token).  targets < 0 mark tokens without loss."""
+    seg = np.asarray(seg)
+    targets = np.asarray(targets)
+    w = np.zeros(seg.shape, dtype=np.float64)
+    samples = []
+    for b in range(seg.shape[0]):
+        for s, e in sample_runs(seg[b]):
+            n = int(np.count_nonzero(targets[b, s:e] >= 0))
+            if n:
+                samples.append((b, s, e, n))
+    for b, s, e, n in samples:
+        w[b, s:e] = np.where(targets[b, s:e] >= 0, 1.0 / (n * len(samples)), 0.0)
+    return w
+
+
+def packed_cross_entropy(logits, targets, seg):
+    """Re-weighted cross-entropy of a packed batch and its gradient, float64.
+
+    logits [B, S, V], targets [B, S] (< 0: no loss), seg [B, S].
+    Returns (loss, dlogits): loss = sum_t w_t * (logsumexp(z_t) - z_t[y_t]),
+    dlogits_t = w_t * (softmax(z_t) - onehot(y_t))."""
+    z = np.asarray(logits, dtype=np.float64)
+    targets = np.asarray(targets)
+    w = packed_loss_weights(seg, targets)
+    m = z.max(axis=-1, keepdims=True)
+    lse = m[..., 0] + np.log(np.exp(z - m).sum(axis=-1))
+    y = np.where(targets >= 0, targets, 0)
+    picked = np.take_along_axis(z, y[..., None], axis=-1)[..., 0]
+    loss = float(np.sum(w * (lse - picked)))
+    g = np.exp(z - lse[..., None])
+    onehot = np.zeros_like(z)
+    np.put_along_axis(onehot, y[..., None], 1.0, axis=-1)
+    d = w[..., None] * (g - onehot)
+    return loss, d

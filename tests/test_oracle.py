@@ -477,3 +477,61 @@ def test_decode_oracle_catches_a_position_shift(monkeypatch):
     monkeypatch.setattr(oracle.attention, "rope_apply", shifted)
     o_d, _ = oracle.attention_decode(q[:, S - T:], k, v, None, theta=100.0)
     assert np.abs(o_d - o_f[:, S - T:]).max() > 1e-3
+
+
+# ------------------------------------------------- packed loss re-weighting
+def test_packed_loss_equals_unpacked_per_sample_mean():
+    """The pages' claim: with the re-weighting, packed training equals
+    training on the samples one by one with padding, i.e. the mean over
+    samples of each sample's own mean token loss (computed here per sample,
+    with torch's cross-entropy)."""
+    import torch
+    rng = np.random.default_rng(41)
+    B, S, V = 2, 40, 11
+    seg = np.stack([np.repeat([0, 1, 2, -1], [12, 5, 20, 3]), np.repeat([0, 1], [33, 7])])
+    targets = rng.integers(0, V, size=(B, S))
+    targets[0, :4] = -1          # prompt tokens without loss
+    targets[1, 33:] = -1         # a sample with no loss token at all
+    targets[0, 37:] = -1         # padding
+    z = rng.standard_normal((B, S, V))
+    loss, d = oracle.packed_cross_entropy(z, targets, seg)
+    per_sample = []
+    for b in range(B):
+        for s, e in oracle.sample_runs(seg[b]):
+            keep = targets[b, s:e] >= 0
+            if keep.any():
+                zz = torch.from_numpy(z[b, s:e][keep])
+                yy = torch.from_numpy(targets[b, s:e][keep])
+                per_sample.append(torch.nn.functional.cross_entropy(zz, yy).item())
+    assert len(per_sample) == 4
+    assert abs(loss - np.mean(per_sample)) < 1e-12
+    w = oracle.packed_loss_weights(seg, targets)
+    assert abs(w.sum() - 1.0) < 1e-12 and np.all(w[targets < 0] == 0)
+    # naive packing (token mean) differs: short samples weigh less there
+    naive = np.mean([torch.nn.functional.cross_entropy(
+        torch.from_numpy(z[b][targets[b] >= 0]), torch.from_numpy(targets[b][targets[b] >= 0]),
+        reduction="sum").item() for b in range(B)]) * B / np.count_nonzero(targets >= 0)
+    assert abs(naive - loss) > 1e-3
+
+
+def test_packed_loss_gradient_matches_autograd():
+    import torch
+    rng = np.random.default_rng(42)
+    B, S, V = 2, 17, 7
+    seg = np.stack([np.repeat([0, 1], [9, 8]), np.repeat([4, -1], [15, 2])])
+    targets = rng.integers(0, V, size=(B, S))
+    targets[1, 15:] = -1
+    z = rng.standard_normal((B, S, V))
+    loss, d = oracle.packed_cross_entropy(z, targets, seg)
+    w = torch.from_numpy(oracle.packed_loss_weights(seg, targets))
+    zt = torch.from_numpy(z).requires_grad_(True)
+    y = torch.from_numpy(np.where(targets >= 0, targets, 0))
+    ce = torch.nn.functional.cross_entropy(zt.reshape(-1, V), y.reshape(-1), reduction="none")
+    tl = (ce.reshape(B, S) * w).sum()
+    tl.backward()
+    assert abs(tl.item() - loss) < 1e-12
+    np.testing.assert_allclose(d, zt.grad.numpy(), atol=1e-14)
+
+
+def test_sample_runs_split_equal_ids_in_separate_runs():
+    assert oracle.sample_runs([0, 0, 1, 1, 0, -1, -1, 2]) == [(0, 2), (2, 4), (4, 5), (7, 8)]
