@@ -249,6 +249,28 @@ lwm_status lwm_attn_merge(int64_t batch, int64_t seqlen, int64_t heads, int64_t 
 lwm_status lwm_accumulate(int64_t n, int32_t dtype, float* acc, const void* x, void* stream);
 lwm_status lwm_convert_f32(int64_t n, int32_t dtype, const float* x, void* y, void* stream);
 
+/* ---- Packed loss re-weighting ------------------------------------------
+ * Cross-entropy of a packed batch, re-weighted so that it equals training on
+ * the samples one by one with padding (research note, "训练方法", Masked
+ * Sequence Packing): a sample is a contiguous run of one segment id; a loss
+ * token of a sample with n loss tokens weighs 1 / (n * number of samples
+ * with a loss token).
+ *   logits [B, S, V] (dtype bf16 or fp32, 16-byte aligned), targets [B, S]
+ *   int32 (< 0 or >= V: no loss at that token), segment_ids [B, S] int32
+ *   (NULL: each row is one sample; id < 0: padding, no loss).
+ *   loss: device float, sum over tokens of w_t * (logsumexp(z_t) - z_t[y_t]),
+ *   summed in a fixed order.  dlogits [B, S, V] of dtype (may be NULL):
+ *   w_t * (softmax(z_t) - onehot(y_t)), zero rows for tokens without loss.
+ *   ws: lwm_packed_ce_workspace_size(B, S) bytes, 256-byte aligned.
+ *   V up to 58,112 (a row of fp32 logits in shared memory); larger returns
+ *   LWM_ERR_UNSUPPORTED.  Reads the logits once and writes dlogits once:
+ *   bound by HBM bandwidth. */
+size_t lwm_packed_ce_workspace_size(int64_t batch, int64_t seqlen);
+lwm_status lwm_packed_cross_entropy(int64_t batch, int64_t seqlen, int64_t vocab, int32_t dtype,
+                                    const void* logits, const int32_t* targets,
+                                    const int32_t* segment_ids, float* loss, void* dlogits,
+                                    void* ws, size_t ws_bytes, void* stream);
+
 /* Failure-path self-test (no counterpart on the pages).  Clears the status
  * word at the start of ws (at least 256 bytes, 256-byte aligned) and runs one
  * CTA that waits on an mbarrier with the same bounded wait the tensor-core

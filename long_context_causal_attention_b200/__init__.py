@@ -11,7 +11,8 @@ _EXPORTS = (
     "lwm_attn_fwd", "lwm_attn_kernel_launches", "lwm_attn_set_timing_events",
     "lwm_attn_read_status", "lwm_attn_workspace_size", "lwm_rope_apply", "lwm_status_string",
     "make_desc", "lwm_attn_selftest_wait", "lwm_rope_apply_at", "lwm_attn_merge",
-    "lwm_accumulate", "lwm_convert_f32", "lwm_attn_fwd_pair", "lwm_attn_bwd_pair", "lwm_attn_decode", "lwm_attn_decode_workspace_size", "DECODE_MAX_NEW",
+    "lwm_accumulate", "lwm_convert_f32", "lwm_attn_fwd_pair", "lwm_attn_bwd_pair",
+    "lwm_packed_cross_entropy", "lwm_attn_decode", "lwm_attn_decode_workspace_size", "DECODE_MAX_NEW",
 )
 
 __all__ = list(_EXPORTS)

@@ -31,7 +31,8 @@ ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_
                 "lwm_attn_kernel_launches", "lwm_attn_fwd_noalloc",
                 "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait",
                 "lwm_rope_apply_at", "lwm_attn_merge", "lwm_accumulate", "lwm_convert_f32",
-                "lwm_attn_fwd_pair", "lwm_attn_bwd_pair")
+                "lwm_attn_fwd_pair", "lwm_attn_bwd_pair", "lwm_packed_ce_workspace_size",
+                "lwm_packed_cross_entropy")
 DECODE_MAX_NEW = 16
 
 
@@ -88,6 +89,11 @@ def _load():
     lib.lwm_attn_decode.restype = ctypes.c_int
     lib.lwm_attn_selftest_wait.argtypes = [P, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int, P]
     lib.lwm_attn_selftest_wait.restype = ctypes.c_int
+    lib.lwm_packed_ce_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    lib.lwm_packed_ce_workspace_size.restype = ctypes.c_size_t
+    lib.lwm_packed_cross_entropy.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_int32, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.lwm_packed_cross_entropy.restype = ctypes.c_int
     lib.lwm_attn_fwd_pair.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P, P,
                                       ctypes.c_size_t, P]
     lib.lwm_attn_fwd_pair.restype = ctypes.c_int
@@ -405,3 +411,30 @@ def lwm_convert_f32(x, dtype, out=None, stream=None):
     _check(_lib.lwm_convert_f32(x.numel(), _dtype_code(out), x.data_ptr(), out.data_ptr(),
                                 _stream(stream)), "lwm_convert_f32")
     return out
+
+
+def lwm_packed_cross_entropy(logits, targets, segment_ids=None, with_grad=True, stream=None):
+    """(loss [1] float32 on the device, dlogits or None) of a packed batch with
+    per-sample re-weighting; logits [B, S, V], targets / segment_ids int32 [B, S]."""
+    _cuda(logits, "logits")
+    _cuda(targets, "targets")
+    if logits.dim() != 3:
+        raise ValueError("logits must be [B, S, V]")
+    B, S, V = logits.shape
+    if targets.dtype != torch.int32 or tuple(targets.shape) != (B, S):
+        raise ValueError("targets must be int32 [B, S]")
+    seg_ptr = None
+    if segment_ids is not None:
+        _cuda(segment_ids, "segment_ids")
+        if segment_ids.dtype != torch.int32 or tuple(segment_ids.shape) != (B, S):
+            raise ValueError("segment_ids must be int32 [B, S]")
+        seg_ptr = segment_ids.data_ptr()
+    loss = torch.empty(1, dtype=torch.float32, device=logits.device)
+    d = torch.empty_like(logits) if with_grad else None
+    ws = torch.empty(int(_lib.lwm_packed_ce_workspace_size(B, S)), dtype=torch.uint8,
+                     device=logits.device)
+    _check(_lib.lwm_packed_cross_entropy(B, S, V, _dtype_code(logits), logits.data_ptr(),
+                                         targets.data_ptr(), seg_ptr, loss.data_ptr(),
+                                         d.data_ptr() if d is not None else None, ws.data_ptr(),
+                                         ws.numel(), _stream(stream)), "lwm_packed_cross_entropy")
+    return loss, d

@@ -377,6 +377,33 @@ lwm_status lwm_convert_f32(int64_t n, int32_t dtype, const float* x, void* y, vo
   return cuda_status(launch_convert_f32(n, dtype, x, y, static_cast<cudaStream_t>(stream)));
 }
 
+size_t lwm_packed_ce_workspace_size(int64_t batch, int64_t seqlen) {
+  if (batch < 0 || seqlen < 0) return 0;
+  return packed_ce_workspace_bytes(batch, seqlen);
+}
+
+lwm_status lwm_packed_cross_entropy(int64_t batch, int64_t seqlen, int64_t vocab, int32_t dtype,
+                                    const void* logits, const int32_t* targets,
+                                    const int32_t* segment_ids, float* loss, void* dlogits,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  if (batch < 0 || seqlen < 0 || vocab < 1) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32) return LWM_ERR_INVALID_ARG;
+  if (batch > 2147483647 || batch * seqlen > 2147483647) return LWM_ERR_UNSUPPORTED;
+  if (packed_ce_smem_bytes(vocab) > 227 * 1024) return LWM_ERR_UNSUPPORTED;
+  if (!loss) return LWM_ERR_INVALID_ARG;
+  if (batch * seqlen == 0) {
+    return cuda_status(cudaMemsetAsync(loss, 0, sizeof(float), static_cast<cudaStream_t>(stream)));
+  }
+  if (!logits || !targets) return LWM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(targets) & 3u) || (reinterpret_cast<uintptr_t>(segment_ids) & 3u) ||
+      (reinterpret_cast<uintptr_t>(logits) & 15u) || (reinterpret_cast<uintptr_t>(dlogits) & 15u))
+    return LWM_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < packed_ce_workspace_bytes(batch, seqlen)) return LWM_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return LWM_ERR_ALIGNMENT;
+  return cuda_status(launch_packed_ce(batch, seqlen, vocab, dtype, logits, targets, segment_ids,
+                                      loss, dlogits, ws, static_cast<cudaStream_t>(stream)));
+}
+
 lwm_status lwm_attn_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_cycles, int arrive,
                                   void* stream) {
   if (!ws || ws_bytes < sizeof(DeviceStatus) || limit_cycles < 0) return LWM_ERR_INVALID_ARG;

@@ -65,6 +65,11 @@ cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, d
 cudaError_t launch_attn_merge(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, float* o_acc,
                               float* lse_acc, const void* o_part, const float* lse_part,
                               cudaStream_t st);
+size_t packed_ce_workspace_bytes(int64_t B, int64_t S);
+size_t packed_ce_smem_bytes(int64_t V);
+cudaError_t launch_packed_ce(int64_t B, int64_t S, int64_t V, int dtype, const void* logits,
+                             const int32_t* targets, const int32_t* seg, float* loss,
+                             void* dlogits, void* ws, cudaStream_t st);
 cudaError_t launch_accumulate(int64_t n, int dtype, float* acc, const void* x, cudaStream_t st);
 cudaError_t launch_convert_f32(int64_t n, int dtype, const float* x, void* y, cudaStream_t st);
 // ranges = false computes only the per-tile bounds (no q_lo / k_hi).
