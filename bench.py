@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 from workloads import WORKLOADS, segment_ids  # noqa: E402
 
 METRIC = "causal attn fwd+bwd TFLOP/s (32x128 heads, bf16) and % of B200 BF16 peak"
+LOSS_METRIC = "packed re-weighted cross-entropy HBM GB/s (bf16 logits and gradient)"
 DECODE_METRIC = "decode attention HBM GB/s (new tokens against a rotated KV cache, 32x128 heads, bf16)"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 L2_BYTES = 126 * 2 ** 20
@@ -41,8 +42,8 @@ L2_BYTES = 126 * 2 ** 20
 # dram__bytes_write.sum, one-pass ncu capture of the full-size workload, see
 # profiles/attn_bwd_dkdv_traffic_long_128k.md); valid only for the kernel
 # source it was taken on (sha256 of the kernel file and the device headers).
-DKDV_TRAFFIC = {"bytes": {"long_128k": 6.43e9 + 2.13e9},
-                "source_sha256": "dd20546d0968e6e8239479b5e3e266cb7dbf6cb462389eeadb9424348f61cb6a"}
+DKDV_TRAFFIC = {"bytes": {"long_128k": 6.24e9 + 2.12e9},
+                "source_sha256": "14298fda6b5d22f8653b20a0bf54c267ce198a4b7ca2896b370b0c6f28e6e7b8"}
 
 
 def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
@@ -660,6 +661,161 @@ def ours_decode(args):
     return 0
 
 
+def loss_inputs(w, seed, device):
+    """Seeded bf16 logits [B, S, V] ~ N(0, 4) and int32 targets (one in five
+    tokens without loss, as prompt tokens of chat samples)."""
+    import torch
+    V = w.extra["vocab"]
+    rng = np.random.default_rng(seed + 17)
+    targets = rng.integers(0, V, size=(w.batch, w.seqlen)).astype(np.int32)
+    targets[rng.random((w.batch, w.seqlen)) < 0.2] = -1
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    logits = (torch.randn((w.batch, w.seqlen, V), generator=g, device=device) * 2.0)
+    return logits.to(torch.bfloat16), targets
+
+
+def loss_line(w, value, ms, args, ws, extra):
+    line = {"metric": LOSS_METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
+                       "vocab": w.extra["vocab"], "segments": w.segments,
+                       "parallelism": f"independent problem per GPU x{ws}",
+                       "l2": "logits larger than L2 (2.1 GB vs 126 MB), no flush"}}
+    line.update(extra)
+    return line
+
+
+def time_oracle_loss(w, seg, seed, rows=64):
+    """Oracle loss and gradient on the first `rows` tokens of row 0 (their
+    weights from the whole batch's samples)."""
+    import oracle
+    V = w.extra["vocab"]
+    rng = np.random.default_rng(seed + 17)
+    targets = rng.integers(0, V, size=(w.batch, w.seqlen)).astype(np.int32)
+    targets[rng.random((w.batch, w.seqlen)) < 0.2] = -1
+    z = np.random.default_rng(seed).standard_normal((1, rows, V)) * 2.0
+    t0 = time.perf_counter()
+    oracle.packed_cross_entropy(z, targets[:1, :rows], seg[:1, :rows])
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    return dt, 2 * rows * V * 2, threads
+
+
+def reference_loss(args):
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    seg = segment_ids(w, seed=args.seed)
+    for _ in range(args.warmup):
+        time_oracle_loss(w, seg, args.seed)
+    tot, nbytes, threads = 0.0, 0, 1
+    for _ in range(args.steps):
+        dt, nbytes, threads = time_oracle_loss(w, seg, args.seed)
+        tot += dt
+    value = nbytes * args.steps / tot / 1e9
+    sample = f"float64 numpy oracle, loss and gradient of 64 tokens of {w.name}"
+    print(json.dumps(loss_line(w, value, 1e3 * tot / args.steps, args, ws, {
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}})), flush=True)
+    return 0
+
+
+def ours_loss(args):
+    import torch
+    import torch.distributed as dist
+
+    import long_context_causal_attention_b200 as lwm
+
+    ws, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = WORKLOADS[args.workload]
+    seed = rank_seed(args.seed, rank)
+    seg = segment_ids(w, seed=seed)
+    logits, targets = loss_inputs(w, seed, dev)
+    t_d = torch.as_tensor(targets, device=dev)
+    s_d = torch.as_tensor(seg, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    nbytes = 2 * logits.numel() * logits.element_size() + 4 * 2 * t_d.numel()
+    for _ in range(args.warmup):
+        lwm.lwm_packed_cross_entropy(logits, t_d, s_d, stream=stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    launches0 = lwm.lwm_attn_kernel_launches()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        loss, d = lwm.lwm_packed_cross_entropy(logits, t_d, s_d, stream=stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    launches = lwm.lwm_attn_kernel_launches() - launches0
+    clk = clocks.stop()
+    ms, = max_over_ranks([start.elapsed_time(stop) / args.steps], ws, dev)
+    value = nbytes * ws / (ms * 1e-3) / 1e9
+    # end to end: logits in from pinned host memory, loss and gradient out
+    hz = logits.cpu().pin_memory()
+    hd = torch.empty(logits.shape, dtype=logits.dtype, pin_memory=True)
+    hl = torch.empty(1, dtype=torch.float32, pin_memory=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        logits.copy_(hz, non_blocking=True)
+        loss, d = lwm.lwm_packed_cross_entropy(logits, t_d, s_d, stream=stream)
+        hd.copy_(d, non_blocking=True)
+        hl.copy_(loss, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ems, = max_over_ranks([e0.elapsed_time(e1) / args.steps], ws, dev)
+    peaks, src = load_peaks()
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, nb, threads = time_oracle_loss(w, seg, seed)
+        cpu = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"float64 numpy oracle, loss and gradient of 64 tokens of {w.name} "
+                         f"({dt:.2f} s)"}
+    if rank == 0:
+        print(json.dumps(loss_line(w, value, ms, args, ws, {
+            "roofline": {"bound": "hbm", "achieved": value / ws, "peak": float(peaks["hbm_gbs"]),
+                         "unit": "GB/s", "frac": value / ws / float(peaks["hbm_gbs"]),
+                         "traffic": None, "kernel": "run_count + ce + loss_sum kernels",
+                         "algorithmic": "logits read once, gradient written once, targets "
+                                        "and segment ids",
+                         "bytes_per_step": nbytes, "peak_source": f"{src} HBM copy bandwidth"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": nbytes * ws / (ems * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": hz.numel() * hz.element_size(),
+                    "d2h_bytes_per_step": hd.numel() * hd.element_size() + 4},
+            "gpu_launches": launches, "clocks": clk})), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -672,10 +828,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    decode = "n_new" in WORKLOADS[args.workload].extra
+    extra = WORKLOADS[args.workload].extra
     if args.impl == "reference":
-        return reference_decode(args) if decode else reference_arm(args)
-    return ours_decode(args) if decode else ours(args)
+        if "n_new" in extra:
+            return reference_decode(args)
+        return reference_loss(args) if "vocab" in extra else reference_arm(args)
+    if "n_new" in extra:
+        return ours_decode(args)
+    return ours_loss(args) if "vocab" in extra else ours(args)
 
 
 if __name__ == "__main__":

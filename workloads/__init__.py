@@ -17,6 +17,8 @@ into one sequence)):
   million_1m        B1 H32 D128 bf16, S=1048576, one segment, theta 5e7, fwd+bwd
   decode_1m         B1 H32 D128 bf16, one new token against a 1048576-token
                     cache (the new token's own key and value included), theta 5e7
+  packed_loss_8k    packed_8k's rows, bf16 logits over a 32000-token vocabulary,
+                    re-weighted cross-entropy and its gradient
 """
 
 from __future__ import annotations
@@ -61,6 +63,10 @@ WORKLOADS = {
     # decode step: n_new new tokens, the cache of `seqlen` tokens includes them
     "decode_1m": Workload("decode_1m", 1, 1048576, 32, 128, "bf16", 5e7, backward=False,
                           extra={"n_new": 1}),
+    # packed loss re-weighting: the packed_8k rows, LLaMA vocabulary (32000)
+    "packed_loss_8k": Workload("packed_loss_8k", 4, 8192, 32, 128, "bf16", 1e6,
+                               segments="packed_video_text", backward=False,
+                               extra={"vocab": 32000}),
     # decode profiling case: 128K-token cache (2 GiB of keys and values, above L2)
     "prof_decode_128k": Workload("prof_decode_128k", 1, 131072, 32, 128, "bf16", 1e7,
                                  backward=False, extra={"n_new": 1}),
