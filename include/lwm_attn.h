@@ -262,9 +262,10 @@ lwm_status lwm_convert_f32(int64_t n, int32_t dtype, const float* x, void* y, vo
  *   summed in a fixed order.  dlogits [B, S, V] of dtype (may be NULL):
  *   w_t * (softmax(z_t) - onehot(y_t)), zero rows for tokens without loss.
  *   ws: lwm_packed_ce_workspace_size(B, S) bytes, 256-byte aligned.
- *   V up to 58,112 (a row of fp32 logits in shared memory); larger returns
- *   LWM_ERR_UNSUPPORTED.  Reads the logits once and writes dlogits once:
- *   bound by HBM bandwidth. */
+ *   V up to 32,768 for bf16 and 16,384 for fp32 (a row held in registers),
+ *   and a multiple of 8 (bf16) or 4 (fp32) so rows are whole 16-byte
+ *   vectors; otherwise LWM_ERR_UNSUPPORTED.  Reads the logits once and
+ *   writes dlogits once: bound by HBM bandwidth. */
 size_t lwm_packed_ce_workspace_size(int64_t batch, int64_t seqlen);
 lwm_status lwm_packed_cross_entropy(int64_t batch, int64_t seqlen, int64_t vocab, int32_t dtype,
                                     const void* logits, const int32_t* targets,

@@ -389,7 +389,8 @@ lwm_status lwm_packed_cross_entropy(int64_t batch, int64_t seqlen, int64_t vocab
   if (batch < 0 || seqlen < 0 || vocab < 1) return LWM_ERR_INVALID_ARG;
   if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32) return LWM_ERR_INVALID_ARG;
   if (batch > 2147483647 || batch * seqlen > 2147483647) return LWM_ERR_UNSUPPORTED;
-  if (packed_ce_smem_bytes(vocab) > 227 * 1024) return LWM_ERR_UNSUPPORTED;
+  if (vocab > packed_ce_max_vocab(dtype)) return LWM_ERR_UNSUPPORTED;
+  if (vocab % (dtype == LWM_DTYPE_BF16 ? 8 : 4) != 0) return LWM_ERR_UNSUPPORTED;  // 16-byte rows
   if (!loss) return LWM_ERR_INVALID_ARG;
   if (batch * seqlen == 0) {
     return cuda_status(cudaMemsetAsync(loss, 0, sizeof(float), static_cast<cudaStream_t>(stream)));

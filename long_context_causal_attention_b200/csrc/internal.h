@@ -66,7 +66,7 @@ cudaError_t launch_attn_merge(int64_t B, int64_t S, int64_t H, int64_t D, int dt
                               float* lse_acc, const void* o_part, const float* lse_part,
                               cudaStream_t st);
 size_t packed_ce_workspace_bytes(int64_t B, int64_t S);
-size_t packed_ce_smem_bytes(int64_t V);
+int64_t packed_ce_max_vocab(int dtype);
 cudaError_t launch_packed_ce(int64_t B, int64_t S, int64_t V, int dtype, const void* logits,
                              const int32_t* targets, const int32_t* seg, float* loss,
                              void* dlogits, void* ws, cudaStream_t st);

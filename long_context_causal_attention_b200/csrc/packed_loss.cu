@@ -14,8 +14,8 @@
 //                      each token belongs to (a chunk per thread, run
 //                      totals stitched across chunk edges by two scans over
 //                      the chunk summaries), and the number of samples.
-//   ce_kernel          one CTA per token: the row of logits into shared
-//                      memory (read once from HBM), log-sum-exp, the
+//   ce_kernel          one CTA per token: the row of logits into registers
+//                      (16-byte loads, read once from HBM), log-sum-exp, the
 //                      weighted loss term and w * (softmax - onehot) (written
 //                      once).  HBM-bound: 2 * V * elt bytes per token.
 //   loss_sum_kernel    the weighted terms summed in a fixed order.
@@ -26,7 +26,8 @@ namespace lwm {
 namespace {
 
 constexpr int kRunThreads = 1024;
-constexpr int kCeThreads = 256;
+constexpr int kCeThreads = 512;
+constexpr int kCeVecs = 8;  // 16-byte vectors per thread: V <= 32768 (bf16), 16384 (fp32)
 
 struct ChunkSummary {
   int32_t first_id, last_id;
@@ -120,57 +121,111 @@ run_count_kernel(const int32_t* __restrict__ seg, const int32_t* __restrict__ ta
   if (tid == 0 && block_samples) atomicAdd(n_samples, block_samples);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kCeThreads)
+// Block-wide max / sum of one value per thread (kCeThreads threads).
+__device__ __forceinline__ float block_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int i = 1; i < kCeThreads / 32; ++i) v = fmaxf(v, red[i]);
+  return v;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = 0.f;
+#pragma unroll
+  for (int i = 0; i < kCeThreads / 32; ++i) v += red[i];
+  return v;
+}
+
+// One CTA per token; the row of logits is read once with 16-byte loads into
+// registers (NV vectors per thread cover V <= kCeThreads * NV * E, E elements
+// per vector), so the log-sum-exp and the gradient need no second read.
+template <typename T, int NV>
+__global__ void __launch_bounds__(kCeThreads, 2)
 ce_kernel(const T* __restrict__ logits, const int32_t* __restrict__ targets,
           const int32_t* __restrict__ run_n, const int32_t* __restrict__ n_samples, int64_t V,
           float* __restrict__ term, T* __restrict__ dlogits) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  float* z = reinterpret_cast<float*>(smem_raw);
+  constexpr int E = 16 / sizeof(T);
   __shared__ float red[kCeThreads / 32];
+  __shared__ float zy;
   const int64_t tok = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int32_t y = targets[tok];
   const int32_t n = run_n[tok];
   const int32_t ns = *n_samples;
   // a target outside the vocabulary counts as "no loss" (never read out of range)
   const float w = (y >= 0 && y < V && n > 0 && ns > 0) ? 1.f / ((float)n * (float)ns) : 0.f;
+  const int64_t nvec = V / E;  // V is a multiple of E (checked by the caller)
   if (w == 0.f) {  // no loss here: zero gradient row
-    if (dlogits)
-      for (int64_t i = tid; i < V; i += kCeThreads) dlogits[tok * V + i] = from_f32<T>(0.f);
+    if (dlogits) {
+      uint4* out = reinterpret_cast<uint4*>(dlogits + tok * V);
+      for (int64_t i = tid; i < nvec; i += kCeThreads) out[i] = make_uint4(0, 0, 0, 0);
+    }
     if (tid == 0) term[tok] = 0.f;
     return;
   }
-  const T* row = logits + tok * V;
-  float mx = -INFINITY;
-  for (int64_t i = tid; i < V; i += kCeThreads) {
-    const float v = to_f32(row[i]);
-    z[i] = v;
-    mx = fmaxf(mx, v);
+  const uint4* row = reinterpret_cast<const uint4*>(logits + tok * V);
+  uint4 raw[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int64_t i = tid + (int64_t)k * kCeThreads;
+    raw[k] = i < nvec ? __ldg(row + i) : make_uint4(0, 0, 0, 0);
   }
+  float mx = -INFINITY;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  mx = red[0];
+  for (int k = 0; k < NV; ++k) {
+    const int64_t i = tid + (int64_t)k * kCeThreads;
+    if (i < nvec) {
+      const T* e = reinterpret_cast<const T*>(&raw[k]);
 #pragma unroll
-  for (int i = 1; i < kCeThreads / 32; ++i) mx = fmaxf(mx, red[i]);
-  __syncthreads();
+      for (int u = 0; u < E; ++u) mx = fmaxf(mx, to_f32(e[u]));
+    }
+  }
+  mx = block_max(mx, red);
   float sum = 0.f;
-  for (int64_t i = tid; i < V; i += kCeThreads) sum += expf(z[i] - mx);
 #pragma unroll
-  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) red[warp] = sum;
-  __syncthreads();
-  sum = 0.f;
+  for (int k = 0; k < NV; ++k) {
+    const int64_t i = tid + (int64_t)k * kCeThreads;
+    if (i < nvec) {
+      const T* e = reinterpret_cast<const T*>(&raw[k]);
 #pragma unroll
-  for (int i = 0; i < kCeThreads / 32; ++i) sum += red[i];
-  const float lse = mx + logf(sum);
-  if (tid == 0) term[tok] = w * (lse - z[y]);
+      for (int u = 0; u < E; ++u) {
+        const float v = to_f32(e[u]);
+        sum += __expf(v - mx);
+        if (i * E + u == y) zy = v;
+      }
+    }
+  }
+  sum = block_sum(sum, red);  // its barriers also publish zy
+  const float lse = mx + __logf(sum);
+  if (tid == 0) term[tok] = w * (lse - zy);
   if (dlogits) {
-    for (int64_t i = tid; i < V; i += kCeThreads) {
-      const float g = expf(z[i] - lse) - (i == y ? 1.f : 0.f);
-      dlogits[tok * V + i] = from_f32<T>(w * g);
+    uint4* out = reinterpret_cast<uint4*>(dlogits + tok * V);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int64_t i = tid + (int64_t)k * kCeThreads;
+      if (i < nvec) {
+        const T* e = reinterpret_cast<const T*>(&raw[k]);
+        uint4 o;
+        T* f = reinterpret_cast<T*>(&o);
+#pragma unroll
+        for (int u = 0; u < E; ++u) {
+          const int64_t c = i * E + u;
+          f[u] = from_f32<T>(w * (__expf(to_f32(e[u]) - lse) - (c == y ? 1.f : 0.f)));
+        }
+        out[i] = o;
+      }
     }
   }
 }
@@ -196,7 +251,9 @@ size_t packed_ce_workspace_bytes(int64_t B, int64_t S) {
   return 256 + ((n * 4 + 255) / 256) * 256 * 2;  // sample counter, run_n, terms
 }
 
-size_t packed_ce_smem_bytes(int64_t V) { return (size_t)V * sizeof(float); }
+int64_t packed_ce_max_vocab(int dtype) {
+  return (int64_t)kCeThreads * kCeVecs * (dtype == LWM_DTYPE_BF16 ? 8 : 4);
+}
 
 cudaError_t launch_packed_ce(int64_t B, int64_t S, int64_t V, int dtype, const void* logits,
                              const int32_t* targets, const int32_t* seg, float* loss,
@@ -209,26 +266,14 @@ cudaError_t launch_packed_ce(int64_t B, int64_t S, int64_t V, int dtype, const v
   cudaError_t e = cudaMemsetAsync(n_samples, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   run_count_kernel<<<(unsigned)B, kRunThreads, 0, st>>>(seg, targets, S, run_n, n_samples);
-  const size_t smem = packed_ce_smem_bytes(V);
-  if (dtype == LWM_DTYPE_BF16) {
-    if (smem > 48 * 1024) {
-      e = cudaFuncSetAttribute(ce_kernel<__nv_bfloat16>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    ce_kernel<__nv_bfloat16><<<(unsigned)n, kCeThreads, smem, st>>>(
+  if (dtype == LWM_DTYPE_BF16)
+    ce_kernel<__nv_bfloat16, kCeVecs><<<(unsigned)n, kCeThreads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(logits), targets, run_n, n_samples, V, term,
         static_cast<__nv_bfloat16*>(dlogits));
-  } else {
-    if (smem > 48 * 1024) {
-      e = cudaFuncSetAttribute(ce_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    ce_kernel<float><<<(unsigned)n, kCeThreads, smem, st>>>(
+  else
+    ce_kernel<float, kCeVecs><<<(unsigned)n, kCeThreads, 0, st>>>(
         static_cast<const float*>(logits), targets, run_n, n_samples, V, term,
         static_cast<float*>(dlogits));
-  }
   loss_sum_kernel<<<1, 1024, 0, st>>>(term, (int64_t)n, loss);
   note_launches(3);
   return cudaGetLastError();

@@ -156,6 +156,21 @@ def test_pair_entry_points_need_both_or_neither_segment_arrays(lwm):
     assert bwd(_desc(lwm, head_dim=32, segment_ids=P), P) == -2
 
 
+def test_packed_cross_entropy_argument_errors(lwm):
+    lib = lwm._lib.lib()
+    P = 0x10000
+    ws = lwm._lib.lib().lwm_packed_ce_workspace_size(2, 100)
+    assert ws >= 2 * 100 * 8
+    ce = lambda V, dt=0, logits=P, ws_b=1 << 30: lib.lwm_packed_cross_entropy(
+        2, 100, V, dt, logits, P, None, P, P, P, ws_b, None)
+    assert ce(40000) == -2            # row does not fit the registers of one CTA
+    assert ce(20000, dt=1) == -2
+    assert ce(1001) == -2             # bf16 rows must be whole 16-byte vectors
+    assert ce(1000, dt=5) == -1
+    assert ce(1000, logits=P + 8) == -3
+    assert ce(1000, ws_b=16) == -4
+
+
 def test_python_binding_requires_cuda_tensors(lwm):
     import torch
     q = torch.zeros(1, 4, 1, 64)
