@@ -43,7 +43,7 @@ L2_BYTES = 126 * 2 ** 20
 # profiles/attn_bwd_dkdv_traffic_long_128k.md); valid only for the kernel
 # source it was taken on (sha256 of the kernel file and the device headers).
 DKDV_TRAFFIC = {"bytes": {"long_128k": 6.24e9 + 2.12e9},
-                "source_sha256": "14298fda6b5d22f8653b20a0bf54c267ce198a4b7ca2896b370b0c6f28e6e7b8"}
+                "source_sha256": "88f50d7a60fb86e4bcb66285ffc1fdbb9b8dc0be947c6e46ceac951a3c116497"}
 
 
 def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:

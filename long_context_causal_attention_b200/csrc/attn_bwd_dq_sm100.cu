@@ -12,7 +12,8 @@
 // no partial sums leave the CTA.  Q~_i and dO_i are the A operands of S and
 // dP for the whole sweep, so they sit in tensor memory and every product of
 // the sweep reads only its B operand (K~_j or V_j) from shared memory.
-// Roles (576 threads, so that each may hold 112 registers):
+// Roles (576 threads; fewer control warps leave more registers to the
+// element-wise ones):
 //   warp 0      TMA producer: K~_j and V_j per step, 3-stage rings, K issued
 //               two tiles ahead of V.
 //   warp 1      MMA issuer (one thread); the whole warp allocates and frees

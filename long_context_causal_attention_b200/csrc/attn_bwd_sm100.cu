@@ -13,8 +13,8 @@
 //
 // One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
 // walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
-// tensor memory for the whole walk.  Roles (576 threads, so that each may
-// hold 112 registers):
+// tensor memory for the whole walk.  Roles (576 threads; fewer control
+// warps leave more registers to the element-wise ones):
 //   warp 0      TMA producer: K~_j, V_j once per item; Q~_i, dO_i, and the
 //               tile's LSE*log2(e) and D (1-D bulk copies) per step, through a
 //               2-stage ring.

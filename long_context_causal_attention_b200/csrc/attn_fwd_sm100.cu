@@ -23,9 +23,11 @@
 // The MMA issue order ping-pongs the two tiles so one softmax warpgroup
 // works while the tensor core runs the other tile's MMAs:
 //   S_0(j) S_1(j) | PV_0(j) S_0(j+1) | PV_1(j) S_1(j+1) | ...
-// Work items (b, h, pair of 128-row query tiles) go to CTAs round-robin in
-// head-major order with the costliest pair of each head first, so CTAs that
-// run at the same time share one head's K/V through L2.
+// Work items (b, h, pair of 128-row query tiles), in head-major order with
+// the costliest pair of each head first, come from a global counter: the
+// TMA thread takes the next one when it is ready for it and publishes it to
+// the CTA through a 4-slot ring, so the CTAs stay on consecutive items of one
+// head and share its K/V through L2.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
