@@ -17,6 +17,7 @@ into one sequence)):
   million_1m        B1 H32 D128 bf16, S=1048576, one segment, theta 5e7, fwd+bwd
   decode_1m         B1 H32 D128 bf16, one new token against a 1048576-token
                     cache (the new token's own key and value included), theta 5e7
+  fp32_8k           B1 H32 D128 fp32, S=8192, one segment, theta 1e6, fwd+bwd
   packed_loss_8k    packed_8k's rows, bf16 logits over a 32000-token vocabulary,
                     re-weighted cross-entropy and its gradient
 """
@@ -63,6 +64,8 @@ WORKLOADS = {
     # decode step: n_new new tokens, the cache of `seqlen` tokens includes them
     "decode_1m": Workload("decode_1m", 1, 1048576, 32, 128, "bf16", 5e7, backward=False,
                           extra={"n_new": 1}),
+    # fp32 end to end (the pages train in fp32): the CUDA-core path at 8K tokens
+    "fp32_8k": Workload("fp32_8k", 1, 8192, 32, 128, "fp32", 1e6),
     # packed loss re-weighting: the packed_8k rows, LLaMA vocabulary (32000)
     "packed_loss_8k": Workload("packed_loss_8k", 4, 8192, 32, 128, "bf16", 1e6,
                                segments="packed_video_text", backward=False,
