@@ -392,14 +392,24 @@ def ours(args):
         traffic = DKDV_TRAFFIC["bytes"][w.name]
     bwd_flops = 2.5 * fwd_flops
     dq_k = bwd_k - dkdv_k
-    if achieved is None:  # the CUDA-core backward (fp32, head_dim 64) is one launch
-        dq_k, dkdv_k = None, None
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak if achieved else None, "traffic": traffic,
-                "kernel": "attn_bwd_dkdv_kernel",
+    kernel, bound, rpeak, peak_note = "attn_bwd_dkdv_kernel", "tensor", peak, \
+        f"{peak_src} bf16 sustained (kernel timed inside a long step)"
+    if w.dtype != "bf16" or w.head_dim != 128:
+        # the CUDA-core kernels (fp32 arithmetic): bound by the FFMA pipes,
+        # 128 fp32 lanes per SM, one fused multiply-add (2 flops) per lane
+        # per clock, at the maximum SM clock the device reports
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        sm_max = float((clk or {}).get("sm_max_mhz") or 1965.0)
+        rpeak = sms * 128 * 2 * sm_max * 1e6 / 1e12
+        kernel, bound, traffic = "simt_bwd_dkdv_kernel", "alu", None
+        peak_note = (f"fp32 FFMA peak derived: {sms} SMs x 128 lanes x 2 flops x "
+                     f"{sm_max:.0f} MHz (maximum SM clock)")
+    roofline = {"bound": bound, "achieved": achieved, "peak": rpeak, "unit": "TFLOP/s",
+                "frac": achieved / rpeak if achieved else None, "traffic": traffic,
+                "kernel": kernel,
                 "algorithmic": "8*D*H flops per kept (query, key) pair: S^T, dP^T, dV, dK",
                 "tile_pairs": units,
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "peak_source": peak_note,
                 "dkdv_kernel_ms": dkdv_k, "dq_kernel_ms": dq_k, "fwd_kernel_ms": fwd_k,
                 "fwd_kernel_tflops": fwd_flops / (fwd_k * 1e-3) / 1e12,
                 "bwd_kernels_tflops": bwd_flops / (bwd_k * 1e-3) / 1e12,

@@ -243,7 +243,9 @@ lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   e = launch_delta(p, o, d_o, w.delta, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   record_event(2, st);
-  e = launch_simt_bwd(p, w, v, lse, d_o, dq, dk, dv, st);
+  e = launch_simt_bwd_dkdv(p, w, v, lse, d_o, dk, dv, st);
+  record_event(4, st);
+  if (e == cudaSuccess) e = launch_simt_bwd_dq(p, w, v, lse, d_o, dq, st);
   record_event(3, st);
   return cuda_status(e);
 }

@@ -101,8 +101,10 @@ cudaError_t launch_selftest_wait(DeviceStatus* status, long long limit_cycles, i
                                  cudaStream_t st);
 cudaError_t launch_simt_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                             float* lse, cudaStream_t st);
-cudaError_t launch_simt_bwd(const Problem& p, const Workspace& ws, const void* v,
-                            const float* lse, const void* d_o, void* dq, void* dk, void* dv,
-                            cudaStream_t st);
+cudaError_t launch_simt_bwd_dkdv(const Problem& p, const Workspace& ws, const void* v,
+                                 const float* lse, const void* d_o, void* dk, void* dv,
+                                 cudaStream_t st);
+cudaError_t launch_simt_bwd_dq(const Problem& p, const Workspace& ws, const void* v,
+                               const float* lse, const void* d_o, void* dq, cudaStream_t st);
 
 }  // namespace lwm

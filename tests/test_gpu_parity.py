@@ -63,6 +63,10 @@ SMALL = [
     ("d64_bf16", 2, 257, 2, 64, "bf16", 1e6, True, 1.0, "random"),
     ("fp32_d128", 1, 200, 2, 128, "fp32", 1e4, True, 1.0, "random"),
     ("fp32_noncausal_d64", 1, 190, 2, 64, "fp32", 1e6, False, 1.0, "random_pad"),
+    ("fp32_packed700_pad", 2, 700, 2, 128, "fp32", 1e6, True, 1.0, "random_pad"),
+    ("fp32_d64_theta5e7", 1, 333, 2, 64, "fp32", 5e7, True, 1.0, "single"),
+    ("fp32_long_segments_600", 1, 600, 2, 128, "fp32", 1e4, True, 1.0, "random_long"),
+    ("d64_bf16_noncausal_pad", 1, 450, 2, 64, "bf16", 1e4, False, 1.0, "random_pad"),
     ("no_rope", 1, 384, 2, 128, "bf16", 0.0, True, 1.0, "single"),
     ("long_segments_1000", 1, 1000, 2, 128, "bf16", 1e6, True, 1.0, "random_long"),
 ]
@@ -99,6 +103,22 @@ def test_tiny_packed_fp32_workload(lwm):
     ref = full_oracle(t, seg, w, backward=True)
     for key in ("o", "lse", "dq", "dk", "dv"):
         assert_close(key, to64(got[key]), ref[key], "fp32")
+
+
+def test_fp32_8k_workload_sampled(lwm):
+    """B1 H32 D128 fp32, S=8192, one segment, theta 1e6, fwd+bwd (the CUDA-core
+    path at scale): 64 random query rows and the last 256 rows of two heads
+    against the oracle at the fp32 bound."""
+    w = WORKLOADS["fp32_8k"]
+    seg = segment_ids(w)
+    t = make_tensors(w, seed=0, device="cuda")
+    got = run(lwm, t, seg, w, backward=True)
+    rng = np.random.default_rng(4)
+    samples = _sampled_rows(rng, w.batch, w.seqlen, w.heads, 64)
+    samples += [(0, 3, w.seqlen - 1), (0, 30, 0), (0, 7, 63), (0, 7, 64)]
+    check_rows(t, got, seg, w, samples, backward=True)
+    for b, h in ((0, 0), (0, 21)):
+        check_tail(t, got, seg, w, b, h, rows=256)
 
 
 def _sampled_rows(rng, B, S, H, n):
