@@ -261,7 +261,9 @@ lwm_status lwm_convert_f32(int64_t n, int32_t dtype, const float* x, void* y, vo
  *   loss: device float, sum over tokens of w_t * (logsumexp(z_t) - z_t[y_t]),
  *   summed in a fixed order.  dlogits [B, S, V] of dtype (may be NULL):
  *   w_t * (softmax(z_t) - onehot(y_t)), zero rows for tokens without loss.
- *   ws: lwm_packed_ce_workspace_size(B, S) bytes, 256-byte aligned.
+ *   ws: lwm_packed_ce_workspace_size(B, S) bytes, 256-byte aligned; it
+ *   starts with the status word, which lwm_attn_read_status(ws) reads after
+ *   the call (LWM_ERR_TIMEOUT if a bounded wait inside the kernel ran out).
  *   V up to 32,768 for bf16 and 16,384 for fp32 (a row held in registers),
  *   and a multiple of 8 (bf16) or 4 (fp32) so rows are whole 16-byte
  *   vectors; otherwise LWM_ERR_UNSUPPORTED.  Reads the logits once and

@@ -413,9 +413,11 @@ def lwm_convert_f32(x, dtype, out=None, stream=None):
     return out
 
 
-def lwm_packed_cross_entropy(logits, targets, segment_ids=None, with_grad=True, stream=None):
+def lwm_packed_cross_entropy(logits, targets, segment_ids=None, with_grad=True, stream=None,
+                             check_status=False):
     """(loss [1] float32 on the device, dlogits or None) of a packed batch with
-    per-sample re-weighting; logits [B, S, V], targets / segment_ids int32 [B, S]."""
+    per-sample re-weighting; logits [B, S, V], targets / segment_ids int32 [B, S].
+    check_status=True reads the kernel's status word after the call (a sync)."""
     _cuda(logits, "logits")
     _cuda(targets, "targets")
     if logits.dim() != 3:
@@ -437,4 +439,6 @@ def lwm_packed_cross_entropy(logits, targets, segment_ids=None, with_grad=True, 
                                          targets.data_ptr(), seg_ptr, loss.data_ptr(),
                                          d.data_ptr() if d is not None else None, ws.data_ptr(),
                                          ws.numel(), _stream(stream)), "lwm_packed_cross_entropy")
+    if check_status:
+        _check(lwm_attn_read_status(ws, stream), "lwm_packed_cross_entropy (device status)")
     return loss, d

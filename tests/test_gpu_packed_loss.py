@@ -17,18 +17,18 @@ from workloads import random_segments
 pytestmark = pytest.mark.gpu
 
 
-def run_case(B, S, V, dtype, packed, seed):
+def run_case(B, S, V, dtype, packed, seed, no_loss_frac=0.2):
     import long_context_causal_attention_b200 as lwm
     rng = np.random.default_rng(seed)
     seg = random_segments(rng, B, S, 5, max(6, S // 4), pad_tail=3) if packed else None
     targets = rng.integers(0, V, size=(B, S)).astype(np.int32)
-    targets[rng.random((B, S)) < 0.2] = -1       # tokens without loss (prompts)
+    targets[rng.random((B, S)) < no_loss_frac] = -1   # tokens without loss (prompts)
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
     logits = (torch.randn((B, S, V), generator=g, device="cuda") * 2.0).to(dtype)
     t_d = torch.as_tensor(targets, device="cuda")
     s_d = torch.as_tensor(seg, dtype=torch.int32, device="cuda") if packed else None
-    loss, d = lwm.lwm_packed_cross_entropy(logits, t_d, s_d)
+    loss, d = lwm.lwm_packed_cross_entropy(logits, t_d, s_d, check_status=True)
     torch.cuda.synchronize()
     z = logits.double().cpu().numpy()
     ref_loss, ref_d = oracle.packed_cross_entropy(z, targets,
@@ -46,6 +46,16 @@ def run_case(B, S, V, dtype, packed, seed):
     (2, 513, 776, torch.bfloat16, False),
     (1, 5000, 2048, torch.bfloat16, True),
     (1, 2048, 32000, torch.bfloat16, True),
+    (1, 600, 32768, torch.bfloat16, True),    # largest bf16 row: 64 KB, three ring stages
+    (1, 400, 16384, torch.float32, True),     # largest fp32 row
+    (2, 3000, 8, torch.bfloat16, True),       # 16-byte rows: sixteen stages, many rows per CTA
+    (1, 5, 64, torch.float32, False),         # fewer rows than SMs
 ])
 def test_packed_cross_entropy(B, S, V, dtype, packed):
     run_case(B, S, V, dtype, packed, seed=B * 1000 + S)
+
+
+def test_packed_cross_entropy_no_loss_rows():
+    """Long stretches of rows without a loss pass through the row ring with
+    no data: most rows here carry none."""
+    run_case(2, 1500, 1024, torch.bfloat16, True, seed=77, no_loss_frac=0.9)
