@@ -302,6 +302,36 @@ def test_gradient_sums_per_segment():
             assert np.allclose(dkt[b, m].sum(0), 0.0, atol=1e-11)
 
 
+def test_key_shift_without_rotation_moves_only_lse():
+    """theta disabled: adding one vector c to every key adds scale q_i.c to
+    every score of row i, a per-row constant the softmax removes.  O, dQ, dK
+    and dV stay (dQ because each row of dS sums to zero) and LSE moves by
+    exactly scale q_i.c."""
+    q, k, v, do, seg = _case(seed=21, pad_tail=3)
+    c = np.random.default_rng(22).standard_normal(q.shape[-1])
+    scale = 1.0 / math.sqrt(q.shape[-1])
+    r0 = A.attention_backward(q, k, v, do, seg, theta=0.0)
+    r1 = A.attention_backward(q, k + c, v, do, seg, theta=0.0)
+    for key in ("o", "dq", "dk", "dv"):
+        assert _close(r1[key], r0[key], 1e-9), key
+    shift = scale * np.einsum("bshd,d->bhs", q, c)
+    assert _close(r1["lse"], r0["lse"] + shift, 1e-9)
+
+
+def test_value_shift_moves_output_by_the_same_vector():
+    """Adding c to every value adds c to every output row that attends to
+    anything (softmax rows sum to one) and leaves all three gradients: dP
+    moves by a per-row constant that D_i absorbs."""
+    q, k, v, do, seg = _case(seed=23, pad_tail=2)
+    c = np.random.default_rng(24).standard_normal(q.shape[-1])
+    r0 = A.attention_backward(q, k, v, do, seg, theta=1e6)
+    r1 = A.attention_backward(q, k, v + c, do, seg, theta=1e6)
+    live = (seg >= 0)[:, :, None, None]
+    assert _close(r1["o"], r0["o"] + np.where(live, c, 0.0), 1e-9)
+    for key in ("lse", "dq", "dk", "dv"):
+        assert _close(r1[key], r0[key], 1e-9), key
+
+
 def test_rows_and_tail_agree_with_full():
     q, k, v, do, seg = _case(seed=13, B=2, S=64)
     full = A.attention_backward(q, k, v, do, seg, theta=1e7)
