@@ -91,7 +91,8 @@ typedef struct {
 /* Bytes of device workspace lwm_attn_fwd (is_bwd = 0) or lwm_attn_bwd
  * (is_bwd != 0) needs for `desc`; 0 if `desc` is invalid.  The workspace
  * holds the status word, per-tile segment bounds, the rotated Q and K and,
- * for the backward, the fp32 dQ accumulator and the per-row dot(dO, O).
+ * for the backward, the per-row LSE and dot(dO, O) (fp32, padded to whole
+ * tiles for the tensor-core kernels).
  * The forward's need is never larger than the backward's. */
 size_t lwm_attn_workspace_size(const lwm_attn_desc* desc, int is_bwd);
 
@@ -197,8 +198,8 @@ const char* lwm_status_string(lwm_status status);
  * NULL) that the next calls record on their stream immediately before and
  * after the main attention kernel(s) of lwm_attn_fwd / lwm_attn_bwd, so the
  * caller can time those kernels alone; bwd_split is recorded between the
- * dK/dV kernel and the dQ kernel of the tensor-core backward (not by the
- * fp32 / head_dim 64 backward).  The handles stay in effect until
+ * dK/dV kernel and the dQ kernel of the backward (both kernel families run
+ * dK/dV first).  The handles stay in effect until
  * replaced; pass NULLs to stop.  Process-wide; guarded by a mutex.
  * lwm_attn_kernel_launches: number of kernels this library has launched
  * since it was loaded. */
