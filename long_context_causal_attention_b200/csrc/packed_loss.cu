@@ -34,7 +34,7 @@
 namespace lwm {
 namespace {
 
-constexpr int kRunThreads = 1024;
+constexpr int kRunThreads = 256;  // chunks per row: short serial stitching scans
 constexpr int kCeConsumerWarps = 16;
 constexpr int kCeConsumers = kCeConsumerWarps * 32;  // threads that hold a row
 constexpr int kCeThreads = kCeConsumers + 32;        // plus the producer warp
@@ -67,13 +67,27 @@ run_count_kernel(const int32_t* __restrict__ seg, const int32_t* __restrict__ ta
   if (tid == 0) block_samples = 0;
   ChunkSummary c{};
   if (t0 < t1) {
+    // one forward pass whose loads do not wait on the previous token: the
+    // first run's loss tokens, whether the chunk is one run, the last run's
+    int32_t cur_id = id_of(t0), cur_cnt = 0;
+    bool in_first = true;
+#pragma unroll 8
+    for (int64_t t = t0; t < t1; ++t) {
+      const int32_t id = id_of(t);
+      const int32_t lt = loss_tok(t);
+      if (id != cur_id) {
+        if (in_first) c.cnt_first = cur_cnt;
+        in_first = false;
+        cur_id = id;
+        cur_cnt = 0;
+      }
+      cur_cnt += lt;
+    }
+    if (in_first) c.cnt_first = cur_cnt;
     c.first_id = id_of(t0);
-    c.last_id = id_of(t1 - 1);
-    int64_t t = t0;
-    while (t < t1 && id_of(t) == c.first_id) c.cnt_first += loss_tok(t++);
-    c.single = t == t1;
-    t = t1 - 1;
-    while (t >= t0 && id_of(t) == c.last_id) c.cnt_last += loss_tok(t--);
+    c.last_id = cur_id;
+    c.single = in_first;
+    c.cnt_last = cur_cnt;
   } else {
     c.first_id = c.last_id = INT_MIN;  // empty chunk: joins nothing
     c.single = 0;

@@ -2,7 +2,7 @@
 
 Rows of packed samples (random segment lengths, padding at the end, tokens
 without loss), with and without segment ids, bf16 and fp32 logits.  Row
-lengths below and above the 1024 chunks of the run-counting kernel make
+lengths below and above the 256 chunks of the run-counting kernel make
 samples cross chunk edges (the stitching of run totals).  The loss must
 match to 1e-4 relative; the gradient within 2e-2 (bf16) or 1e-4 (fp32) of
 its largest magnitude, since its values scale with the per-token weights.
