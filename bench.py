@@ -685,6 +685,15 @@ def loss_inputs(w, seed, device):
     return logits.to(torch.bfloat16), targets
 
 
+def loss_bytes(V, elt, targets, seg):
+    """Algorithmic bytes of one packed-loss step: the logits of the tokens
+    that carry a loss are read once (the kernel never reads the others), the
+    gradient of every token is written once (zero rows included), targets
+    and segment ids are read once."""
+    has_loss = (targets >= 0) & (targets < V) & (np.asarray(seg) >= 0)
+    return V * elt * (int(has_loss.sum()) + targets.size) + 4 * 2 * targets.size
+
+
 def loss_line(w, value, ms, args, ws, extra):
     line = {"metric": LOSS_METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -762,7 +771,7 @@ def ours_loss(args):
     t_d = torch.as_tensor(targets, device=dev)
     s_d = torch.as_tensor(seg, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
-    nbytes = 2 * logits.numel() * logits.element_size() + 4 * 2 * t_d.numel()
+    nbytes = loss_bytes(logits.shape[-1], logits.element_size(), targets, seg)
     for _ in range(args.warmup):
         lwm.lwm_packed_cross_entropy(logits, t_d, s_d, stream=stream)
     torch.cuda.synchronize()
@@ -813,8 +822,9 @@ def ours_loss(args):
             "roofline": {"bound": "hbm", "achieved": value / ws, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": value / ws / float(peaks["hbm_gbs"]),
                          "traffic": None, "kernel": "run_count + ce + loss_sum kernels",
-                         "algorithmic": "logits read once, gradient written once, targets "
-                                        "and segment ids",
+                         "algorithmic": "logits of the tokens with a loss read once, the "
+                                        "gradient of every token written once, targets and "
+                                        "segment ids",
                          "bytes_per_step": nbytes, "peak_source": f"{src} HBM copy bandwidth"},
             "cpu_baseline": cpu,
             "e2e": {"value": nbytes * ws / (ems * 1e-3) / 1e9, "unit": "GB/s",

@@ -8,7 +8,7 @@
 // then over the samples, so a loss token of a sample with n loss tokens
 // weighs 1 / (n * number of samples with a loss token).  A sample is a
 // contiguous run of one segment id (what packing produces); ids < 0 are
-// padding, targets < 0 tokens without loss.
+// padding, targets < 0 or >= V tokens without loss.
 //
 //   run_count_kernel   one CTA per row: the loss-token count n of the run
 //                      each token belongs to (a chunk per thread, run
@@ -53,7 +53,7 @@ struct ChunkSummary {
 
 __global__ void __launch_bounds__(kRunThreads)
 run_count_kernel(const int32_t* __restrict__ seg, const int32_t* __restrict__ targets,
-                 int64_t S, int32_t* __restrict__ run_n, int32_t* __restrict__ n_samples) {
+                 int64_t S, int64_t V, int32_t* __restrict__ run_n, int32_t* __restrict__ n_samples) {
   __shared__ ChunkSummary cs[kRunThreads];
   __shared__ int32_t block_samples;
   const int64_t b = blockIdx.x;
@@ -63,7 +63,11 @@ run_count_kernel(const int32_t* __restrict__ seg, const int32_t* __restrict__ ta
   const int32_t* sg = seg ? seg + b * S : nullptr;
   const int32_t* tg = targets + b * S;
   auto id_of = [&](int64_t t) { return sg ? sg[t] : 0; };
-  auto loss_tok = [&](int64_t t) { return tg[t] >= 0 && id_of(t) >= 0 ? 1 : 0; };
+  // the predicate of ce_weight: a target outside [0, V) carries no loss
+  auto loss_tok = [&](int64_t t) {
+    const int32_t y = tg[t];
+    return y >= 0 && y < V && id_of(t) >= 0 ? 1 : 0;
+  };
   if (tid == 0) block_samples = 0;
   ChunkSummary c{};
   if (t0 < t1) {
@@ -461,7 +465,7 @@ cudaError_t launch_packed_ce(int64_t B, int64_t S, int64_t V, int dtype, const v
   const int nst = (int)std::min<size_t>(kCeMaxStages, kCeRingBytes / stage_bytes);
   const size_t smem = (size_t)nst * stage_bytes;
   const unsigned grid = (unsigned)std::min<size_t>(n, (size_t)sms);
-  run_count_kernel<<<(unsigned)B, kRunThreads, 0, st>>>(seg, targets, S, run_n, n_samples);
+  run_count_kernel<<<(unsigned)B, kRunThreads, 0, st>>>(seg, targets, S, V, run_n, n_samples);
   if (dtype == LWM_DTYPE_BF16) {
     auto kern = ce_kernel<__nv_bfloat16, kCeVecs>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=

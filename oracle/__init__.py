@@ -42,5 +42,4 @@ from .attention import (  # noqa: F401
     packed_loss_weights,
     packed_cross_entropy,
     kept_pairs,
-    attention_flops,
 )

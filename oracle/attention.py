@@ -318,15 +318,6 @@ def kept_pairs(seg, causal=True) -> int:
     return total
 
 
-def attention_flops(seg, heads: int, head_dim: int, causal=True) -> dict:
-    """Algorithmic FLOPs: forward 4 D H Pi (two matmuls, 2 flops per MAC),
-    backward 2.5x forward (five matmuls), as stated for blockwise exact
-    attention with recomputation (FlashAttention entry of the reference list)."""
-    pi = kept_pairs(seg, causal)
-    fwd = 4.0 * head_dim * heads * pi
-    return {"pairs": pi, "fwd": fwd, "bwd": 2.5 * fwd, "fwd_bwd": 3.5 * fwd}
-
-
 def sample_runs(seg_row):
     """Samples of one packed row: maximal runs of equal non-negative segment
     id, as (start, end) index pairs (research note, "训练方法": each packed
@@ -341,40 +332,46 @@ def sample_runs(seg_row):
     return runs
 
 
-def packed_loss_weights(seg, targets):
+def packed_loss_weights(seg, targets, vocab=None):
     """Per-token loss weights that make packed training equal to unpacked
     training with padding (research note, "训练方法", Masked Sequence
     Packing, and the ablation of section "评测": naive packing down-weights
     short samples).  Unpacked training averages each sample's loss over its
     own loss tokens, then averages over the samples of the batch; so a loss
     token of a sample with n loss tokens weighs 1 / (n * number of samples
-    that have a loss token).  targets < 0 mark tokens without loss."""
+    that have a loss token).  A token carries a loss iff its target is a
+    class index: 0 <= y (and y < vocab when the vocabulary size is given);
+    any other target marks a token without loss (prompts, padding)."""
     seg = np.asarray(seg)
     targets = np.asarray(targets)
+    has_loss = targets >= 0
+    if vocab is not None:
+        has_loss &= targets < vocab
     w = np.zeros(seg.shape, dtype=np.float64)
     samples = []
     for b in range(seg.shape[0]):
         for s, e in sample_runs(seg[b]):
-            n = int(np.count_nonzero(targets[b, s:e] >= 0))
+            n = int(np.count_nonzero(has_loss[b, s:e]))
             if n:
                 samples.append((b, s, e, n))
     for b, s, e, n in samples:
-        w[b, s:e] = np.where(targets[b, s:e] >= 0, 1.0 / (n * len(samples)), 0.0)
+        w[b, s:e] = np.where(has_loss[b, s:e], 1.0 / (n * len(samples)), 0.0)
     return w
 
 
 def packed_cross_entropy(logits, targets, seg):
     """Re-weighted cross-entropy of a packed batch and its gradient, float64.
 
-    logits [B, S, V], targets [B, S] (< 0: no loss), seg [B, S].
+    logits [B, S, V], targets [B, S] (outside [0, V): no loss), seg [B, S].
     Returns (loss, dlogits): loss = sum_t w_t * (logsumexp(z_t) - z_t[y_t]),
     dlogits_t = w_t * (softmax(z_t) - onehot(y_t))."""
     z = np.asarray(logits, dtype=np.float64)
     targets = np.asarray(targets)
-    w = packed_loss_weights(seg, targets)
+    V = z.shape[-1]
+    w = packed_loss_weights(seg, targets, vocab=V)
     m = z.max(axis=-1, keepdims=True)
     lse = m[..., 0] + np.log(np.exp(z - m).sum(axis=-1))
-    y = np.where(targets >= 0, targets, 0)
+    y = np.where((targets >= 0) & (targets < V), targets, 0)
     picked = np.take_along_axis(z, y[..., None], axis=-1)[..., 0]
     loss = float(np.sum(w * (lse - picked)))
     g = np.exp(z - lse[..., None])

@@ -52,3 +52,20 @@ def test_single_segment_counts_are_the_causal_triangle():
     assert bench.kept_pairs(seg) == S * (S + 1) // 2
     n = S // tile
     assert bench.tile_pairs(seg, heads) == heads * n * (n + 1) // 2
+
+
+def test_loss_bytes_count_only_the_logit_rows_read():
+    """Packed-loss bytes: logits of loss tokens (target in [0, V), segment id
+    >= 0) read once, every gradient row written once, targets and segment
+    ids read once; counted token by token here."""
+    rng = np.random.default_rng(9)
+    B, S, V, elt = 2, 50, 40, 2
+    seg = random_segments(rng, B, S, 3, 15, pad_tail=4)
+    targets = rng.integers(-1, V + 5, size=(B, S)).astype(np.int32)
+    read = 0
+    for b in range(B):
+        for t in range(S):
+            if 0 <= targets[b, t] < V and seg[b, t] >= 0:
+                read += V * elt
+    want = read + B * S * V * elt + B * S * 8
+    assert bench.loss_bytes(V, elt, targets, seg) == want

@@ -17,12 +17,14 @@ from workloads import random_segments
 pytestmark = pytest.mark.gpu
 
 
-def run_case(B, S, V, dtype, packed, seed, no_loss_frac=0.2):
+def run_case(B, S, V, dtype, packed, seed, no_loss_frac=0.2, out_of_vocab_frac=0.0):
     import long_context_causal_attention_b200 as lwm
     rng = np.random.default_rng(seed)
     seg = random_segments(rng, B, S, 5, max(6, S // 4), pad_tail=3) if packed else None
     targets = rng.integers(0, V, size=(B, S)).astype(np.int32)
     targets[rng.random((B, S)) < no_loss_frac] = -1   # tokens without loss (prompts)
+    oov = rng.random((B, S)) < out_of_vocab_frac        # targets >= V: no loss either
+    targets[oov] = V + rng.integers(0, 3 * V, size=int(oov.sum()))
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
     logits = (torch.randn((B, S, V), generator=g, device="cuda") * 2.0).to(dtype)
@@ -59,3 +61,11 @@ def test_packed_cross_entropy_no_loss_rows():
     """Long stretches of rows without a loss pass through the row ring with
     no data: most rows here carry none."""
     run_case(2, 1500, 1024, torch.bfloat16, True, seed=77, no_loss_frac=0.9)
+
+
+def test_packed_cross_entropy_out_of_vocabulary_targets():
+    """Targets >= V carry no loss: they must not count towards their
+    sample's token count n nor make a sample count, in the run-counting
+    kernel as in the loss kernel."""
+    run_case(2, 900, 500, torch.bfloat16, True, seed=91, out_of_vocab_frac=0.3)
+    run_case(1, 300, 64, torch.float32, True, seed=92, no_loss_frac=0.0, out_of_vocab_frac=0.6)

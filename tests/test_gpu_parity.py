@@ -69,7 +69,26 @@ SMALL = [
     ("d64_bf16_noncausal_pad", 1, 450, 2, 64, "bf16", 1e4, False, 1.0, "random_pad"),
     ("no_rope", 1, 384, 2, 128, "bf16", 0.0, True, 1.0, "single"),
     ("long_segments_1000", 1, 1000, 2, 128, "bf16", 1e6, True, 1.0, "random_long"),
+    # ids in any order: padding in the middle of a row, an id that comes back
+    # after other ids, a row that is all padding (both kernel families)
+    ("irregular_ids_bf16", 3, 700, 2, 128, "bf16", 1e6, True, 1.0, "irregular"),
+    ("irregular_ids_bf16_noncausal", 3, 300, 2, 128, "bf16", 1e4, False, 1.0, "irregular"),
+    ("irregular_ids_fp32", 3, 400, 2, 128, "fp32", 1e6, True, 1.0, "irregular"),
+    ("irregular_ids_d64_bf16", 3, 333, 2, 64, "bf16", 1e6, True, 1.0, "irregular"),
 ]
+
+
+def irregular_segments(rng, B, S):
+    """Packed rows, then: row 0 gets a padding run in its middle and its
+    first segment's id again on a later stretch (those tokens attend to the
+    first segment's tokens, since the mask compares ids only); row 1 is all
+    padding; row 2 alternates two ids in short runs."""
+    seg = random_segments(rng, B, S, 20, 150)
+    seg[0, S // 3:S // 3 + 40] = -1
+    seg[0, 2 * S // 3:2 * S // 3 + 60] = seg[0, 0]
+    seg[1, :] = -1
+    seg[2, :] = (np.arange(S) // 37) % 2
+    return seg
 
 
 @pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
@@ -83,6 +102,8 @@ def test_small_cases_full(lwm, case):
         seg = random_segments(rng, B, S, 1, 150)
     elif segkind == "random_long":
         seg = random_segments(rng, B, S, 100, 700)
+    elif segkind == "irregular":
+        seg = irregular_segments(rng, B, S)
     else:
         seg = random_segments(rng, B, S, 1, 150, pad_tail=min(5, S - 1))
         seg[:, :3] = -1

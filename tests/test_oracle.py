@@ -544,6 +544,37 @@ def test_packed_loss_equals_unpacked_per_sample_mean():
     assert abs(naive - loss) > 1e-3
 
 
+def test_packed_loss_out_of_vocabulary_targets_carry_no_loss():
+    """A target outside [0, V) marks a token without loss, like a negative
+    one: the loss is the mean over samples of torch's per-sample mean
+    cross-entropy over the in-vocabulary targets only, and such tokens get a
+    zero gradient row."""
+    import torch
+    rng = np.random.default_rng(43)
+    B, S, V = 2, 30, 9
+    seg = np.stack([np.repeat([0, 1, 2], [10, 6, 14]), np.repeat([3, -1], [26, 4])])
+    targets = rng.integers(0, V, size=(B, S))
+    targets[0, 10:16] = V + rng.integers(0, 5, size=6)   # the whole of sample 1
+    targets[0, [2, 20, 21]] = V                          # a few inside other samples
+    targets[1, 5] = 2 ** 30
+    z = rng.standard_normal((B, S, V))
+    loss, d = oracle.packed_cross_entropy(z, targets, seg)
+    keep_all = (targets >= 0) & (targets < V)
+    per_sample = []
+    for b in range(B):
+        for s, e in oracle.sample_runs(seg[b]):
+            keep = keep_all[b, s:e]
+            if keep.any():
+                zz = torch.from_numpy(z[b, s:e][keep])
+                yy = torch.from_numpy(targets[b, s:e][keep])
+                per_sample.append(torch.nn.functional.cross_entropy(zz, yy).item())
+    assert len(per_sample) == 3   # sample 1 of row 0 has no in-vocabulary target
+    assert abs(loss - np.mean(per_sample)) < 1e-12
+    assert np.all(d[~keep_all] == 0)
+    w = oracle.packed_loss_weights(seg, targets, vocab=V)
+    assert abs(w.sum() - 1.0) < 1e-12 and np.all(w[~keep_all] == 0)
+
+
 def test_packed_loss_gradient_matches_autograd():
     import torch
     rng = np.random.default_rng(42)

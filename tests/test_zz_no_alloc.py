@@ -6,9 +6,10 @@ must not take the synchronisation or out-of-memory risk of one).  For them
 the library keeps a fixed 40 MiB scratch array per device and this entry
 point uses it instead of a caller workspace.  The test calls it through the
 C ABI twice in a row, on two different inputs, and checks each result
-against the ordinary lwm_attn_fwd (own workspace) within the bf16 parity
-bound; it also checks that a problem too big for the array is refused before
-anything runs.  This file is collected last so that a failure here cannot
+against the ordinary lwm_attn_fwd (own workspace) and against the float64
+oracle, within the bf16 parity bound, and reads the device status word of
+each call back through lwm_attn_fwd_noalloc_read_status; it also checks that
+a problem too big for the array is refused before anything runs.  This file is collected last so that a failure here cannot
 stop the other tests from running.
 """
 import ctypes
@@ -17,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from tests.parity_util import assert_close, to64
 from workloads import Workload, make_tensors, random_segments
 
@@ -47,6 +49,13 @@ def test_noalloc_forward_matches_workspace_forward():
         t = make_tensors(w, seed=seed, device="cuda", with_grad_out=False)
         st, o, lse = _noalloc(lwm, t["q"], t["k"], t["v"], seg, theta)
         assert st == 0, lwm.lwm_status_string(st)
+        dev_st = lwm._lib.lib().lwm_attn_fwd_noalloc_read_status(
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert dev_st == 0, lwm.lwm_status_string(dev_st)
+        ref = oracle.attention_forward(to64(t["q"]), to64(t["k"]), to64(t["v"]),
+                                       seg.cpu().numpy(), causal=True, theta=theta)
+        assert_close("o vs oracle", to64(o), ref[0], "bf16")
+        assert_close("lse vs oracle", to64(lse), ref[1], "bf16")
         o_ref, lse_ref = lwm.lwm_attn_fwd(t["q"], t["k"], t["v"], seg, True, theta,
                                           check_status=True)
         torch.cuda.synchronize()
