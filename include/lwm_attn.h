@@ -135,15 +135,26 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
  *   - Set-up: the first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
  *     first call before any stream capture.  A failed lookup returns
- *     LWM_ERR_CUDA.
+ *     LWM_ERR_CUDA.  The address is kept for the life of the process: after
+ *     cudaDeviceReset (or anything else that replaces the device's primary
+ *     context) it is stale, and this entry point must not be called again
+ *     in that process.
  *   - Sharing: all calls on a device share the one array, which keeps the
  *     last call's contents (the call clears what must start at zero).  Calls
  *     that overlap on the GPU (different streams, or host threads) race on
  *     it; serialise them.
- *   - lwm_attn_read_status reads nothing for this entry point (there is no
- *     caller workspace); device-side errors stay in the library's array. */
+ *   - Device-side status (a bounded wait that ran out) lands in the status
+ *     word at the start of the library's array, not in a caller workspace:
+ *     read it with lwm_attn_fwd_noalloc_read_status. */
 lwm_status lwm_attn_fwd_noalloc(const lwm_attn_desc* desc, const void* q, const void* k,
                                 const void* v, void* o, float* lse, void* stream);
+
+/* Status word of the last lwm_attn_fwd_noalloc call on the current device,
+ * as lwm_attn_read_status gives it for a caller workspace: waits for
+ * `stream`, then returns LWM_OK or the code a kernel recorded.  The same
+ * once-per-device set-up as lwm_attn_fwd_noalloc (no allocation); LWM_ERR_CUDA
+ * if the lookup or the copy fails. */
+lwm_status lwm_attn_fwd_noalloc_read_status(void* stream);
 
 /* Decode step (research note, "模型架构" and "Infra": generation over a
  * million-token context).  n_new new tokens are the last n_new positions of

@@ -32,7 +32,7 @@ ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_
                 "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait",
                 "lwm_rope_apply_at", "lwm_attn_merge", "lwm_accumulate", "lwm_convert_f32",
                 "lwm_attn_fwd_pair", "lwm_attn_bwd_pair", "lwm_packed_ce_workspace_size",
-                "lwm_packed_cross_entropy")
+                "lwm_packed_cross_entropy", "lwm_attn_fwd_noalloc_read_status")
 DECODE_MAX_NEW = 16
 
 
@@ -82,6 +82,8 @@ def _load():
     lib.lwm_attn_set_timing_events.restype = None
     lib.lwm_attn_fwd_noalloc.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P]
     lib.lwm_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.lwm_attn_fwd_noalloc_read_status.argtypes = [P]
+    lib.lwm_attn_fwd_noalloc_read_status.restype = ctypes.c_int
     lib.lwm_attn_decode_workspace_size.argtypes = [ctypes.POINTER(LwmAttnDesc), ctypes.c_int64]
     lib.lwm_attn_decode_workspace_size.restype = ctypes.c_size_t
     lib.lwm_attn_decode.argtypes = [ctypes.POINTER(LwmAttnDesc), ctypes.c_int64, P, P, P, P, P, P,

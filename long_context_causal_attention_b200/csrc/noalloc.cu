@@ -60,4 +60,11 @@ lwm_status lwm_attn_fwd_noalloc(const lwm_attn_desc* desc, const void* q, const 
   return lwm_attn_fwd(desc, q, k, v, o, lse, scratch, kNoAllocScratchBytes, stream);
 }
 
+lwm_status lwm_attn_fwd_noalloc_read_status(void* stream) {
+  void* scratch = nullptr;
+  const lwm_status s = scratch_for_current_device(&scratch);
+  if (s != LWM_OK) return s;
+  return lwm_attn_read_status(scratch, stream);
+}
+
 }  // extern "C"
