@@ -45,6 +45,16 @@ Path choose_fwd_path(const Problem& p) {
   return Path::kSm100;
 }
 
+// LWM_ATTN_SPLIT_BWD=1 runs the tensor-core backward as two kernels (key-
+// stationary dK/dV, query-stationary dQ) instead of the one-pass kernel.
+static bool split_bwd() {
+  static const bool v = [] {
+    const char* e = std::getenv("LWM_ATTN_SPLIT_BWD");
+    return e && e[0] == '1';
+  }();
+  return v;
+}
+
 Path choose_bwd_path(const Problem& p) {
   if (force_simt() || !tensor_core_shape(p) || !sm100_available()) return Path::kSimt;
   return Path::kSm100;
@@ -83,6 +93,7 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
       const size_t padded = (size_t)p.B * p.H * (size_t)p.n_tiles * kTile * sizeof(float);
       w.lse2_pad = static_cast<float*>(take(padded));
       w.delta_pad = static_cast<float*>(take(padded));
+      w.dq_acc = static_cast<float*>(take(fused_dq_acc_bytes(p.B, p.H, p.n_tiles)));
     }
   }
   w.bytes = align_up(off, 1024);
@@ -232,11 +243,19 @@ lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   if (choose_bwd_path(p) == Path::kSm100) {
     e = launch_bwd_prep(p, o, d_o, lse, w, st);
+    if (e == cudaSuccess && !split_bwd())
+      e = cudaMemsetAsync(w.dq_acc, 0, fused_dq_acc_bytes(p.B, p.H, p.n_tiles), st);
     if (e != cudaSuccess) return LWM_ERR_CUDA;
     record_event(2, st);
-    e = launch_sm100_bwd_dkdv(p, w, v, d_o, dk, dv, st);
-    record_event(4, st);
-    if (e == cudaSuccess) e = launch_sm100_bwd_dq(p, w, v, d_o, dq, st);
+    if (split_bwd()) {
+      e = launch_sm100_bwd_dkdv(p, w, v, d_o, dk, dv, st);
+      record_event(4, st);
+      if (e == cudaSuccess) e = launch_sm100_bwd_dq(p, w, v, d_o, dq, st);
+    } else {
+      e = launch_sm100_bwd_fused(p, w, v, d_o, dq, dk, dv, st);
+      record_event(4, st);
+      if (e == cudaSuccess) e = launch_dq_finish(p, w, dq, st);
+    }
     record_event(3, st);
     return cuda_status(e);
   }

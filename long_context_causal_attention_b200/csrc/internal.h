@@ -38,6 +38,7 @@ struct Workspace {
   float* delta;        // [B, H, S] fp32 dot(dO, O) per row (backward, CUDA-core path)
   float* lse2_pad;     // [B, H, n_tiles*128] LSE*log2(e) or +inf (backward, tensor-core path)
   float* delta_pad;    // [B, H, n_tiles*128] dot(dO, O) or 0 (backward, tensor-core path)
+  float* dq_acc;       // [B*H, n_tiles, 32, 128, 4] fp32 dQ~ sums (backward, tensor-core path)
   float* dec_ml;       // [B, H, T, n_chunks, 2] decode chunk max and sum (log2 domain)
   float* dec_o;        // [B, H, T, n_chunks, D] decode chunk sums of p * v
   size_t bytes;        // total bytes the layout needs
@@ -93,6 +94,12 @@ cudaError_t launch_sm100_bwd_dkdv(const Problem& p, const Workspace& ws, const v
                                   const void* d_o, void* dk, void* dv, cudaStream_t st);
 cudaError_t launch_sm100_bwd_dq(const Problem& p, const Workspace& ws, const void* v,
                                 const void* d_o, void* dq, cudaStream_t st);
+// One-pass backward: dK, dV, and dQ~ partial sums added into ws.dq_acc
+// (which must be zero beforehand); launch_dq_finish turns those into bf16 dq.
+size_t fused_dq_acc_bytes(int64_t B, int64_t H, int64_t n_tiles);
+cudaError_t launch_sm100_bwd_fused(const Problem& p, const Workspace& ws, const void* v,
+                                   const void* d_o, void* dq, void* dk, void* dv, cudaStream_t st);
+cudaError_t launch_dq_finish(const Problem& p, const Workspace& ws, void* dq, cudaStream_t st);
 
 // Bounded-wait self-test: one CTA waits on an mbarrier (armed by an arrival
 // or not) for at most limit_cycles; a wait that runs out records

@@ -288,6 +288,17 @@ __device__ __forceinline__ void mma_km128(uint32_t d, uint64_t a_desc, uint64_t 
   }
 }
 
+// D (+)= A * B over K = 128, A and B both MN-major tiles whose rows are K
+// (a k-step is 16 rows = 2048 bytes in each).
+__device__ __forceinline__ void mma_mm128(uint32_t d, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t off = (uint64_t)((kk * 2048) >> 4);
+    mma_ss(d, a_desc + off, b_desc + off, idesc, kk > 0 ? 1u : acc);
+  }
+}
+
 // D (+)= A * B over K = 128 with A (bf16) in tensor memory and B an MN-major
 // tile whose rows are K (a k-step is 16 rows = 2048 bytes).  A's k-step kk
 // starts at column a_col(kk): QUARTERS = false packs the 128 K values into 64
@@ -330,6 +341,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Fire-and-forget fp32 add of four consecutive floats in global memory
+// (performed in L2; the address must be 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
