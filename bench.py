@@ -10,10 +10,15 @@ Work is counted algorithmically: forward 4*D*H*Pi flops, backward 2.5x that,
 Pi = allowed (i, j) pairs (causal within segments; skipped tiles and masked
 elements are not counted).
 
-Under torchrun each rank runs an independent problem of the same size
-(different seed): weak scaling, no collective on the data path.  Timing is
-on the device (CUDA events) with a barrier and a synchronize on both sides;
-rank 0 prints one JSON line with the max time over ranks.
+With --gpus N > 1 the bench launches N ranks itself (torch.distributed.run,
+one process per GPU) unless it already runs under torchrun with WORLD_SIZE =
+N.  Default --parallel heads: the heads of one problem are split over the
+ranks (the pages' tensor-parallel axis; each rank runs the single-GPU
+kernels on H/N heads, no collective on the data path), strong scaling.
+--parallel replicas: each rank runs an independent problem of the same size
+(different seed), weak scaling.  Timing is on the device (CUDA events) with a
+barrier and a synchronize on both sides; rank 0 prints one JSON line with
+the max time over ranks and the whole job's throughput.
 """
 from __future__ import annotations
 
@@ -53,6 +58,16 @@ def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
         c = counts.astype(np.int64)
         total += int((c * (c + 1) // 2).sum()) if causal else int((c * c).sum())
     return total
+
+
+# The same for the one-pass backward kernel (attn_bwd_fused_kernel); empty
+# until a capture of the current kernel is recorded.
+FUSED_TRAFFIC = {"bytes": {}, "source_sha256": ""}
+
+
+def split_backward() -> bool:
+    """The library runs the two-kernel backward (LWM_ATTN_SPLIT_BWD=1)."""
+    return os.environ.get("LWM_ATTN_SPLIT_BWD") == "1"
 
 
 def load_peaks():
@@ -253,11 +268,19 @@ def ours(args):
             dist.barrier()
 
     w = WORKLOADS[args.workload]
-    seed = rank_seed(args.seed, rank)
+    heads_split = ws > 1 and args.parallel == "heads"
+    # head split: every rank draws the same whole problem and keeps its heads
+    # (the scatter); replicas: each rank draws its own problem
+    seed = args.seed if heads_split else rank_seed(args.seed, rank)
     seg = segment_ids(w, seed=seed)
     single = w.segments == "single"
     seg_d = None if single else torch.as_tensor(seg, dtype=torch.int32, device=dev)
     t = make_tensors(w, seed=seed, device=dev, with_grad_out=True)
+    if heads_split:
+        from long_context_causal_attention_b200.heads import scatter_heads
+        t = {name: scatter_heads(x, rank, ws) for name, x in t.items()}
+        torch.cuda.empty_cache()
+        w = w.with_(heads=w.heads // ws)
     q, k, v, do = t["q"], t["k"], t["v"], t["do"]
     desc = lwm.make_desc(q, seg_d, w.causal, w.theta, w.scale)
     ws_f = lwm.alloc_workspace(desc, False, dev)
@@ -381,20 +404,33 @@ def ours(args):
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
-    # dominant kernel: dK/dV, whose four GEMMs per kept pair (S^T, dP^T, dV,
-    # dK) are all algorithmic work: 8*D flops per pair and head
-    dkdv_flops = 8.0 * w.head_dim * w.heads * pairs
-    achieved = dkdv_flops / (dkdv_k * 1e-3) / 1e12 if dkdv_k > 0.0 else None
-    traffic = None
     units = tile_pairs(seg, w.heads, w.causal)
-    if (w.name in DKDV_TRAFFIC["bytes"] and
-            DKDV_TRAFFIC["source_sha256"] == kernel_source_sha256("attn_bwd_sm100.cu")):
-        traffic = DKDV_TRAFFIC["bytes"][w.name]
     bwd_flops = 2.5 * fwd_flops
     dq_k = bwd_k - dkdv_k
-    kernel, bound, rpeak, peak_note = "attn_bwd_dkdv_kernel", "tensor", peak, \
+    traffic = None
+    tensor_cores = w.dtype == "bf16" and w.head_dim == 128
+    if split_backward() or not tensor_cores:
+        # dominant kernel: dK/dV, whose four GEMMs per kept pair (S^T, dP^T,
+        # dV, dK) are all algorithmic work: 8*D flops per pair and head
+        main_flops = 8.0 * w.head_dim * w.heads * pairs
+        kernel, algorithmic = "attn_bwd_dkdv_kernel", \
+            "8*D*H flops per kept (query, key) pair: S^T, dP^T, dV, dK"
+        if (w.name in DKDV_TRAFFIC["bytes"] and
+                DKDV_TRAFFIC["source_sha256"] == kernel_source_sha256("attn_bwd_sm100.cu")):
+            traffic = DKDV_TRAFFIC["bytes"][w.name]
+    else:
+        # dominant kernel: the one-pass backward, all five GEMMs per kept pair
+        # (S^T, dP^T, dV, dK, dQ): the whole backward's algorithmic work
+        main_flops = bwd_flops
+        kernel, algorithmic = "attn_bwd_fused_kernel", \
+            "10*D*H flops per kept (query, key) pair: S^T, dP^T, dV, dK, dQ"
+        if (w.name in FUSED_TRAFFIC["bytes"] and
+                FUSED_TRAFFIC["source_sha256"] == kernel_source_sha256("attn_bwd_fused_sm100.cu")):
+            traffic = FUSED_TRAFFIC["bytes"][w.name]
+    achieved = main_flops / (dkdv_k * 1e-3) / 1e12 if dkdv_k > 0.0 else None
+    bound, rpeak, peak_note = "tensor", peak, \
         f"{peak_src} bf16 sustained (kernel timed inside a long step)"
-    if w.dtype != "bf16" or w.head_dim != 128:
+    if not tensor_cores:
         # the CUDA-core kernels (fp32 arithmetic): bound by the FFMA pipes,
         # 128 fp32 lanes per SM, one fused multiply-add (2 flops) per lane
         # per clock, at the maximum SM clock the device reports
@@ -406,15 +442,18 @@ def ours(args):
                      f"{sm_max:.0f} MHz (maximum SM clock)")
     roofline = {"bound": bound, "achieved": achieved, "peak": rpeak, "unit": "TFLOP/s",
                 "frac": achieved / rpeak if achieved else None, "traffic": traffic,
-                "kernel": kernel,
-                "algorithmic": "8*D*H flops per kept (query, key) pair: S^T, dP^T, dV, dK",
+                "kernel": kernel, "algorithmic": algorithmic,
                 "tile_pairs": units,
                 "peak_source": peak_note,
-                "dkdv_kernel_ms": dkdv_k, "dq_kernel_ms": dq_k, "fwd_kernel_ms": fwd_k,
+                "bwd_main_kernel_ms": dkdv_k, "bwd_tail_ms": dq_k, "fwd_kernel_ms": fwd_k,
                 "fwd_kernel_tflops": fwd_flops / (fwd_k * 1e-3) / 1e12,
-                "bwd_kernels_tflops": bwd_flops / (bwd_k * 1e-3) / 1e12,
-                "dq_kernel_tflops_incl_recompute": (6.0 * w.head_dim * w.heads * pairs
-                                                    / (dq_k * 1e-3) / 1e12) if dq_k else None}
+                "bwd_kernels_tflops": bwd_flops / (bwd_k * 1e-3) / 1e12}
+    if tensor_cores and clk and clk.get("sm_mhz") and achieved:
+        # clock-normalised: the dense bf16 rate of one SM is 8192 flops per
+        # clock (a 128x128x16 MMA every 64 clocks), at the SM clock measured
+        # during the timed region
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        roofline["frac_of_clock_peak"] = achieved * 1e12 / (sms * 8192.0 * clk["sm_mhz"] * 1e6)
 
     # the HBM-bound pre-pass on its own (step A2): lwm_rope_apply over q,
     # reading and writing every element once, against the copy bandwidth
@@ -445,18 +484,26 @@ def ours(args):
                          f"of one head of {w.name} ({fl / 1e9:.2f} GFLOP in {dt:.1f} s)"}
 
     if rank == 0:
+        if heads_split:
+            parallelism = f"tp{ws}: the heads of one problem split, {w.heads} per GPU"
+            tokens = w.batch * w.seqlen
+        else:
+            parallelism = f"independent problem per GPU x{ws}"
+            tokens = w.batch * w.seqlen * ws
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "higher_is_better": True, "scaling": "strong" if heads_split else "weak",
+            "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
-                       "heads": w.heads, "head_dim": w.head_dim, "theta": w.theta,
+                       "heads": w.heads * ws if heads_split else w.heads,
+                       "head_dim": w.head_dim, "theta": w.theta,
                        "causal": w.causal, "segments": w.segments,
-                       "parallelism": f"independent problem per GPU x{ws}",
+                       "parallelism": parallelism,
                        "l2": "inputs larger than L2 (1 GiB per tensor vs 126 MB), no flush",
                        "algorithmic_fwd_bwd_tflop_per_gpu": step_flops / 1e12,
-                       "tokens_per_s": w.batch * w.seqlen * ws / (ms_step * 1e-3),
+                       "tokens_per_s": tokens / (ms_step * 1e-3),
                        "pct_of_bf16_peak": 100.0 * value / ws / peak},
             "roofline": roofline,
             "cpu_baseline": cpu,
@@ -836,6 +883,19 @@ def ours_loss(args):
     return 0
 
 
+def launch_ranks(n: int) -> int:
+    """Run this command as n ranks on this node (one process per GPU),
+    rendezvous on 127.0.0.1; returns the launcher's exit status."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -847,7 +907,17 @@ def main():
     ap.add_argument("--oracle-rows", type=int, default=1024)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", choices=["heads", "replicas"], default="heads",
+                    help="N > 1: split the heads of one problem (strong scaling) or run "
+                         "one independent problem per GPU (weak scaling)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(args.gpus)
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={ws}: launch one rank per GPU")
     extra = WORKLOADS[args.workload].extra
     if args.impl == "reference":
         if "n_new" in extra:
