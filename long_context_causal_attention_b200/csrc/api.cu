@@ -40,9 +40,26 @@ static bool force_simt() {
   return v;
 }
 
+// LWM_ATTN_FP32_SIMT=1 keeps fp32 problems on the CUDA-core kernels (full
+// fp32 arithmetic) instead of the split-precision tensor-core path.
+static bool fp32_simt() {
+  static const bool v = [] {
+    const char* e = std::getenv("LWM_ATTN_FP32_SIMT");
+    return e && e[0] == '1';
+  }();
+  return v;
+}
+
+// fp32, head_dim 64 or 128: the shapes the split-precision kernels take.
+bool x3_shape(const Problem& p) {
+  return p.dtype == LWM_DTYPE_FP32 && (p.D == 64 || p.D == 128) && p.S < ((int64_t)1 << 31);
+}
+
 Path choose_fwd_path(const Problem& p) {
-  if (force_simt() || !tensor_core_shape(p) || !sm100_available()) return Path::kSimt;
-  return Path::kSm100;
+  if (force_simt() || !sm100_available()) return Path::kSimt;
+  if (tensor_core_shape(p)) return Path::kSm100;
+  if (x3_shape(p) && !fp32_simt()) return Path::kSm100X3;
+  return Path::kSimt;
 }
 
 // LWM_ATTN_SPLIT_BWD=1 runs the tensor-core backward as two kernels (key-
@@ -83,7 +100,15 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
   w.q_lo = static_cast<int32_t*>(take(tiles));
   w.k_hi = static_cast<int32_t*>(take(tiles));
   const size_t nel = (size_t)p.B * p.S * p.H * p.D;
-  if (p.theta > 0.0) {
+  if (!bwd && choose_fwd_path(p) == Path::kSm100X3) {
+    // split planes replace the rotated copies (the split pre-pass rotates)
+    w.qx_hi = take(nel * 2);
+    w.qx_lo = take(nel * 2);
+    w.kx_hi = take(nel * 2);
+    w.kx_lo = take(nel * 2);
+    w.vx_hi = take(nel * 2);
+    w.vx_lo = take(nel * 2);
+  } else if (p.theta > 0.0) {
     w.q_rot = take(nel * p.elt);
     w.k_rot = take(nel * p.elt);
   }
@@ -211,10 +236,28 @@ lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   s = check_ws(p, false, ws, ws_bytes, &w);
   if (s != LWM_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = prologue(p, w, q, k, st);
+  const Path path = choose_fwd_path(p);
+  cudaError_t e;
+  if (path == Path::kSm100X3) {
+    e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
+    if (e == cudaSuccess) e = launch_segment_bounds(p, w, st);
+    if (e == cudaSuccess)
+      e = launch_split(p.B, p.S, p.H, p.D, p.theta, static_cast<const float*>(q), w.qx_hi,
+                       w.qx_lo, st);
+    if (e == cudaSuccess)
+      e = launch_split(p.B, p.S, p.H, p.D, p.theta, static_cast<const float*>(k), w.kx_hi, w.kx_lo, st);
+    if (e == cudaSuccess)
+      e = launch_split(p.B, p.S, p.H, p.D, 0.0, static_cast<const float*>(v), w.vx_hi, w.vx_lo, st);
+    if (e != cudaSuccess) return LWM_ERR_CUDA;
+    record_event(0, st);
+    e = launch_sm100_fwd_x3(p, w, static_cast<float*>(o), lse, st);
+    record_event(1, st);
+    return cuda_status(e);
+  }
+  e = prologue(p, w, q, k, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   record_event(0, st);
-  if (choose_fwd_path(p) == Path::kSm100)
+  if (path == Path::kSm100)
     e = launch_sm100_fwd(p, w, v, o, lse, st);
   else
     e = launch_simt_fwd(p, w, v, o, lse, st);

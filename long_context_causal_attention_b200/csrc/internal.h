@@ -39,12 +39,21 @@ struct Workspace {
   float* lse2_pad;     // [B, H, n_tiles*128] LSE*log2(e) or +inf (backward, tensor-core path)
   float* delta_pad;    // [B, H, n_tiles*128] dot(dO, O) or 0 (backward, tensor-core path)
   float* dq_acc;       // [B*H, n_tiles, 32, 128, 4] fp32 dQ~ sums (backward, tensor-core path)
+  // fp32 on the tensor cores: bf16 hi / lo planes [B, S, H, D] of the rotated
+  // q and k and of v (forward)
+  void* qx_hi;
+  void* qx_lo;
+  void* kx_hi;
+  void* kx_lo;
+  void* vx_hi;
+  void* vx_lo;
   float* dec_ml;       // [B, H, T, n_chunks, 2] decode chunk max and sum (log2 domain)
   float* dec_o;        // [B, H, T, n_chunks, D] decode chunk sums of p * v
   size_t bytes;        // total bytes the layout needs
 };
 
-enum class Path { kSimt = 0, kSm100 = 1 };
+// kSm100X3: fp32 data on the bf16 tensor cores through hi/lo splits.
+enum class Path { kSimt = 0, kSm100 = 1, kSm100X3 = 2 };
 
 // Which kernels serve the forward / backward of this problem on this device.
 Path choose_fwd_path(const Problem& p);
@@ -61,6 +70,10 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws);
 // pos0: position of token 0 of each row (p = pos0 + index in the row).
 cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, double theta,
                         const void* x, void* y, int inverse, cudaStream_t st, int64_t pos0 = 0);
+// fp32 x [B,S,H,D] -> bf16 planes hi = bf16(y), lo = bf16(y - hi) with y =
+// R(p) x when theta > 0 (p = pos0 + index in the row), else y = x.
+cudaError_t launch_split(int64_t B, int64_t S, int64_t H, int64_t D, double theta, const float* x,
+                         void* hi, void* lo, cudaStream_t st, int64_t pos0 = 0);
 // Block results of one sequence split into key blocks (ring order):
 // o_acc/lse_acc <- exact log-sum-exp merge with (o_part, lse_part).
 cudaError_t launch_attn_merge(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, float* o_acc,
@@ -87,6 +100,9 @@ cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float
 
 cudaError_t launch_sm100_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                              float* lse, cudaStream_t st);
+// fp32 forward on the tensor cores from the split planes in ws (head_dim 64 or 128).
+cudaError_t launch_sm100_fwd_x3(const Problem& p, const Workspace& ws, float* o, float* lse,
+                                cudaStream_t st);
 
 cudaError_t launch_bwd_prep(const Problem& p, const void* o, const void* d_o, const float* lse,
                             const Workspace& ws, cudaStream_t st);

@@ -58,6 +58,55 @@ __global__ void __launch_bounds__(128) rope_kernel(const T* __restrict__ x, T* _
   }
 }
 
+// fp32 operand -> two bf16 planes for the split-precision tensor-core path:
+// y = R(p) x when `rotate` (RoPE as rope_kernel computes it), else y = x;
+// hi = bf16(y), lo = bf16(y - hi), both rounded to nearest, so hi + lo
+// carries y to about 2^-17 relative.  Thread layout as in rope_kernel, four
+// fp32 elements (two rotary pairs) per thread and step.
+__global__ void __launch_bounds__(128) split_kernel(const float* __restrict__ x,
+                                                    __nv_bfloat16* __restrict__ hi,
+                                                    __nv_bfloat16* __restrict__ lo, int64_t n_tok,
+                                                    int64_t S, int H, int D, double log2_theta,
+                                                    int rotate, int64_t pos0) {
+  constexpr int N = 4, P = 2;
+  const int per_head = D / N;
+  const int c = threadIdx.x % per_head;
+  const int hg = threadIdx.x / per_head;
+  const int heads_per_pass = blockDim.x / per_head;
+  if (hg >= heads_per_pass) return;
+  double w[P];
+#pragma unroll
+  for (int u = 0; u < P; ++u) w[u] = rotate ? rope_freq(c * P + u, D, log2_theta) : 0.0;
+  for (int64_t tok = blockIdx.x; tok < n_tok; tok += gridDim.x) {
+    const int64_t pos = pos0 + tok % S;
+    float cs[P] = {1.f, 1.f}, sn[P] = {0.f, 0.f};
+    if (rotate) {
+#pragma unroll
+      for (int u = 0; u < P; ++u) rope_cos_sin_w(pos, w[u], &cs[u], &sn[u]);
+    }
+    const size_t base = (size_t)tok * H * D;
+    for (int h = hg; h < H; h += heads_per_pass) {
+      const size_t off = base + (size_t)h * D + (size_t)c * N;
+      const float4 v = *reinterpret_cast<const float4*>(x + off);
+      const float e[4] = {v.x, v.y, v.z, v.w};
+      float y[4];
+#pragma unroll
+      for (int u = 0; u < P; ++u) {
+        y[2 * u] = e[2 * u] * cs[u] - e[2 * u + 1] * sn[u];
+        y[2 * u + 1] = e[2 * u] * sn[u] + e[2 * u + 1] * cs[u];
+      }
+      __nv_bfloat16 h4[4], l4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        h4[k] = __float2bfloat16_rn(y[k]);
+        l4[k] = __float2bfloat16_rn(y[k] - __bfloat162float(h4[k]));
+      }
+      *reinterpret_cast<uint2*>(hi + off) = *reinterpret_cast<const uint2*>(h4);
+      *reinterpret_cast<uint2*>(lo + off) = *reinterpret_cast<const uint2*>(l4);
+    }
+  }
+}
+
 // delta[b, h, i] = sum_d dO[b, i, h, d] * O[b, i, h, d]; one warp per (token, head).
 template <typename T>
 __global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, const T* __restrict__ d_o,
@@ -139,6 +188,18 @@ cudaError_t launch_rope(int64_t B, int64_t S, int64_t H, int64_t D, int dtype, d
     rope_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(x), static_cast<float*>(y),
                                              n_tok, S, (int)H, (int)D, l2t, inverse, pos0);
   }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split(int64_t B, int64_t S, int64_t H, int64_t D, double theta, const float* x,
+                         void* hi, void* lo, cudaStream_t st, int64_t pos0) {
+  const int64_t n_tok = B * S;
+  if (n_tok == 0) return cudaSuccess;
+  const int rotate = theta > 0.0;
+  split_kernel<<<grid_for(n_tok), 128, 0, st>>>(x, static_cast<__nv_bfloat16*>(hi),
+                                                static_cast<__nv_bfloat16*>(lo), n_tok, S, (int)H,
+                                                (int)D, rotate ? log2(theta) : 0.0, rotate, pos0);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -266,6 +266,11 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr) {
   return smem_desc_sw128(saddr, kOperandBoxBytes, 1024);
 }
 
+// MN-major operand whose 64-element MN blocks (TMA boxes) lie lbo_bytes apart.
+__device__ __forceinline__ uint64_t mnmajor_desc_lbo(uint32_t saddr, uint32_t lbo_bytes) {
+  return smem_desc_sw128(saddr, lbo_bytes, 1024);
+}
+
 // D (+)= A * B^T over K = 128, A and B K-major tiles (8 MMAs of K = 16): a
 // k-step walks 32 bytes inside the 128-byte row, then moves to the second box.
 __device__ __forceinline__ void mma_kk128(uint32_t d, uint64_t a_desc, uint64_t b_desc,
