@@ -409,7 +409,17 @@ def ours(args):
     dq_k = bwd_k - dkdv_k
     traffic = None
     tensor_cores = w.dtype == "bf16" and w.head_dim == 128
-    if split_backward() or not tensor_cores:
+    split_fp32 = (w.dtype == "fp32" and w.head_dim in (64, 128)
+                  and os.environ.get("LWM_ATTN_FP32_SIMT") != "1")
+    if split_fp32:
+        # fp32 on the tensor cores: every product is three bf16 products, so
+        # the roofline is the dense bf16 peak / 3; the dominant part is the
+        # backward (dK/dV then dQ kernels, timed together): 10*D*H flops per
+        # kept pair of algorithmic work
+        main_flops = bwd_flops
+        kernel, algorithmic = "attn_bwd_dkdv_x3_kernel + attn_bwd_dq_x3_kernel", \
+            "10*D*H flops per kept (query, key) pair (fp32 products as three bf16 products)"
+    elif split_backward() or not tensor_cores:
         # dominant kernel: dK/dV, whose four GEMMs per kept pair (S^T, dP^T,
         # dV, dK) are all algorithmic work: 8*D flops per pair and head
         main_flops = 8.0 * w.head_dim * w.heads * pairs
@@ -430,7 +440,10 @@ def ours(args):
     achieved = main_flops / (dkdv_k * 1e-3) / 1e12 if dkdv_k > 0.0 else None
     bound, rpeak, peak_note = "tensor", peak, \
         f"{peak_src} bf16 sustained (kernel timed inside a long step)"
-    if not tensor_cores:
+    if split_fp32:
+        rpeak = peak / 3.0
+        peak_note = f"{peak_src} bf16 sustained / 3 (three bf16 products per fp32 product)"
+    elif not tensor_cores:
         # the CUDA-core kernels (fp32 arithmetic): bound by the FFMA pipes,
         # 128 fp32 lanes per SM, one fused multiply-add (2 flops) per lane
         # per clock, at the maximum SM clock the device reports

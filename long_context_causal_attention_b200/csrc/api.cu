@@ -73,8 +73,10 @@ static bool split_bwd() {
 }
 
 Path choose_bwd_path(const Problem& p) {
-  if (force_simt() || !tensor_core_shape(p) || !sm100_available()) return Path::kSimt;
-  return Path::kSm100;
+  if (force_simt() || !sm100_available()) return Path::kSimt;
+  if (tensor_core_shape(p)) return Path::kSm100;
+  if (x3_shape(p) && !fp32_simt()) return Path::kSm100X3;
+  return Path::kSimt;
 }
 
 size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
@@ -100,7 +102,8 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
   w.q_lo = static_cast<int32_t*>(take(tiles));
   w.k_hi = static_cast<int32_t*>(take(tiles));
   const size_t nel = (size_t)p.B * p.S * p.H * p.D;
-  if (!bwd && choose_fwd_path(p) == Path::kSm100X3) {
+  const bool x3 = bwd ? choose_bwd_path(p) == Path::kSm100X3 : choose_fwd_path(p) == Path::kSm100X3;
+  if (x3) {
     // split planes replace the rotated copies (the split pre-pass rotates)
     w.qx_hi = take(nel * 2);
     w.qx_lo = take(nel * 2);
@@ -108,11 +111,18 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
     w.kx_lo = take(nel * 2);
     w.vx_hi = take(nel * 2);
     w.vx_lo = take(nel * 2);
+    if (bwd) {
+      w.dox_hi = take(nel * 2);
+      w.dox_lo = take(nel * 2);
+      const size_t padded = (size_t)p.B * p.H * (size_t)p.n_tiles * kTile * sizeof(float);
+      w.lse2_pad = static_cast<float*>(take(padded));
+      w.delta_pad = static_cast<float*>(take(padded));
+    }
   } else if (p.theta > 0.0) {
     w.q_rot = take(nel * p.elt);
     w.k_rot = take(nel * p.elt);
   }
-  if (bwd) {
+  if (bwd && !x3) {
     w.delta = static_cast<float*>(take((size_t)p.B * p.H * p.S * sizeof(float)));
     if (tensor_core_shape(p)) {
       const size_t padded = (size_t)p.B * p.H * (size_t)p.n_tiles * kTile * sizeof(float);
@@ -282,9 +292,31 @@ lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   s = check_ws(p, true, ws, ws_bytes, &w);
   if (s != LWM_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = prologue(p, w, q, k, st);
+  const Path path = choose_bwd_path(p);
+  cudaError_t e;
+  if (path == Path::kSm100X3) {
+    e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
+    if (e == cudaSuccess) e = launch_segment_bounds(p, w, st);
+    const float* fq = static_cast<const float*>(q);
+    const float* fk = static_cast<const float*>(k);
+    if (e == cudaSuccess) e = launch_split(p.B, p.S, p.H, p.D, p.theta, fq, w.qx_hi, w.qx_lo, st);
+    if (e == cudaSuccess) e = launch_split(p.B, p.S, p.H, p.D, p.theta, fk, w.kx_hi, w.kx_lo, st);
+    if (e == cudaSuccess)
+      e = launch_split(p.B, p.S, p.H, p.D, 0.0, static_cast<const float*>(v), w.vx_hi, w.vx_lo, st);
+    if (e == cudaSuccess)
+      e = launch_split(p.B, p.S, p.H, p.D, 0.0, static_cast<const float*>(d_o), w.dox_hi, w.dox_lo,
+                       st);
+    if (e == cudaSuccess) e = launch_bwd_prep(p, o, d_o, lse, w, st);
+    if (e != cudaSuccess) return LWM_ERR_CUDA;
+    record_event(2, st);
+    e = launch_sm100_bwd_x3(p, w, dq, dk, dv, st);
+    record_event(4, st);
+    record_event(3, st);
+    return cuda_status(e);
+  }
+  e = prologue(p, w, q, k, st);
   if (e != cudaSuccess) return LWM_ERR_CUDA;
-  if (choose_bwd_path(p) == Path::kSm100) {
+  if (path == Path::kSm100) {
     e = launch_bwd_prep(p, o, d_o, lse, w, st);
     if (e == cudaSuccess && !split_bwd())
       e = cudaMemsetAsync(w.dq_acc, 0, fused_dq_acc_bytes(p.B, p.H, p.n_tiles), st);

@@ -47,6 +47,8 @@ struct Workspace {
   void* kx_lo;
   void* vx_hi;
   void* vx_lo;
+  void* dox_hi;        // and of dO (backward)
+  void* dox_lo;
   float* dec_ml;       // [B, H, T, n_chunks, 2] decode chunk max and sum (log2 domain)
   float* dec_o;        // [B, H, T, n_chunks, D] decode chunk sums of p * v
   size_t bytes;        // total bytes the layout needs
@@ -100,6 +102,10 @@ cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float
 
 cudaError_t launch_sm100_fwd(const Problem& p, const Workspace& ws, const void* v, void* o,
                              float* lse, cudaStream_t st);
+// fp32 backward on the tensor cores from the split planes in ws and the
+// padded LSE*log2(e) and dot(dO, O) (head_dim 64 or 128); dq, dk, dv fp32.
+cudaError_t launch_sm100_bwd_x3(const Problem& p, const Workspace& ws, void* dq, void* dk,
+                                void* dv, cudaStream_t st);
 // fp32 forward on the tensor cores from the split planes in ws (head_dim 64 or 128).
 cudaError_t launch_sm100_fwd_x3(const Problem& p, const Workspace& ws, float* o, float* lse,
                                 cudaStream_t st);

@@ -133,8 +133,9 @@ __global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, con
 //               past the end (so exp2(s - lse2) is exactly 0 there),
 //   dpad[row] = dot(dO, O), or 0 past the end.
 // One warp per padded row.
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
-                                                       const __nv_bfloat16* __restrict__ d_o,
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const T* __restrict__ o,
+                                                       const T* __restrict__ d_o,
                                                        const float* __restrict__ lse,
                                                        float* __restrict__ lse2,
                                                        float* __restrict__ dpad, int64_t n_rows,
@@ -228,9 +229,14 @@ cudaError_t launch_bwd_prep(const Problem& p, const void* o, const void* d_o, co
   const int64_t rows = p.B * p.H * s_pad;
   if (rows == 0) return cudaSuccess;
   const int64_t grid = (rows + 7) / 8;
-  bwd_prep_kernel<<<(unsigned)grid, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse,
-      ws.lse2_pad, ws.delta_pad, rows, p.S, s_pad, (int)p.H, (int)p.D);
+  if (p.dtype == LWM_DTYPE_BF16)
+    bwd_prep_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse,
+        ws.lse2_pad, ws.delta_pad, rows, p.S, s_pad, (int)p.H, (int)p.D);
+  else
+    bwd_prep_kernel<float><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const float*>(o), static_cast<const float*>(d_o), lse, ws.lse2_pad,
+        ws.delta_pad, rows, p.S, s_pad, (int)p.H, (int)p.D);
   note_launches(1);
   return cudaGetLastError();
 }
