@@ -119,8 +119,12 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
       w.delta_pad = static_cast<float*>(take(padded));
     }
   } else if (p.theta > 0.0) {
-    w.q_rot = take(nel * p.elt);
-    w.k_rot = take(nel * p.elt);
+    // rotated copies the chosen kernels read: the tensor-core forward rotates
+    // its Q tiles itself and the one-pass backward its K tiles
+    const Path path = bwd ? choose_bwd_path(p) : choose_fwd_path(p);
+    const bool one_pass = path == Path::kSm100 && (!bwd || !split_bwd());
+    if (!(one_pass && !bwd)) w.q_rot = take(nel * p.elt);
+    if (!(one_pass && bwd)) w.k_rot = take(nel * p.elt);
   }
   if (bwd && !x3) {
     w.delta = static_cast<float*>(take((size_t)p.B * p.H * p.S * sizeof(float)));
@@ -201,16 +205,17 @@ lwm_status check_ws(const Problem& p, bool bwd, void* ws, size_t ws_bytes, Works
 lwm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LWM_OK : LWM_ERR_CUDA; }
 
 // Shared front half of forward and backward: status word, segment bounds,
-// rotated q and k.
+// rotated q and k (those the workspace has room for: the kernels that rotate
+// a tile themselves read the un-rotated input).
 cudaError_t prologue(const Problem& p, Workspace& w, const void* q, const void* k, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
   if (e != cudaSuccess) return e;
   e = launch_segment_bounds(p, w, st);
   if (e != cudaSuccess) return e;
   if (p.theta > 0.0) {
-    e = launch_rope(p.B, p.S, p.H, p.D, p.dtype, p.theta, q, w.q_rot, 0, st);
-    if (e != cudaSuccess) return e;
-    e = launch_rope(p.B, p.S, p.H, p.D, p.dtype, p.theta, k, w.k_rot, 0, st);
+    if (w.q_rot) e = launch_rope(p.B, p.S, p.H, p.D, p.dtype, p.theta, q, w.q_rot, 0, st);
+    if (e == cudaSuccess && w.k_rot)
+      e = launch_rope(p.B, p.S, p.H, p.D, p.dtype, p.theta, k, w.k_rot, 0, st);
   } else {
     w.q_rot = const_cast<void*>(q);
     w.k_rot = const_cast<void*>(k);
@@ -268,7 +273,7 @@ lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   record_event(0, st);
   if (path == Path::kSm100)
-    e = launch_sm100_fwd(p, w, v, o, lse, st);
+    e = launch_sm100_fwd(p, w, q, v, o, lse, st);
   else
     e = launch_simt_fwd(p, w, v, o, lse, st);
   record_event(1, st);
@@ -327,7 +332,7 @@ lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
       record_event(4, st);
       if (e == cudaSuccess) e = launch_sm100_bwd_dq(p, w, v, d_o, dq, st);
     } else {
-      e = launch_sm100_bwd_fused(p, w, v, d_o, dq, dk, dv, st);
+      e = launch_sm100_bwd_fused(p, w, k, v, d_o, dq, dk, dv, st);
       record_event(4, st);
       if (e == cudaSuccess) e = launch_dq_finish(p, w, dq, st);
     }

@@ -18,7 +18,8 @@
 // accumulator in global memory with vector reductions (performed in L2); a
 // short kernel then scales it, applies the inverse rotation and writes bf16
 // dq.  Roles (576 threads):
-//   warp 0      TMA producer: K~_j, V_j once per item; per step Q~_i with the
+//   warp 0      TMA producer: K_j (un-rotated: the element-wise warps apply
+//               RoPE to it in shared memory), V_j once per item; per step Q~_i with the
 //               tile's LSE*log2(e) and D (2-stage ring) and dO_i (2-stage
 //               ring).
 //   warp 1      MMA issuer (one thread); the whole warp allocates and frees
@@ -95,7 +96,8 @@ enum : uint32_t {
   B_DQ_FULL = 16, B_DKV_FULL = 17, B_DKV_EMPTY = 18, B_FIN = 19,
   B_ITEM_FULL = 20,   // 4 slots
   B_ITEM_EMPTY = 24,  // 4 slots
-  B_COUNT = 28
+  B_K_ROT = 28,       // the element-wise warps rotated K~_j in place
+  B_COUNT = 29
 };
 static_assert(B_COUNT * 8 <= SOFF_MISC, "barrier slots");
 constexpr uint32_t kItemSlots = 4;
@@ -243,6 +245,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       mbar_init(bar(B_ITEM_FULL + sl), 1);
       mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kEWWarps);
     }
+    mbar_init(bar(B_K_ROT), kEWWarps);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -345,6 +348,8 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         int i = first_rel(p, it);
         if (i < 0) continue;
         if (!mbar_wait(bar(B_KV_FULL), kv_items & 1, ab, 76)) { ok = false; break; }
+        // K~_j arrives un-rotated: the element-wise warps rotate it in place
+        if (p.rotate && !mbar_wait(bar(B_K_ROT), kv_items & 1, ab, 108)) { ok = false; break; }
         ++kv_items;
         tc_fence_after();
         // X is free: the previous item's last dP^T was read before its dK
@@ -399,7 +404,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // 32w..32w+31 = 16-byte chunks 4(w&1)..4(w&1)+3 of box w>>1, swizzled
     const uint32_t sDSrow = base + OFF_DS + (uint32_t)(w >> 1) * kBoxBytes + (uint32_t)row * 128u;
     const uint32_t chunk0 = (uint32_t)(w & 1) * 4u, swz = (uint32_t)row & 7u;
-    uint32_t steps = 0, dkv = 0, dqc = 0;
+    uint32_t steps = 0, dkv = 0, dqc = 0, kv_items = 0;
     bool ok = true;
     for (uint32_t cons = 0; ok;) {
       const uint32_t sl = cons % kItemSlots;
@@ -418,6 +423,37 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int32_t seg_k = key_ok ? (p.seg ? p.kseg[(size_t)it.b * p.S + key] : 0) : -1;
       float* acc_bh = p.dq_acc + ((size_t)it.b * p.H + it.h) * (size_t)p.n_tiles * (128 * kD);
       int n = 0, dq_tile = -1;
+      if (p.rotate && first_rel(p, it) >= 0) {
+        // RoPE on this thread's 32 columns of key row `row` of K~_j, in place
+        // in shared memory (the producer loaded it un-rotated): pair (2i,
+        // 2i+1) turns by key * w_i, the angle reduced in fp64 and cos/sin from
+        // the fast approximation (absolute error below 1e-6, far under the
+        // bf16 rounding of the result)
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_KV_FULL), kv_items & 1, ab, 109))) {
+          ok = false;
+          break;
+        }
+        const uint32_t krow = base + OFF_K + (uint32_t)(w >> 1) * kBoxBytes + (uint32_t)row * 128u;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t a = krow + (((chunk0 + (uint32_t)c) ^ swz) << 4);
+          uint32_t v4[4];
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v4[0]), "=r"(v4[1]), "=r"(v4[2]), "=r"(v4[3]) : "r"(a));
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float cs, sn;
+            rope_cos_sin_fast(key, freq[16 * w + 4 * c + u], &cs, &sn);
+            const float x0 = __uint_as_float(v4[u] << 16), x1 = __uint_as_float(v4[u] & 0xffff0000u);
+            v4[u] = pack_bf16(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+          }
+          st_shared_v4(a, v4[0], v4[1], v4[2], v4[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_K_ROT));
+        ++kv_items;
+      }
       for (int i = it.lo; i <= it.hi; ++i) {
         if (!rel(p, it, i)) continue;
         const int64_t q0 = (int64_t)i * 128 + 32 * w;  // first query column of this quarter
@@ -739,11 +775,12 @@ size_t fused_dq_acc_bytes(int64_t B, int64_t H, int64_t n_tiles) {
   return (size_t)B * (size_t)H * (size_t)n_tiles * 128 * kD * sizeof(float);
 }
 
-cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const void* v,
-                                   const void* d_o, void* dq, void* dk, void* dv, cudaStream_t st) {
+cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const void* k,
+                                   const void* v, const void* d_o, void* dq, void* dk, void* dv,
+                                   cudaStream_t st) {
   CUtensorMap tq, tk, tv, tdo;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tk, k, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;

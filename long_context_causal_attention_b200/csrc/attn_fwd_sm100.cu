@@ -54,7 +54,8 @@ constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;     // K ring, 2 stages
 constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;     // V ring, 2 stages
 constexpr uint32_t OFF_BAR = OFF_V + 2 * kTileBytes;   // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;           // TMEM base, abort flag
-constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;  // + alignment slack
+constexpr uint32_t OFF_FREQ = OFF_MISC + 64;          // 64 RoPE frequencies, fp64
+constexpr uint32_t kSmemBytes = OFF_FREQ + 512 + 1024;  // + alignment slack
 
 // barrier slots (8 bytes each)
 enum : uint32_t {
@@ -70,8 +71,10 @@ enum : uint32_t {
   B_FIN = 18,
   B_ITEM_FULL = 19,   // 4 slots
   B_ITEM_EMPTY = 23,  // 4 slots
-  B_COUNT = 27
+  B_Q_ROT = 27,       // per tile: the softmax warps rotated Q_t in place
+  B_COUNT = 29
 };
+static_assert(B_COUNT * 8 <= 256, "barrier slots");
 constexpr uint32_t kItemSlots = 4;
 constexpr uint32_t kSoftmaxWarps = 8;
 
@@ -90,6 +93,8 @@ struct FwdParams {
   int H, B, n_tiles, n_pairs;
   float scale_log2;
   int causal;
+  int rotate;          // Q tiles arrive un-rotated: RoPE them in shared memory
+  double log2_theta;
 };
 
 struct Item {
@@ -203,11 +208,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(bar(B_ITEM_FULL + sl), 1);
       mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kSoftmaxWarps);
     }
+    mbar_init(bar(B_Q_ROT), kSoftmaxWarps / 2);
+    mbar_init(bar(B_Q_ROT + 1), kSoftmaxWarps / 2);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  double* freq = reinterpret_cast<double*>(smem + OFF_FREQ);
+  if (threadIdx.x >= 128 && threadIdx.x < 128 + kD / 2 && p.rotate)
+    freq[threadIdx.x - 128] = rope_freq(threadIdx.x - 128, kD, p.log2_theta);
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -287,7 +297,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
       constexpr uint32_t kIdPV = idesc_bf16(128, 128, 0, 1); // P (TMEM) x V (MN-major)
-      uint32_t k_it = 0, v_it = 0, p_cnt[2] = {0, 0}, act[2] = {0, 0};
+      uint32_t k_it = 0, v_it = 0, p_cnt[2] = {0, 0}, act[2] = {0, 0}, rot[2] = {0, 0};
       int items = 0;
       bool ok = true;
       const uint32_t sq0 = base + OFF_Q;
@@ -300,6 +310,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (idx >= n_items) break;
         const Item it = decode(p, idx);
         if (!mbar_wait(bar(B_Q_FULL), items & 1, ab, 4)) { ok = false; break; }
+        if (p.rotate) {  // and the softmax warps have rotated the tiles in place
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (it.qt[t] < 0) continue;
+            ok = mbar_wait(bar(B_Q_ROT + t), rot[t] & 1, ab, 24);
+            ++rot[t];
+          }
+          if (!ok) break;
+        }
         tc_fence_after();
         int jlo, jhi;
         union_range(it, &jlo, &jhi);
@@ -379,7 +397,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + (uint32_t)(t * 128);
     const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(t * 128);
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, q_items = 0;
     bool ok = true;
     for (uint32_t cons = 0; ok;) {
       const uint32_t sl = cons % kItemSlots;
@@ -393,8 +411,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ++cons;
       if (idx >= n_items) break;
       const Item it = decode(p, idx);
+      const uint32_t q_phase = q_items++ & 1;  // Q_FULL completes once per item
       if (it.qt[t] < 0) continue;
       const int64_t row = (int64_t)it.qt[t] * 128 + tid;
+      if (p.rotate) {
+        // RoPE on this row of the Q tile, in place in shared memory: pair
+        // (2i, 2i+1) turns by row * w_i, the angle reduced in fp64 and cos/sin
+        // from the fast approximation (absolute error below 1e-6, far under
+        // the bf16 rounding of the result)
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_Q_FULL), q_phase, ab, 25))) {
+          ok = false;
+          break;
+        }
+        const uint32_t qrow = base + OFF_Q + (uint32_t)t * kTileBytes + (uint32_t)tid * 128u;
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {  // 16-byte chunks: box c / 8, chunk c % 8
+          const uint32_t a = qrow + (uint32_t)(c >> 3) * kBoxBytes +
+                             ((((uint32_t)c & 7u) ^ ((uint32_t)tid & 7u)) << 4);
+          uint32_t w[4];
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(a));
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float cs, sn;
+            rope_cos_sin_fast(row, freq[4 * c + u], &cs, &sn);
+            const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+            w[u] = pack_bf16(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+          }
+          st_shared_v4(a, w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_Q_ROT + t));
+      }
       const bool row_ok = row < p.S;
       int32_t seg_row = row_ok ? (p.seg ? p.seg[(size_t)it.b * p.S + row] : 0) : -1;
       const size_t tok = (size_t)it.b * p.S + (size_t)(row_ok ? row : 0);
@@ -615,10 +664,10 @@ bool sm100_available() {
   return major == 10 && minor == 0 && encode_fn() != nullptr;
 }
 
-cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void* v, void* o,
-                             float* lse, cudaStream_t st) {
+cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void* q, const void* v,
+                             void* o, float* lse, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
-  if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
+  if (!make_qkv_map(&tq, q, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
@@ -640,6 +689,8 @@ cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void*
   p.n_pairs = (int)((pb.n_tiles + 1) / 2);
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.causal = pb.causal;
+  p.rotate = pb.theta > 0.0;
+  p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
   const int64_t n_items = pb.B * pb.H * p.n_pairs;
   if (n_items == 0) return cudaSuccess;
   static std::once_flag attr_once;

@@ -8,6 +8,7 @@ uses: in full where the oracle finishes in seconds, otherwise on sampled
 query rows (exact O/LSE/dQ per row) and on the last rows of sampled heads
 (exact dK/dV for the keys there).
 """
+import ctypes
 import math
 import zlib
 
@@ -245,3 +246,19 @@ def chunked_sum(x, chunk=65536):
     for s0 in range(0, x.shape[1], chunk):
         acc += x[:, s0:s0 + chunk].double().sum(1)
     return acc
+
+
+def test_workspace_holds_one_rotated_copy_per_pass(lwm):
+    """On the tensor-core path the forward rotates its Q tiles in shared
+    memory and the one-pass backward its K tiles, so each pass's workspace
+    holds one rotated copy (K~ for the forward, Q~ for the backward) instead
+    of two: the workspace with RoPE exceeds the one without by exactly one
+    tensor (up to the 1 KB alignment of its region)."""
+    q = torch.empty(1, 4096, 32, 128, dtype=torch.bfloat16, device="cuda")
+    nbytes = q.numel() * q.element_size()
+    for is_bwd in (False, True):
+        with_rope = lwm._lib.lib().lwm_attn_workspace_size(
+            ctypes.byref(lwm.make_desc(q, None, True, 1e6, 0.0)), int(is_bwd))
+        no_rope = lwm._lib.lib().lwm_attn_workspace_size(
+            ctypes.byref(lwm.make_desc(q, None, True, 0.0, 0.0)), int(is_bwd))
+        assert 0 <= with_rope - no_rope - nbytes < 1024, (is_bwd, with_rope, no_rope, nbytes)
