@@ -252,6 +252,23 @@ lwm_status lwm_attn_bwd_pair(const lwm_attn_desc* desc, const int32_t* k_segment
                              const float* lse, const void* d_o, void* dq, void* dk, void* dv,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* lwm_attn_fwd_pair_f32 / lwm_attn_bwd_pair_f32: the same block-pair
+ *   products with fp32 outputs (o, dq, dk, dv fp32 [B,S,H,D]) whatever the
+ *   input dtype, so the partial results of a ring are merged and summed
+ *   without a bf16 rounding per block (N blocks would otherwise add N
+ *   roundings).  Supported for fp32 inputs (identical to the pair calls) and
+ *   for bf16, head_dim 128 on sm_100 (the tensor-core kernels write fp32);
+ *   other shapes, or the two-kernel backward (LWM_ATTN_SPLIT_BWD=1), return
+ *   LWM_ERR_UNSUPPORTED before any launch.  Same workspace as the pair
+ *   calls. */
+lwm_status lwm_attn_fwd_pair_f32(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                                 const void* q, const void* k, const void* v, float* o, float* lse,
+                                 void* ws, size_t ws_bytes, void* stream);
+lwm_status lwm_attn_bwd_pair_f32(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                                 const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* d_o, float* dq, float* dk, float* dv,
+                                 void* ws, size_t ws_bytes, void* stream);
+
 lwm_status lwm_rope_apply_at(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
                              int32_t dtype, double theta, int64_t position_offset, const void* x,
                              void* y, int inverse, void* stream);

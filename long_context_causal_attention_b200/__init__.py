@@ -13,6 +13,7 @@ _EXPORTS = (
     "make_desc", "lwm_attn_selftest_wait", "lwm_rope_apply_at", "lwm_attn_merge",
     "lwm_accumulate", "lwm_convert_f32", "lwm_attn_fwd_pair", "lwm_attn_bwd_pair",
     "lwm_packed_cross_entropy", "lwm_attn_decode", "lwm_attn_decode_workspace_size", "DECODE_MAX_NEW",
+    "lwm_attn_fwd_pair_f32", "lwm_attn_bwd_pair_f32",
 )
 
 __all__ = list(_EXPORTS)

@@ -32,7 +32,8 @@ ENTRY_POINTS = ("lwm_attn_workspace_size", "lwm_attn_fwd", "lwm_attn_bwd", "lwm_
                 "lwm_attn_decode_workspace_size", "lwm_attn_decode", "lwm_attn_selftest_wait",
                 "lwm_rope_apply_at", "lwm_attn_merge", "lwm_accumulate", "lwm_convert_f32",
                 "lwm_attn_fwd_pair", "lwm_attn_bwd_pair", "lwm_packed_ce_workspace_size",
-                "lwm_packed_cross_entropy", "lwm_attn_fwd_noalloc_read_status")
+                "lwm_packed_cross_entropy", "lwm_attn_fwd_noalloc_read_status",
+                "lwm_attn_fwd_pair_f32", "lwm_attn_bwd_pair_f32")
 DECODE_MAX_NEW = 16
 
 
@@ -102,6 +103,10 @@ def _load():
     lib.lwm_attn_bwd_pair.argtypes = [ctypes.POINTER(LwmAttnDesc), P, P, P, P, P, P, P, P, P, P,
                                       P, ctypes.c_size_t, P]
     lib.lwm_attn_bwd_pair.restype = ctypes.c_int
+    lib.lwm_attn_fwd_pair_f32.argtypes = lib.lwm_attn_fwd_pair.argtypes
+    lib.lwm_attn_fwd_pair_f32.restype = ctypes.c_int
+    lib.lwm_attn_bwd_pair_f32.argtypes = lib.lwm_attn_bwd_pair.argtypes
+    lib.lwm_attn_bwd_pair_f32.restype = ctypes.c_int
     lib.lwm_rope_apply_at.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int32, ctypes.c_double,
                                       ctypes.c_int64, P, P, ctypes.c_int, P]
@@ -321,6 +326,45 @@ def lwm_attn_bwd_pair(q, k, v, o, lse, d_o, segment_ids, k_segment_ids, causal=T
                                   d_o.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                   workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "lwm_attn_bwd_pair")
+    return dq, dk, dv
+
+
+def lwm_attn_fwd_pair_f32(q, k, v, segment_ids, k_segment_ids, causal=True, rope_theta=1e4,
+                          softmax_scale=0.0, workspace=None, stream=None):
+    """lwm_attn_fwd_pair with an fp32 O whatever the input dtype (block
+    partials of a ring, merged without a bf16 rounding)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, name)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    desc = make_desc(q, segment_ids, causal, rope_theta, softmax_scale)
+    B, S, H, D = q.shape
+    o = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    workspace = alloc_workspace(desc, False, q.device) if workspace is None else workspace
+    _check(_lib.lwm_attn_fwd_pair_f32(ctypes.byref(desc), _kseg_ptr(k_segment_ids, q),
+                                      q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                      _stream(stream)), "lwm_attn_fwd_pair_f32")
+    return o, lse
+
+
+def lwm_attn_bwd_pair_f32(q, k, v, o, lse, d_o, segment_ids, k_segment_ids, causal=True,
+                          rope_theta=1e4, softmax_scale=0.0, workspace=None, stream=None):
+    """lwm_attn_bwd_pair with fp32 dq, dk, dv whatever the input dtype."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("d_o", d_o)):
+        _cuda(t, name)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    _cuda(lse, "lse")
+    desc = make_desc(q, segment_ids, causal, rope_theta, softmax_scale)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
+    workspace = alloc_workspace(desc, True, q.device) if workspace is None else workspace
+    _check(_lib.lwm_attn_bwd_pair_f32(ctypes.byref(desc), _kseg_ptr(k_segment_ids, q),
+                                      q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), d_o.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                      dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                      _stream(stream)), "lwm_attn_bwd_pair_f32")
     return dq, dk, dv
 
 

@@ -236,9 +236,11 @@ lwm_status set_key_segments(Problem* p, const int32_t* k_segment_ids) {
   return LWM_OK;
 }
 
+// out_f32: the outputs are fp32 whatever the input dtype (block partials of
+// a ring); supported on the fp32 paths and the tensor-core bf16 path.
 lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_ids,
                     const void* q, const void* k, const void* v, void* o, float* lse, void* ws,
-                    size_t ws_bytes, void* stream) {
+                    size_t ws_bytes, void* stream, bool out_f32 = false) {
   Problem p{};
   lwm_status s = make_problem(desc, &p);
   if (s != LWM_OK) return s;
@@ -252,6 +254,8 @@ lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   if (s != LWM_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Path path = choose_fwd_path(p);
+  const bool f32_out = out_f32 && p.dtype == LWM_DTYPE_BF16;
+  if (f32_out && path != Path::kSm100) return LWM_ERR_UNSUPPORTED;
   cudaError_t e;
   if (path == Path::kSm100X3) {
     e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
@@ -273,7 +277,7 @@ lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   if (e != cudaSuccess) return LWM_ERR_CUDA;
   record_event(0, st);
   if (path == Path::kSm100)
-    e = launch_sm100_fwd(p, w, q, v, o, lse, st);
+    e = launch_sm100_fwd(p, w, q, v, o, lse, st, f32_out);
   else
     e = launch_simt_fwd(p, w, v, o, lse, st);
   record_event(1, st);
@@ -283,7 +287,7 @@ lwm_status attn_fwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
 lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_ids,
                     const void* q, const void* k, const void* v, const void* o, const float* lse,
                     const void* d_o, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
-                    void* stream) {
+                    void* stream, bool out_f32 = false) {
   Problem p{};
   lwm_status s = make_problem(desc, &p);
   if (s != LWM_OK) return s;
@@ -298,6 +302,8 @@ lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
   if (s != LWM_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Path path = choose_bwd_path(p);
+  const bool f32_out = out_f32 && p.dtype == LWM_DTYPE_BF16;
+  if (f32_out && (path != Path::kSm100 || split_bwd())) return LWM_ERR_UNSUPPORTED;
   cudaError_t e;
   if (path == Path::kSm100X3) {
     e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st);
@@ -332,9 +338,9 @@ lwm_status attn_bwd(const lwm_attn_desc* desc, const int32_t* const* k_segment_i
       record_event(4, st);
       if (e == cudaSuccess) e = launch_sm100_bwd_dq(p, w, v, d_o, dq, st);
     } else {
-      e = launch_sm100_bwd_fused(p, w, k, v, d_o, dq, dk, dv, st);
+      e = launch_sm100_bwd_fused(p, w, k, v, d_o, dq, dk, dv, st, f32_out);
       record_event(4, st);
-      if (e == cudaSuccess) e = launch_dq_finish(p, w, dq, st);
+      if (e == cudaSuccess) e = launch_dq_finish(p, w, dq, st, f32_out);
     }
     record_event(3, st);
     return cuda_status(e);
@@ -385,6 +391,20 @@ lwm_status lwm_attn_bwd_pair(const lwm_attn_desc* desc, const int32_t* k_segment
                              const float* lse, const void* d_o, void* dq, void* dk, void* dv,
                              void* ws, size_t ws_bytes, void* stream) {
   return attn_bwd(desc, &k_segment_ids, q, k, v, o, lse, d_o, dq, dk, dv, ws, ws_bytes, stream);
+}
+
+lwm_status lwm_attn_fwd_pair_f32(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                                 const void* q, const void* k, const void* v, float* o, float* lse,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return attn_fwd(desc, &k_segment_ids, q, k, v, o, lse, ws, ws_bytes, stream, true);
+}
+
+lwm_status lwm_attn_bwd_pair_f32(const lwm_attn_desc* desc, const int32_t* k_segment_ids,
+                                 const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* d_o, float* dq, float* dk, float* dv,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return attn_bwd(desc, &k_segment_ids, q, k, v, o, lse, d_o, dq, dk, dv, ws, ws_bytes, stream,
+                  true);
 }
 
 size_t lwm_attn_decode_workspace_size(const lwm_attn_desc* desc, int64_t n_new) {

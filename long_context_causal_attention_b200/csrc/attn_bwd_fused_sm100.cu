@@ -116,6 +116,8 @@ struct FusedParams {
   float* dq_acc;         // [B*H, nT, 32, 128, 4]: unscaled dQ~ partial sums (zeroed)
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dk32;           // non-null: dK, dV written in fp32 here instead (block partials)
+  float* dv32;
   DeviceStatus* status;
   int64_t S;
   int H, B, n_tiles;
@@ -645,15 +647,22 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
       }
       // ---- dK, dV epilogue for this key tile (this quarter's 32 columns) ----
-      __nv_bfloat16* dkrow = p.dk + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 32 * w;
-      __nv_bfloat16* dvrow = p.dv + (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 32 * w;
+      const size_t orow_off = (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 32 * w;
       if (n == 0) {
         if (key_ok) {
           const uint4 z = make_uint4(0, 0, 0, 0);
+          if (p.dk32) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            reinterpret_cast<uint4*>(dkrow)[c] = z;
-            reinterpret_cast<uint4*>(dvrow)[c] = z;
+            for (int c = 0; c < 8; ++c) {
+              reinterpret_cast<uint4*>(p.dk32 + orow_off)[c] = z;
+              reinterpret_cast<uint4*>(p.dv32 + orow_off)[c] = z;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              reinterpret_cast<uint4*>(p.dk + orow_off)[c] = z;
+              reinterpret_cast<uint4*>(p.dv + orow_off)[c] = z;
+            }
           }
         }
         continue;
@@ -661,20 +670,30 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DKV_FULL), dkv & 1, ab, 104 + w))) { ok = false; break; }
       ++dkv;
       tc_fence_after();
-      uint32_t out[16];
+      // 32 fp32 values of a row out: bf16 pairs, or fp32 for block partials
+      auto store_row = [&](__nv_bfloat16* dst16, float* dst32, const float (&x)[32]) {
+        if (!key_ok) return;
+        if (dst32) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            reinterpret_cast<float4*>(dst32)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(x[2 * u], x[2 * u + 1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            reinterpret_cast<uint4*>(dst16)[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+      };
       {
         uint32_t r[32];
         tmem_ld32(tDV, r);
         tmem_wait_ld();
+        float x[32];
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          out[u] = pack_bf16(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
-      }
-      if (key_ok) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          reinterpret_cast<uint4*>(dvrow)[c] =
-              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        for (int u = 0; u < 32; ++u) x[u] = __uint_as_float(r[u]);
+        store_row(p.dv + orow_off, p.dv32 ? p.dv32 + orow_off : nullptr, x);
       }
       {
         uint32_t r[32];
@@ -683,6 +702,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_DKV_EMPTY));
+        float x[32];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           float a = __uint_as_float(r[2 * u]) * p.scale, b = __uint_as_float(r[2 * u + 1]) * p.scale;
@@ -693,14 +713,10 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             a = a2;
             b = b2;
           }
-          out[u] = pack_bf16(a, b);
+          x[2 * u] = a;
+          x[2 * u + 1] = b;
         }
-      }
-      if (key_ok) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          reinterpret_cast<uint4*>(dkrow)[c] =
-              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        store_row(p.dk + orow_off, p.dk32 ? p.dk32 + orow_off : nullptr, x);
       }
     }
   }
@@ -732,8 +748,8 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // (b, h, query tile), one thread per row.  Reads of a column group are 512
 // contiguous bytes per warp; each thread writes its row's 256 bytes.
 __global__ void __launch_bounds__(128)
-dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int64_t S, int H,
-                 int n_tiles, float scale, int rotate, double log2_theta) {
+dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, float* __restrict__ dq32,
+                 int64_t S, int H, int n_tiles, float scale, int rotate, double log2_theta) {
   __shared__ double freq[kD / 2];
   if (threadIdx.x < kD / 2 && rotate) freq[threadIdx.x] = rope_freq(threadIdx.x, kD, log2_theta);
   __syncthreads();
@@ -745,6 +761,7 @@ dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, 
   const int64_t b = bh / H, h = bh % H;
   const float4* src = reinterpret_cast<const float4*>(acc + (size_t)blockIdx.x * (128 * kD)) + row;
   uint4* dst = reinterpret_cast<uint4*>(dq + (((size_t)b * S + q) * H + h) * kD);
+  float4* dst32 = reinterpret_cast<float4*>(dq32 + (((size_t)b * S + q) * H + h) * kD);
 #pragma unroll 4
   for (int m = 0; m < kD / 8; ++m) {  // 8 columns: column groups 2m, 2m+1
     uint32_t pk[4];
@@ -762,10 +779,11 @@ dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, 
           x[2 * u + 1] = bb * c - a * s;
         }
       }
+      if (dq32) dst32[2 * m + g] = make_float4(x[0], x[1], x[2], x[3]);
       pk[2 * g] = pack_bf16(x[0], x[1]);
       pk[2 * g + 1] = pack_bf16(x[2], x[3]);
     }
-    dst[m] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    if (!dq32) dst[m] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
 }
 
@@ -777,7 +795,7 @@ size_t fused_dq_acc_bytes(int64_t B, int64_t H, int64_t n_tiles) {
 
 cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const void* k,
                                    const void* v, const void* d_o, void* dq, void* dk, void* dv,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, bool out_f32) {
   CUtensorMap tq, tk, tv, tdo;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, k, pb.B, pb.S, pb.H, pb.D) ||
@@ -797,8 +815,10 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
   p.lse2 = ws.lse2_pad;
   p.dpad = ws.delta_pad;
   p.dq_acc = ws.dq_acc;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk = out_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
+  p.dv = out_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
+  p.dk32 = out_f32 ? static_cast<float*>(dk) : nullptr;
+  p.dv32 = out_f32 ? static_cast<float*>(dv) : nullptr;
   p.status = ws.status;
   p.S = pb.S;
   p.H = (int)pb.H;
@@ -822,13 +842,15 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
   return cudaGetLastError();
 }
 
-cudaError_t launch_dq_finish(const Problem& pb, const Workspace& ws, void* dq, cudaStream_t st) {
+cudaError_t launch_dq_finish(const Problem& pb, const Workspace& ws, void* dq, cudaStream_t st,
+                             bool out_f32) {
   const int64_t blocks = pb.B * pb.H * pb.n_tiles;
   if (blocks == 0) return cudaSuccess;
   const int rotate = pb.theta > 0.0;
-  dq_finish_kernel<<<(unsigned)blocks, 128, 0, st>>>(ws.dq_acc, static_cast<__nv_bfloat16*>(dq),
-                                                      pb.S, (int)pb.H, (int)pb.n_tiles, pb.scale,
-                                                      rotate, rotate ? log2(pb.theta) : 0.0);
+  dq_finish_kernel<<<(unsigned)blocks, 128, 0, st>>>(
+      ws.dq_acc, out_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq),
+      out_f32 ? static_cast<float*>(dq) : nullptr, pb.S, (int)pb.H, (int)pb.n_tiles, pb.scale,
+      rotate, rotate ? log2(pb.theta) : 0.0);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -87,6 +87,7 @@ struct FwdParams {
   const int32_t* ktmax;
   const int32_t* q_lo;
   __nv_bfloat16* o;
+  float* o32;          // non-null: O is written in fp32 here instead (block partials of a ring)
   float* lse;
   DeviceStatus* status;
   int64_t S;
@@ -546,11 +547,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       if (!ok) break;
       __nv_bfloat16* orow = p.o + (tok * p.H + it.h) * kD;
+      float* orow32 = p.o32 + (tok * p.H + it.h) * kD;
       if (ntiles == 0) {
         if (row_ok) {
           const uint4 z = make_uint4(0, 0, 0, 0);
+          if (p.o32) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+            for (int c = 0; c < 32; ++c) reinterpret_cast<uint4*>(orow32)[c] = z;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+          }
           p.lse[((size_t)it.b * p.H + it.h) * p.S + row] = -INFINITY;
         }
         continue;
@@ -567,7 +574,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t r[32];
         tmem_ld32(tO + c * 32, r);
         tmem_wait_ld();
-        if (row_ok) {
+        if (row_ok && p.o32) {
+          float4* dst = reinterpret_cast<float4*>(orow32 + c * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            dst[u] = make_float4(__uint_as_float(r[4 * u]) * inv, __uint_as_float(r[4 * u + 1]) * inv,
+                                 __uint_as_float(r[4 * u + 2]) * inv, __uint_as_float(r[4 * u + 3]) * inv);
+        } else if (row_ok) {
           uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u)
@@ -665,7 +678,7 @@ bool sm100_available() {
 }
 
 cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void* q, const void* v,
-                             void* o, float* lse, cudaStream_t st) {
+                             void* o, float* lse, cudaStream_t st, bool o_f32) {
   CUtensorMap tq, tk, tv;
   if (!make_qkv_map(&tq, q, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
@@ -679,7 +692,8 @@ cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void*
   p.ktmin = ws.ktile_min;
   p.ktmax = ws.ktile_max;
   p.q_lo = ws.q_lo;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o);
+  p.o32 = o_f32 ? static_cast<float*>(o) : nullptr;
   p.lse = lse;
   p.status = ws.status;
   p.S = pb.S;

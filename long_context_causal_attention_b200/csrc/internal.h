@@ -101,8 +101,9 @@ cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float
                          cudaStream_t st);
 
 // q un-rotated (the kernel applies RoPE to its Q tiles), k rotated in ws.k_rot.
+// o_f32: O written as fp32 (block partials a ring merges) instead of bf16.
 cudaError_t launch_sm100_fwd(const Problem& p, const Workspace& ws, const void* q, const void* v,
-                             void* o, float* lse, cudaStream_t st);
+                             void* o, float* lse, cudaStream_t st, bool o_f32 = false);
 // fp32 backward on the tensor cores from the split planes in ws and the
 // padded LSE*log2(e) and dot(dO, O) (head_dim 64 or 128); dq, dk, dv fp32.
 cudaError_t launch_sm100_bwd_x3(const Problem& p, const Workspace& ws, void* dq, void* dk,
@@ -123,8 +124,9 @@ size_t fused_dq_acc_bytes(int64_t B, int64_t H, int64_t n_tiles);
 // k un-rotated (the kernel applies RoPE to its K tiles), q rotated in ws.q_rot.
 cudaError_t launch_sm100_bwd_fused(const Problem& p, const Workspace& ws, const void* k,
                                    const void* v, const void* d_o, void* dq, void* dk, void* dv,
-                                   cudaStream_t st);
-cudaError_t launch_dq_finish(const Problem& p, const Workspace& ws, void* dq, cudaStream_t st);
+                                   cudaStream_t st, bool out_f32 = false);
+cudaError_t launch_dq_finish(const Problem& p, const Workspace& ws, void* dq, cudaStream_t st,
+                             bool out_f32 = false);
 
 // Bounded-wait self-test: one CTA waits on an mbarrier (armed by an arrival
 // or not) for at most limit_cycles; a wait that runs out records

@@ -16,8 +16,11 @@ same work on every rank).
 Backward: every rank computes, for each visiting key/value block, the
 contributions to its own dq and to the visitor's dk and dv (FlashAttention
 recomputation with the GLOBAL log-sum-exp and D = dO . O, so block
-contributions simply add); the visitor's dk/dv accumulators travel with it
-and are home after N shifts.
+contributions simply add); the visitor's dk/dv sums travel after it and are
+home after N shifts.  The next key/value block is sent before the current
+one is computed, so only the sums wait for the step's compute.  Block
+results are fp32 where the library writes them so, so the merge and the
+sums carry no per-block bf16 rounding.
 
 Each step of the arithmetic runs in the library's CUDA kernels
 (lwm_rope_apply_at, lwm_attn_fwd / lwm_attn_bwd on rotated inputs,
@@ -39,17 +42,38 @@ from . import _lib as L
 
 
 class GpuBlockOps:
-    """Per-block operations of the ring, on the library's kernels."""
+    """Per-block operations of the ring, on the library's kernels.  Block
+    results come back in fp32 where the library can write them so (fp32
+    inputs; bf16 at head_dim 128 on the tensor cores), so the merge and the
+    gradient sums see no per-block bf16 rounding; other shapes fall back to
+    results in the input dtype."""
+
+    def __init__(self):
+        self.f32 = True
 
     def rotate(self, x, theta, pos0, inverse=False):
         return L.lwm_rope_apply_at(x, theta, pos0, inverse)
 
+    def _try_f32(self, f32_call, call):
+        if self.f32:
+            try:
+                return f32_call()
+            except L.LwmError as e:
+                if e.status != -2:  # anything but LWM_ERR_UNSUPPORTED is an error
+                    raise
+                self.f32 = False
+        return call()
+
     def block_fwd(self, q, k, v, causal, scale, q_seg=None, k_seg=None):
         # inputs are rotated already: rope_theta = 0
-        return L.lwm_attn_fwd_pair(q, k, v, q_seg, k_seg, causal, 0.0, scale)
+        return self._try_f32(
+            lambda: L.lwm_attn_fwd_pair_f32(q, k, v, q_seg, k_seg, causal, 0.0, scale),
+            lambda: L.lwm_attn_fwd_pair(q, k, v, q_seg, k_seg, causal, 0.0, scale))
 
     def block_bwd(self, q, k, v, o, lse, d_o, causal, scale, q_seg=None, k_seg=None):
-        return L.lwm_attn_bwd_pair(q, k, v, o, lse, d_o, q_seg, k_seg, causal, 0.0, scale)
+        return self._try_f32(
+            lambda: L.lwm_attn_bwd_pair_f32(q, k, v, o, lse, d_o, q_seg, k_seg, causal, 0.0, scale),
+            lambda: L.lwm_attn_bwd_pair(q, k, v, o, lse, d_o, q_seg, k_seg, causal, 0.0, scale))
 
     def merge(self, o_acc, lse_acc, o_part, lse_part):
         L.lwm_attn_merge(o_acc, lse_acc, o_part, lse_part)
@@ -157,29 +181,42 @@ def _backward_steps(rank, size, q, k, v, o, lse, d_o, theta, scale, ops, layout,
     os_, dos, lses = cut(o), cut(d_o), cut(lse, 2)
     qseg = cut(seg) if seg is not None else [None] * c
     dq_acc = [ops.zeros_f32((B, n, H, D), q.device) for _ in ids]
-    # the travelling block: rotated keys, values, their gradient sums (and the
-    # keys' segment ids)
+    # the travelling block: rotated keys, values (and the keys' segment ids);
+    # its gradient sums travel as a second message, sent once this rank has
+    # added its contributions
     blk = [ops.rotate(x, theta, g * n) for x, g in zip(cut(k), ids)] + cut(v)
-    blk += [ops.zeros_f32((B, n, H, D), q.device) for _ in range(2 * c)]
     if seg is not None:
         blk += qseg
+    sums = [ops.zeros_f32((B, n, H, D), q.device) for _ in range(2 * c)]
+    sums_h = None
     for s in range(size):
         src = (rank - s) % size
+        # the next block is in flight while this one is computed
+        kv_h = (yield ("start", blk)) if s < size - 1 else None
+        parts = []
         for a, b, causal in _pairs(ids, chunk_ids(src, size, layout)):
-            kseg = blk[4 * c + b] if seg is not None else None
+            kseg = blk[2 * c + b] if seg is not None else None
             dq_p, dk_p, dv_p = ops.block_bwd(qr[a], blk[b], blk[c + b], os_[a], lses[a], dos[a],
                                              causal, scale, qseg[a], kseg)
             ops.accumulate(dq_acc[a], dq_p)
-            ops.accumulate(blk[2 * c + b], dk_p)
-            ops.accumulate(blk[3 * c + b], dv_p)
-        # N shifts in all: after the last one every block is home with its sums
-        h = yield ("start", blk)
-        blk = yield ("wait", h)
+            parts.append((b, dk_p, dv_p))
+        # the visiting block's sums, from the previous rank after its own step
+        if s > 0:
+            sums = yield ("wait", sums_h)
+        for b, dk_p, dv_p in parts:
+            ops.accumulate(sums[b], dk_p)
+            ops.accumulate(sums[c + b], dv_p)
+        # N shifts of the sums in all: after the last one every block's sums
+        # are home
+        sums_h = yield ("start", sums)
+        if s < size - 1:
+            blk = yield ("wait", kv_h)
+    sums = yield ("wait", sums_h)
     dq = torch.cat([ops.convert(ops.rotate(x, theta, g * n, inverse=True), q.dtype)
                     for x, g in zip(dq_acc, ids)], dim=1)
-    dk = torch.cat([ops.convert(ops.rotate(blk[2 * c + b], theta, g * n, inverse=True), k.dtype)
+    dk = torch.cat([ops.convert(ops.rotate(sums[b], theta, g * n, inverse=True), k.dtype)
                     for b, g in enumerate(ids)], dim=1)
-    dv = torch.cat([ops.convert(blk[3 * c + b], v.dtype) for b in range(c)], dim=1)
+    dv = torch.cat([ops.convert(sums[c + b], v.dtype) for b in range(c)], dim=1)
     return dq, dk, dv
 
 
@@ -211,32 +248,33 @@ def _run_distributed(gen, group):
 
 
 def _run_emulated(gens):
-    """Step N per-rank generators in lockstep; a shift rotates the blocks."""
+    """Step N per-rank generators in lockstep, one operation at a time (every
+    rank runs the same sequence of starts and waits); a start records each
+    rank's payload under a new handle, a wait hands every rank the payload
+    its previous rank started under that handle (a shift of the ring)."""
     size = len(gens)
     msgs = [None] * size
     results = [None] * size
+    in_flight, next_handle = {}, 0
     while True:
-        outgoing = [None] * size
-        active = 0
+        ops_ = []
         for r, g in enumerate(gens):
-            if results[r] is not None:
-                continue
             try:
-                kind, payload = g.send(msgs[r])
+                ops_.append(g.send(msgs[r]))
             except StopIteration as done:
                 results[r] = done.value
-                continue
-            assert kind == "start"
-            outgoing[r] = payload
-            active += 1
-        if active == 0:
+                ops_.append(None)
+        if all(o is None for o in ops_):
             return results
-        if active != size:
+        if any(o is None for o in ops_) or len({o[0] for o in ops_}) != 1:
             raise RuntimeError("ring ranks fell out of step")
-        for r, g in enumerate(gens):
-            kind, handle = g.send(r)  # the handle is just the rank index
-            assert kind == "wait"
-        msgs = [outgoing[(r - 1) % size] for r in range(size)]
+        if ops_[0][0] == "start":
+            in_flight[next_handle] = [o[1] for o in ops_]
+            msgs = [next_handle] * size
+            next_handle += 1
+        else:
+            sent = in_flight.pop(ops_[0][1])
+            msgs = [sent[(r - 1) % size] for r in range(size)]
 
 
 def ring_forward(q, k, v, rope_theta=1e4, softmax_scale=0.0, group=None, ops=None,

@@ -18,7 +18,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("n_ranks,n,theta,layout", [(4, 256, 1e6, "zigzag"), (3, 384, 1e7, "contiguous"),
-                                                   (2, 200, 1e4, "zigzag"), (4, 128, 1e6, "contiguous")])
+                                                   (2, 200, 1e4, "zigzag"), (4, 128, 1e6, "contiguous"),
+                                                   (8, 128, 1e6, "zigzag"), (8, 256, 1e7, "contiguous")])
 def test_emulated_ring_matches_oracle(n_ranks, n, theta, layout):
     from long_context_causal_attention_b200 import ring
     B, H, D = 1, 4, 128
@@ -106,3 +107,28 @@ def test_merge_kernel_equals_joint_softmax():
     ref_o = np.einsum("bhst,bthd->bshd", e / e.sum(-1, keepdims=True), V)
     assert_close("o", to64(o_acc), ref_o, "bf16")
     assert_close("lse", to64(l_acc), ref_l, "bf16")
+
+
+def test_fp32_block_results_are_the_bf16_ones_unrounded():
+    """The fp32-output pair calls return what the bf16 pair calls round: each
+    bf16 result lies within half a bf16 ulp of the fp32 one (2^-9 relative;
+    2^-8 allowed, since dq's fp32 partial sums are added in an order that
+    differs between launches), for the forward O and the backward dq, dk,
+    dv."""
+    import long_context_causal_attention_b200 as lwm
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    B, S, H, D = 1, 300, 2, 128
+    q, k, v, do = (torch.randn((B, S, H, D), generator=g, device="cuda").to(torch.bfloat16)
+                   for _ in range(4))
+    o16, lse16 = lwm.lwm_attn_fwd_pair(q, k, v, None, None, True, 0.0)
+    o32, lse32 = lwm.lwm_attn_fwd_pair_f32(q, k, v, None, None, True, 0.0)
+    g16 = lwm.lwm_attn_bwd_pair(q, k, v, o16, lse16, do, None, None, True, 0.0)
+    g32 = lwm.lwm_attn_bwd_pair_f32(q, k, v, o16, lse16, do, None, None, True, 0.0)
+    torch.cuda.synchronize()
+    assert o32.dtype == torch.float32 and torch.equal(lse16, lse32)
+    for a16, a32 in zip((o16,) + tuple(g16), (o32,) + tuple(g32)):
+        assert a32.dtype == torch.float32
+        ref = a16.float()
+        assert bool(((a32 - ref).abs() <= ref.abs() * 2.0 ** -8 + 1e-6).all())
+        assert not torch.equal(a32, ref)  # the fp32 results are not rounded
