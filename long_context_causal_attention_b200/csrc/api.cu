@@ -122,9 +122,9 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
     // rotated copies the chosen kernels read: the tensor-core forward rotates
     // its Q tiles itself and the one-pass backward its K tiles
     const Path path = bwd ? choose_bwd_path(p) : choose_fwd_path(p);
-    const bool one_pass = path == Path::kSm100 && (!bwd || !split_bwd());
-    if (!(one_pass && !bwd)) w.q_rot = take(nel * p.elt);
-    if (!(one_pass && bwd)) w.k_rot = take(nel * p.elt);
+    const bool on_load = path == Path::kSm100 && (!bwd || !split_bwd()) && rope_on_load(p);
+    if (!(on_load && !bwd)) w.q_rot = take(nel * p.elt);
+    if (!(on_load && bwd)) w.k_rot = take(nel * p.elt);
   }
   if (bwd && !x3) {
     w.delta = static_cast<float*>(take((size_t)p.B * p.H * p.S * sizeof(float)));

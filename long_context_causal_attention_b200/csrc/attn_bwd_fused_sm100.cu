@@ -122,7 +122,8 @@ struct FusedParams {
   int64_t S;
   int H, B, n_tiles;
   float scale, scale_log2;
-  int causal, rotate;
+  int causal, rotate;    // rotate: RoPE on (inverse rotation of dK, dQ)
+  int rot_k;             // K_j arrives un-rotated: RoPE it in shared memory
   double log2_theta;
 };
 
@@ -351,7 +352,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (i < 0) continue;
         if (!mbar_wait(bar(B_KV_FULL), kv_items & 1, ab, 76)) { ok = false; break; }
         // K~_j arrives un-rotated: the element-wise warps rotate it in place
-        if (p.rotate && !mbar_wait(bar(B_K_ROT), kv_items & 1, ab, 108)) { ok = false; break; }
+        if (p.rot_k && !mbar_wait(bar(B_K_ROT), kv_items & 1, ab, 108)) { ok = false; break; }
         ++kv_items;
         tc_fence_after();
         // X is free: the previous item's last dP^T was read before its dK
@@ -425,7 +426,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int32_t seg_k = key_ok ? (p.seg ? p.kseg[(size_t)it.b * p.S + key] : 0) : -1;
       float* acc_bh = p.dq_acc + ((size_t)it.b * p.H + it.h) * (size_t)p.n_tiles * (128 * kD);
       int n = 0, dq_tile = -1;
-      if (p.rotate && first_rel(p, it) >= 0) {
+      if (p.rot_k && first_rel(p, it) >= 0) {
         // RoPE on this thread's 32 columns of key row `row` of K~_j, in place
         // in shared memory (the producer loaded it un-rotated): pair (2i,
         // 2i+1) turns by key * w_i, the angle reduced in fp64 and cos/sin from
@@ -744,46 +745,50 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   }
 }
 
-// dq = R(p)^T (scale * dQ~) in bf16, from the fp32 accumulator: one CTA per
-// (b, h, query tile), one thread per row.  Reads of a column group are 512
-// contiguous bytes per warp; each thread writes its row's 256 bytes.
+// dq = R(p)^T (scale * dQ~) in bf16 (or fp32), from the fp32 accumulator:
+// one CTA per (b, h, query tile).  The 64 KB tile ([32 column groups][128
+// rows][4]) comes in with fully coalesced 16-byte loads and is transposed
+// through shared memory (rows padded by 4 floats: conflict-free 16-byte
+// stores); then each warp writes whole rows, lane l holding columns 4l..4l+3,
+// so a row's 256 (or 512) bytes leave in one contiguous store.
+constexpr int kFinRow = kD + 4;  // padded shared-memory row, floats
 __global__ void __launch_bounds__(128)
 dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, float* __restrict__ dq32,
                  int64_t S, int H, int n_tiles, float scale, int rotate, double log2_theta) {
+  extern __shared__ float tile[];  // [128][kFinRow]
   __shared__ double freq[kD / 2];
   if (threadIdx.x < kD / 2 && rotate) freq[threadIdx.x] = rope_freq(threadIdx.x, kD, log2_theta);
+  const float4* src = reinterpret_cast<const float4*>(acc + (size_t)blockIdx.x * (128 * kD));
+#pragma unroll 8
+  for (int k = 0; k < 32; ++k) {
+    const int i = threadIdx.x + 128 * k;  // float4 index: column group i / 128, row i % 128
+    *reinterpret_cast<float4*>(&tile[(i & 127) * kFinRow + (i >> 7) * 4]) = src[i];
+  }
   __syncthreads();
-  const int tile = blockIdx.x % n_tiles;
+  const int tile_i = blockIdx.x % n_tiles;
   const int64_t bh = blockIdx.x / n_tiles;
-  const int row = threadIdx.x;
-  const int64_t q = (int64_t)tile * 128 + row;
-  if (q >= S) return;
   const int64_t b = bh / H, h = bh % H;
-  const float4* src = reinterpret_cast<const float4*>(acc + (size_t)blockIdx.x * (128 * kD)) + row;
-  uint4* dst = reinterpret_cast<uint4*>(dq + (((size_t)b * S + q) * H + h) * kD);
-  float4* dst32 = reinterpret_cast<float4*>(dq32 + (((size_t)b * S + q) * H + h) * kD);
-#pragma unroll 4
-  for (int m = 0; m < kD / 8; ++m) {  // 8 columns: column groups 2m, 2m+1
-    uint32_t pk[4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < 128; r += 4) {
+    const int64_t q = (int64_t)tile_i * 128 + r;
+    if (q >= S) break;
+    const float4 v = *reinterpret_cast<const float4*>(&tile[r * kFinRow + 4 * lane]);
+    float x[4] = {v.x * scale, v.y * scale, v.z * scale, v.w * scale};
+    if (rotate) {
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const float4 v = src[(size_t)(2 * m + g) * 128];
-      float x[4] = {v.x * scale, v.y * scale, v.z * scale, v.w * scale};
-      if (rotate) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          float c, s;
-          rope_cos_sin_fast(q, freq[4 * m + 2 * g + u], &c, &s);
-          const float a = x[2 * u], bb = x[2 * u + 1];
-          x[2 * u] = a * c + bb * s;
-          x[2 * u + 1] = bb * c - a * s;
-        }
+      for (int u = 0; u < 2; ++u) {
+        float c, sn;
+        rope_cos_sin_fast(q, freq[2 * lane + u], &c, &sn);
+        const float a = x[2 * u], bb = x[2 * u + 1];
+        x[2 * u] = a * c + bb * sn;
+        x[2 * u + 1] = bb * c - a * sn;
       }
-      if (dq32) dst32[2 * m + g] = make_float4(x[0], x[1], x[2], x[3]);
-      pk[2 * g] = pack_bf16(x[0], x[1]);
-      pk[2 * g + 1] = pack_bf16(x[2], x[3]);
     }
-    if (!dq32) dst[m] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    const size_t off = (((size_t)b * S + q) * H + h) * kD + 4 * lane;
+    if (dq32)
+      *reinterpret_cast<float4*>(dq32 + off) = make_float4(x[0], x[1], x[2], x[3]);
+    else
+      *reinterpret_cast<uint2*>(dq + off) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
   }
 }
 
@@ -798,7 +803,7 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
                                    cudaStream_t st, bool out_f32) {
   CUtensorMap tq, tk, tv, tdo;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tk, k, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tk, rope_on_load(pb) ? k : ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
@@ -828,6 +833,7 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.causal = pb.causal;
   p.rotate = pb.theta > 0.0;
+  p.rot_k = rope_on_load(pb);
   p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -847,7 +853,15 @@ cudaError_t launch_dq_finish(const Problem& pb, const Workspace& ws, void* dq, c
   const int64_t blocks = pb.B * pb.H * pb.n_tiles;
   if (blocks == 0) return cudaSuccess;
   const int rotate = pb.theta > 0.0;
-  dq_finish_kernel<<<(unsigned)blocks, 128, 0, st>>>(
+  constexpr int kFinSmem = 128 * kFinRow * (int)sizeof(float);
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(dq_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kFinSmem);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  dq_finish_kernel<<<(unsigned)blocks, 128, kFinSmem, st>>>(
       ws.dq_acc, out_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq),
       out_f32 ? static_cast<float*>(dq) : nullptr, pb.S, (int)pb.H, (int)pb.n_tiles, pb.scale,
       rotate, rotate ? log2(pb.theta) : 0.0);

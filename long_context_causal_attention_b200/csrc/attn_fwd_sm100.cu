@@ -680,7 +680,8 @@ bool sm100_available() {
 cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void* q, const void* v,
                              void* o, float* lse, cudaStream_t st, bool o_f32) {
   CUtensorMap tq, tk, tv;
-  if (!make_qkv_map(&tq, q, pb.B, pb.S, pb.H, pb.D) ||
+  const bool rot_q = rope_on_load(pb);  // else the workspace holds the rotated q
+  if (!make_qkv_map(&tq, rot_q ? q : ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
@@ -703,7 +704,7 @@ cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void*
   p.n_pairs = (int)((pb.n_tiles + 1) / 2);
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.causal = pb.causal;
-  p.rotate = pb.theta > 0.0;
+  p.rotate = rot_q;
   p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
   const int64_t n_items = pb.B * pb.H * p.n_pairs;
   if (n_items == 0) return cudaSuccess;

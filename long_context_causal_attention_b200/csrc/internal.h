@@ -57,6 +57,14 @@ struct Workspace {
 // kSm100X3: fp32 data on the bf16 tensor cores through hi/lo splits.
 enum class Path { kSimt = 0, kSm100 = 1, kSm100X3 = 2 };
 
+// RoPE applied by the tensor-core kernels to their stationary tiles in
+// shared memory (Q in the forward, K in the one-pass backward) instead of a
+// rotated copy in the workspace: from 64K tokens on, where the copy is large;
+// below, the copy is small and the rotation would lengthen every short work
+// item.
+constexpr int64_t kRopeOnLoadMinS = 65536;
+inline bool rope_on_load(const Problem& p) { return p.theta > 0.0 && p.S >= kRopeOnLoadMinS; }
+
 // Which kernels serve the forward / backward of this problem on this device.
 Path choose_fwd_path(const Problem& p);
 Path choose_bwd_path(const Problem& p);

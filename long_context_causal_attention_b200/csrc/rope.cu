@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, con
 //   lse2[row] = LSE * log2(e), or +inf when the row has no allowed key or is
 //               past the end (so exp2(s - lse2) is exactly 0 there),
 //   dpad[row] = dot(dO, O), or 0 past the end.
-// One warp per padded row.
+// A group of D / V lanes per row, V elements (16 bytes) per lane, so each row
+// of O and of dO is one contiguous load per group; 32 / (D / V) rows per warp.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const T* __restrict__ o,
                                                        const T* __restrict__ d_o,
@@ -140,21 +141,29 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const T* __restrict__ o,
                                                        float* __restrict__ lse2,
                                                        float* __restrict__ dpad, int64_t n_rows,
                                                        int64_t S, int64_t S_pad, int H, int D) {
+  constexpr int V = 16 / sizeof(T);
+  const int per_row = D / V;              // lanes per row: 4..32, a power of two
   const int lane = threadIdx.x & 31;
-  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (r >= n_rows) return;  // r = (b * H + h) * S_pad + s
+  const int sub = lane % per_row;
+  const int64_t r = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (32 / per_row) +
+                    lane / per_row;  // r = (b * H + h) * S_pad + s
   const int64_t s = r % S_pad, bh = r / S_pad;
   const int64_t b = bh / H, h = bh % H;
+  const bool live = r < n_rows && s < S;
   float acc = 0.f, L2 = INFINITY;
-  if (s < S) {
-    const size_t off = (((size_t)b * S + s) * H + h) * D;
-    for (int d = lane; d < D; d += 32) acc += to_f32(o[off + d]) * to_f32(d_o[off + d]);
+  if (live) {
+    const size_t off = (((size_t)b * S + s) * H + h) * D + (size_t)sub * V;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 g = *reinterpret_cast<const uint4*>(d_o + off);
+    const T* ea = reinterpret_cast<const T*>(&a);
+    const T* eg = reinterpret_cast<const T*>(&g);
 #pragma unroll
-    for (int k = 16; k > 0; k >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
+    for (int e = 0; e < V; ++e) acc += to_f32(ea[e]) * to_f32(eg[e]);
     const float L = lse[(size_t)bh * S + s];
     L2 = L == -INFINITY ? INFINITY : L * 1.4426950408889634f;
   }
-  if (lane == 0) {
+  for (int k = per_row >> 1; k > 0; k >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
+  if (r < n_rows && sub == 0) {
     lse2[r] = L2;
     dpad[r] = acc;
   }
@@ -228,7 +237,8 @@ cudaError_t launch_bwd_prep(const Problem& p, const void* o, const void* d_o, co
   const int64_t s_pad = p.n_tiles * kTile;
   const int64_t rows = p.B * p.H * s_pad;
   if (rows == 0) return cudaSuccess;
-  const int64_t grid = (rows + 7) / 8;
+  const int64_t rows_per_warp = 32 / (p.D / (p.dtype == LWM_DTYPE_BF16 ? 8 : 4));
+  const int64_t grid = (rows + 8 * rows_per_warp - 1) / (8 * rows_per_warp);
   if (p.dtype == LWM_DTYPE_BF16)
     bwd_prep_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse,

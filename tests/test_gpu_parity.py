@@ -249,16 +249,17 @@ def chunked_sum(x, chunk=65536):
 
 
 def test_workspace_holds_one_rotated_copy_per_pass(lwm):
-    """On the tensor-core path the forward rotates its Q tiles in shared
-    memory and the one-pass backward its K tiles, so each pass's workspace
-    holds one rotated copy (K~ for the forward, Q~ for the backward) instead
-    of two: the workspace with RoPE exceeds the one without by exactly one
-    tensor (up to the 1 KB alignment of its region)."""
-    q = torch.empty(1, 4096, 32, 128, dtype=torch.bfloat16, device="cuda")
-    nbytes = q.numel() * q.element_size()
-    for is_bwd in (False, True):
-        with_rope = lwm._lib.lib().lwm_attn_workspace_size(
-            ctypes.byref(lwm.make_desc(q, None, True, 1e6, 0.0)), int(is_bwd))
-        no_rope = lwm._lib.lib().lwm_attn_workspace_size(
-            ctypes.byref(lwm.make_desc(q, None, True, 0.0, 0.0)), int(is_bwd))
-        assert 0 <= with_rope - no_rope - nbytes < 1024, (is_bwd, with_rope, no_rope, nbytes)
+    """From 64K tokens on, the tensor-core forward rotates its Q tiles in
+    shared memory and the one-pass backward its K tiles, so each pass's
+    workspace holds one rotated copy (K~ for the forward, Q~ for the
+    backward): the workspace with RoPE exceeds the one without by one tensor
+    (up to the 1 KB alignment of its region).  Shorter sequences keep both
+    copies (the rotation would lengthen every short work item)."""
+    lib = lwm._lib.lib()
+    for S, copies in ((65536, 1), (1 << 20, 1), (4096, 2)):
+        nbytes = S * 32 * 128 * 2
+        for is_bwd in (False, True):
+            size = lambda theta: lib.lwm_attn_workspace_size(
+                ctypes.byref(lwm.LwmAttnDesc(1, S, 32, 128, 0, 1, theta, 0.0, None)), int(is_bwd))
+            extra = size(1e6) - size(0.0)
+            assert 0 <= extra - copies * nbytes < 1024 * copies, (S, is_bwd, extra, nbytes)

@@ -64,7 +64,8 @@ WORKLOADS = {
     # decode step: n_new new tokens, the cache of `seqlen` tokens includes them
     "decode_1m": Workload("decode_1m", 1, 1048576, 32, 128, "bf16", 5e7, backward=False,
                           extra={"n_new": 1}),
-    # fp32 end to end (the pages train in fp32): the CUDA-core path at 8K tokens
+    # fp32 end to end (the pages train in fp32) at 8K tokens: the split-precision
+    # tensor-core path (LWM_ATTN_FP32_SIMT=1: the CUDA-core kernels)
     "fp32_8k": Workload("fp32_8k", 1, 8192, 32, 128, "fp32", 1e6),
     # packed loss re-weighting: the packed_8k rows, LLaMA vocabulary (32000)
     "packed_loss_8k": Workload("packed_loss_8k", 4, 8192, 32, 128, "bf16", 1e6,
