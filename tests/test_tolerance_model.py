@@ -39,3 +39,54 @@ def test_rotated_operand_rounding_fits_bounds(sigma, S, tol):
         d = np.abs(mod[key] - ref[key])
         # leave room for the outputs' own bf16 rounding on top of the model
         assert d.max() <= 0.75 * mx and d.mean() <= 0.75 * mean, (key, d.max(), d.mean())
+
+
+def _split(a):
+    """bf16 hi plane and bf16 lo plane of an fp32 operand, as the split
+    pre-pass and the kernels' register splits form them."""
+    hi = _bf16(np.asarray(a, np.float32))
+    lo = _bf16(np.asarray(a, np.float64) - hi)
+    return hi, lo
+
+
+def _mm3(a, b):
+    """a @ b as the split-precision kernels form it: hi*hi + hi*lo + lo*hi
+    in float64 (the fp32 accumulation adds far less)."""
+    ah, al = _split(a)
+    bh, bl = _split(b)
+    return ah @ bh + ah @ bl + al @ bh
+
+
+@pytest.mark.parametrize("S,D,sigma,bound", [(256, 64, 1.0, 1e-4), (1024, 128, 1.0, 1e-4),
+                                             (1024, 128, 2.0, 1e-3)])
+def test_split_precision_products_fit_the_fp32_bound(S, D, sigma, bound):
+    """fp32 attention with every product taken as three bf16 products of
+    split operands (rotated q, k and v split; P and dS split before their
+    products), against float64: the errors stay inside the fp32 bound at
+    the fp32 workloads' sigma = 1 (they measure ~2e-5); sharper inputs
+    (sigma = 2) need the looser bound, which is why full fp32 arithmetic
+    stays available."""
+    rng = np.random.default_rng(3)
+    q, k, v, do = (rng.standard_normal((S, D)).astype(np.float32) * s
+                   for s in (sigma, sigma, 1.0, 1.0))
+    scale = 1.0 / np.sqrt(D)
+    mask = np.tril(np.ones((S, S), bool))
+
+    def run(mm):
+        s = np.where(mask, mm(q, k.T) * scale, -np.inf)
+        m = s.max(1, keepdims=True)
+        p = np.exp(s - m)
+        lse = (m + np.log(p.sum(1, keepdims=True)))[:, 0]
+        p = p / p.sum(1, keepdims=True)
+        o = mm(p, v)
+        dp = mm(do, v.T)
+        ds = p * (dp - (do.astype(np.float64) * o).sum(1, keepdims=True))
+        return {"o": o, "lse": lse, "dq": mm(ds, k) * scale, "dk": mm(ds.T, q) * scale,
+                "dv": mm(p.T, do)}
+
+    exact = run(lambda a, b: np.asarray(a, np.float64) @ np.asarray(b, np.float64))
+    split = run(_mm3)
+    worst = max(float(np.abs(split[key] - exact[key]).max()) for key in exact)
+    assert worst <= bound, worst
+    if sigma == 1.0:
+        assert worst <= bound / 3, worst  # a margin for the device's own fp32 rounding
