@@ -122,7 +122,8 @@ size_t layout_workspace(const Problem& p, bool bwd, void* base, Workspace* ws) {
     // rotated copies the chosen kernels read: the tensor-core forward rotates
     // its Q tiles itself and the one-pass backward its K tiles
     const Path path = bwd ? choose_bwd_path(p) : choose_fwd_path(p);
-    const bool on_load = path == Path::kSm100 && (!bwd || !split_bwd()) && rope_on_load(p);
+    const bool on_load = path == Path::kSm100 &&
+                         (bwd ? !split_bwd() && rope_on_load_bwd(p) : rope_on_load_fwd(p));
     if (!(on_load && !bwd)) w.q_rot = take(nel * p.elt);
     if (!(on_load && bwd)) w.k_rot = take(nel * p.elt);
   }

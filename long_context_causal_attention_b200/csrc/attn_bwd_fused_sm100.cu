@@ -49,10 +49,6 @@
 #include "internal.h"
 #include "sm100.cuh"
 
-#ifndef LWM_RED_SPREAD
-#define LWM_RED_SPREAD 0
-#endif
-
 namespace lwm {
 
 bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
@@ -495,59 +491,6 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         tc_fence_after();
         float pr[32];
-#if LWM_RED_SPREAD
-        {
-          uint32_t r[32];
-          tmem_ld32(tX, r);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_S_READ));  // dP^T(i) may overwrite X now
-          // the previous step's dQ partial out of Y (same lanes/columns); its
-          // eight vector reductions are spread over the exponentials
-          uint32_t dqv[32];
-          const bool drain = dq_tile >= 0;
-          float* dst = nullptr;
-          if (drain) {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), dqc & 1, ab, 92 + w))) { ok = false; break; }
-            ++dqc;
-            tc_fence_after();
-            tmem_ld32(tY, dqv);
-            tmem_wait_ld();
-            dst = acc_bh + (size_t)dq_tile * (128 * kD) + ((size_t)(8 * w) * 128 + row) * 4;
-            dq_tile = -1;
-          }
-          const float4* l4 = reinterpret_cast<const float4*>(lse2);
-          if (partial) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float4 L = l4[u];
-              const float Ls[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int c = 4 * u + e;
-                pr[c] = ((mw >> c) & 1u) ? fast_exp2(fmaf(__uint_as_float(r[c]), p.scale_log2, -Ls[e]))
-                                         : 0.f;
-              }
-              if (drain)
-                red_add_v4(dst + (size_t)u * 512, __uint_as_float(dqv[4 * u]), __uint_as_float(dqv[4 * u + 1]),
-                           __uint_as_float(dqv[4 * u + 2]), __uint_as_float(dqv[4 * u + 3]));
-            }
-          } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float4 L = l4[u];
-              const float Ls[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                pr[4 * u + e] = fast_exp2(fmaf(__uint_as_float(r[4 * u + e]), p.scale_log2, -Ls[e]));
-              if (drain)
-                red_add_v4(dst + (size_t)u * 512, __uint_as_float(dqv[4 * u]), __uint_as_float(dqv[4 * u + 1]),
-                           __uint_as_float(dqv[4 * u + 2]), __uint_as_float(dqv[4 * u + 3]));
-            }
-          }
-        }
-#else
         {
           uint32_t r[32];
           tmem_ld32(tX, r);
@@ -587,7 +530,6 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           drain_dq(tY, acc_bh + (size_t)dq_tile * (128 * kD), row, w);
           dq_tile = -1;
         }
-#endif
         // ---- P^T (bf16) into the first 16 columns of this quarter of Y ----
         {
           uint32_t pk[16];
@@ -803,7 +745,7 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
                                    cudaStream_t st, bool out_f32) {
   CUtensorMap tq, tk, tv, tdo;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
-      !make_qkv_map(&tk, rope_on_load(pb) ? k : ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
+      !make_qkv_map(&tk, rope_on_load_bwd(pb) ? k : ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tdo, d_o, pb.B, pb.S, pb.H, pb.D))
     return cudaErrorInvalidValue;
@@ -833,7 +775,7 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.causal = pb.causal;
   p.rotate = pb.theta > 0.0;
-  p.rot_k = rope_on_load(pb);
+  p.rot_k = rope_on_load_bwd(pb);
   p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;

@@ -680,7 +680,7 @@ bool sm100_available() {
 cudaError_t launch_sm100_fwd(const Problem& pb, const Workspace& ws, const void* q, const void* v,
                              void* o, float* lse, cudaStream_t st, bool o_f32) {
   CUtensorMap tq, tk, tv;
-  const bool rot_q = rope_on_load(pb);  // else the workspace holds the rotated q
+  const bool rot_q = rope_on_load_fwd(pb);  // else the workspace holds the rotated q
   if (!make_qkv_map(&tq, rot_q ? q : ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D))
