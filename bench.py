@@ -63,8 +63,8 @@ def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
 # The same for the one-pass backward kernel (attn_bwd_fused_kernel), from a
 # one-pass capture of the full-size 128K launch (profiles/
 # attn_bwd_fused_traffic_long_128k.md).
-FUSED_TRAFFIC = {"bytes": {"long_128k": 14.53e9 + 8.59e9},
-                 "source_sha256": "f8e36b7d58c794409fc35cd65e0a0610830a745d28e1e870250d4b681414c4b0"}
+FUSED_TRAFFIC = {"bytes": {"long_128k": 14.82e9 + 8.81e9},
+                 "source_sha256": "5fd22d1b8eeecfcaec4ea269951036564e770e4d3f6ec43762440492fae9d706"}
 
 
 def split_backward() -> bool:

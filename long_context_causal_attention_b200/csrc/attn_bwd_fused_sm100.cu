@@ -13,34 +13,35 @@
 //
 // One persistent CTA per SM owns a key tile j (128 keys) of one (b, h) and
 // walks the query tiles i that may attend to it; dK_j and dV_j accumulate in
-// tensor memory for the whole walk.  The dQ~_i partial of each step is read
-// out of tensor memory by the element-wise warps and added into an fp32
-// accumulator in global memory with vector reductions (performed in L2); a
-// short kernel then scales it, applies the inverse rotation and writes bf16
-// dq.  Roles (576 threads):
+// tensor memory for the whole walk.  The dQ~_i partial of each step is
+// computed in two 64-column halves; dedicated reducer warps read each half
+// out of tensor memory and add it into an fp32 accumulator in global memory
+// with vector reductions (performed in L2), so the element-wise chain never
+// waits on the L2 reduction path; a short kernel then scales the
+// accumulator, applies the inverse rotation and writes dq.  Roles (704
+// threads):
 //   warp 0      TMA producer: K_j (un-rotated: the element-wise warps apply
-//               RoPE to it in shared memory), V_j once per item; per step Q~_i with the
-//               tile's LSE*log2(e) and D (2-stage ring) and dO_i (2-stage
-//               ring).
+//               RoPE to it in shared memory), V_j once per item; per step Q~_i
+//               with the tile's LSE*log2(e) and D (2-stage ring) and dO_i
+//               (2-stage ring).
 //   warp 1      MMA issuer (one thread); the whole warp allocates and frees
 //               the tensor memory.
-//   warps 2-17  element-wise work, four groups of four warps (one per TMEM
-//               lane quarter, warp % 4) on 32 columns each: P^T and dS^T
-//               (bf16) into tensor memory, dS into a shared-memory tile, the
-//               dQ partial out to global memory, then the dK/dV epilogue.
+//   warps 4-19  element-wise work, four groups of four warps (one per TMEM
+//               lane quarter, warp % 4) on 32 columns each: P^T (bf16) into
+//               tensor memory, dS into a shared-memory tile, then the dK/dV
+//               epilogue.
+//   warps 2, 3, 20, 21  dQ reducers, one per TMEM lane quarter.
 // TMEM columns:
 //   X  [0,128)    S^T(i), then dP^T(i) once S^T(i) is in registers
-//   Y  [128,256)  per 32-column quarter: P^T(i) in the first 16 columns and
-//                 dS^T(i) in the last 16 (bf16 pairs); then the dQ(i)
-//                 partial (fp32, lanes = queries) once dV(i) and dK(i) have
-//                 read them
+//   P  [128,192)  P^T(i), bf16 pairs (A operand of dV)
+//   R  [192,256)  one 64-column half of the dQ~(i) partial (lanes = queries)
 //   dV [256,384), dK [384,512)
-// Each element-wise warp reads and writes only its own lane quarter and
-// 32-column slice of Y, so draining dQ(i-1) and writing P^T(i) need no
-// barrier between warps.
+// dS lives only in the shared tile: K-major it is the A operand of dK, MN-
+// major the A operand of both dQ halves.
 // MMA issue order per step:
-//   dP^T(i) once S^T(i) is read | dV(i) after P(i) | S^T(i+1) once dP^T(i)
-//   is read | dK(i) after dS(i) | dQ(i) into Y
+//   dP^T(i) once S^T(i) is read | dQ(i-1) second half once R is read |
+//   dV(i) after P(i) | S^T(i+1) once dP^T(i) is read | dK(i) after dS(i) |
+//   dQ(i) first half once R is read
 #include <cuda.h>
 
 #include <mutex>
@@ -59,8 +60,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 576;   // 2 control warps + 4 element-wise warpgroups
+constexpr int kThreads = 704;   // TMA, MMA, 4 dQ reducer warps, 16 element-wise warps
 constexpr int kEW = 512;        // element-wise threads
+constexpr int kReducers = 4;    // dQ reducer warps, one per TMEM lane quarter
 constexpr uint32_t kTileBytes = 128 * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;
 
@@ -89,11 +91,13 @@ enum : uint32_t {
   B_DO_FULL = 6,   // 2 stages
   B_DO_EMPTY = 8,  // 2 stages
   B_S_FULL = 10, B_S_READ = 11, B_DP_FULL = 12, B_DP_READ = 13, B_P_FULL = 14, B_DS_FULL = 15,
-  B_DQ_FULL = 16, B_DKV_FULL = 17, B_DKV_EMPTY = 18, B_FIN = 19,
+  B_DQA_FULL = 16, B_DKV_FULL = 17, B_DKV_EMPTY = 18, B_FIN = 19,
   B_ITEM_FULL = 20,   // 4 slots
   B_ITEM_EMPTY = 24,  // 4 slots
   B_K_ROT = 28,       // the element-wise warps rotated K~_j in place
-  B_COUNT = 29
+  B_DQB_FULL = 29,    // second dQ half done: R holds it, and the dS tile is free
+  B_R_EMPTY = 30,     // the reducer warps read R
+  B_COUNT = 31
 };
 static_assert(B_COUNT * 8 <= SOFF_MISC, "barrier slots");
 constexpr uint32_t kItemSlots = 4;
@@ -177,22 +181,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// The dQ partial of one step, read out of tensor memory (Y) by one element-
-// wise warp -- TMEM lanes 32*(warp%4).. = query rows, its 32 columns -- and
-// added into the accumulator tile: [32 column groups][128 rows][4] floats,
-// so each of the eight vector reductions of a warp covers 512 contiguous
-// bytes.
-__device__ __forceinline__ void drain_dq(uint32_t tY, float* acc_tile, int row, int w) {
-  uint32_t r[32];
-  tmem_ld32(tY, r);
-  tmem_wait_ld();
-  float* dst = acc_tile + ((size_t)(8 * w) * 128 + row) * 4;
-#pragma unroll
-  for (int g = 0; g < 8; ++g)
-    red_add_v4(dst + (size_t)g * 512, __uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-               __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -236,13 +224,15 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     mbar_init(bar(B_DP_READ), kEWWarps);
     mbar_init(bar(B_P_FULL), kEWWarps);
     mbar_init(bar(B_DS_FULL), kEWWarps);
-    mbar_init(bar(B_DQ_FULL), 1);
+    mbar_init(bar(B_DQA_FULL), 1);
+    mbar_init(bar(B_DQB_FULL), 1);
+    mbar_init(bar(B_R_EMPTY), kReducers);
     mbar_init(bar(B_DKV_FULL), 1);
     mbar_init(bar(B_DKV_EMPTY), kEWWarps);
     mbar_init(bar(B_FIN), 1);
     for (uint32_t sl = 0; sl < kItemSlots; ++sl) {
       mbar_init(bar(B_ITEM_FULL + sl), 1);
-      mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kEWWarps);
+      mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kEWWarps + kReducers);
     }
     mbar_init(bar(B_K_ROT), kEWWarps);
     fence_mbar_init();
@@ -319,14 +309,14 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);   // K-major x K-major
-      constexpr uint32_t kIdKM = idesc_bf16(128, 128, 0, 1);   // TMEM (K-major) x MN-major
-      constexpr uint32_t kIdMM = idesc_bf16(128, 128, 1, 1);   // MN-major x MN-major
+      constexpr uint32_t kIdKM = idesc_bf16(128, 128, 0, 1);   // K-major (TMEM or smem) x MN-major
+      constexpr uint32_t kIdMM = idesc_bf16(128, 64, 1, 1);    // MN-major x MN-major, N = 64
       const uint32_t sK = base + OFF_K, sV = base + OFF_V;
-      const uint32_t tX = tmem, tY = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
-      uint32_t q_it = 0, do_it = 0, steps = 0, dkv = 0, kv_items = 0;
+      const uint32_t tX = tmem, tP = tmem + 128, tR = tmem + 192, tDV = tmem + 256, tDK = tmem + 384;
+      uint32_t q_it = 0, do_it = 0, steps = 0, dkv = 0, kv_items = 0, halves = 0;
       bool ok = true;
       const uint64_t dK = kmajor_desc(sK), dV = kmajor_desc(sV);
-      const uint64_t dKmn = mnmajor_desc(sK), dDSmn = mnmajor_desc(base + OFF_DS);
+      const uint64_t dDSk = kmajor_desc(base + OFF_DS), dDSmn = mnmajor_desc(base + OFF_DS);
       auto sq_of = [&](uint32_t n) { return base + OFF_Q + (n & 1) * kTileBytes; };
       auto sdo_of = [&](uint32_t n) { return base + OFF_DO + (n & 1) * kTileBytes; };
       auto issue_s = [&](uint32_t n) -> bool {
@@ -334,6 +324,16 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_after();
         mma_kk128(tX, dK, kmajor_desc(sq_of(n)), kIdKK, 0u);
         mma_commit(bar(B_S_FULL));
+        return true;
+      };
+      // half h of dQ~(i) = dS(i) K~ (D columns 64h..64h+63) into R, once the
+      // reducer warps have read the previous half out of it
+      auto issue_half = [&](uint32_t h) -> bool {
+        if (halves > 0 && !mbar_wait(bar(B_R_EMPTY), (halves - 1) & 1, ab, 110)) return false;
+        tc_fence_after();
+        mma_mm128(tR, dDSmn, mnmajor_desc(sK + h * kBoxBytes), kIdMM, 0u);
+        mma_commit(bar(h ? B_DQB_FULL : B_DQA_FULL));
+        ++halves;
         return true;
       };
       for (uint32_t cons = 0; ok;) {
@@ -353,7 +353,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_after();
         // X is free: the previous item's last dP^T was read before its dK
         if (!issue_s(q_it)) { ok = false; break; }
-        bool first = true;
+        bool first = true, pend_b = false;
         while (i >= 0) {
           // dP^T(i) into X once S^T(i) is in registers
           if (!mbar_wait(bar(B_S_READ), steps & 1, ab, 77)) { ok = false; break; }
@@ -361,49 +361,54 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tc_fence_after();
           mma_kk128(tX, dV, kmajor_desc(sdo_of(do_it)), kIdKK, 0u);
           mma_commit(bar(B_DP_FULL));
-          // dV(i) += P^T dO  (P^T from Y)
+          // the previous step's second dQ half, behind dP^T(i) in the pipe
+          if (pend_b && !issue_half(1)) { ok = false; break; }
+          pend_b = false;
+          // dV(i) += P^T dO  (P^T from TMEM)
           if (first && dkv > 0 && !mbar_wait(bar(B_DKV_EMPTY), (dkv - 1) & 1, ab, 79)) { ok = false; break; }
           if (!mbar_wait(bar(B_P_FULL), steps & 1, ab, 80)) { ok = false; break; }
           tc_fence_after();
-          mma_tm128<true>(tDV, tY, mnmajor_desc(sdo_of(do_it)), kIdKM, first ? 0u : 1u);
+          mma_tm128<false>(tDV, tP, mnmajor_desc(sdo_of(do_it)), kIdKM, first ? 0u : 1u);
           mma_commit(bar(B_DO_EMPTY + (do_it & 1)));
           ++do_it;
           // S^T(next) into X once dP^T(i) is in registers
           const int inext = next_rel(p, it, i);
           if (!mbar_wait(bar(B_DP_READ), steps & 1, ab, 81)) { ok = false; break; }
           if (inext >= 0 && !issue_s(q_it + 1)) { ok = false; break; }
-          // dK(i) += dS^T Q~ (dS^T from Y), then dQ(i) = dS K~ into Y
+          // dK(i) += dS^T Q~ (dS^T: the shared dS tile read K-major), then the
+          // first dQ half (the same tile read MN-major)
           if (!mbar_wait(bar(B_DS_FULL), steps & 1, ab, 82)) { ok = false; break; }
           tc_fence_after();
-          mma_tm128<true>(tDK, tY + 16u, mnmajor_desc(sq_of(q_it)), kIdKM, first ? 0u : 1u);
+          mma_km128(tDK, dDSk, mnmajor_desc(sq_of(q_it)), kIdKM, first ? 0u : 1u);
           mma_commit(bar(B_Q_EMPTY + (q_it & 1)));
-          mma_mm128(tY, dDSmn, dKmn, kIdMM, 0u);
-          mma_commit(bar(B_DQ_FULL));
+          if (!issue_half(0)) { ok = false; break; }
+          pend_b = true;
           ++q_it;
           ++steps;
           first = false;
           i = inext;
         }
         if (!ok) break;
+        if (pend_b && !issue_half(1)) { ok = false; break; }
         mma_commit(bar(B_DKV_FULL));
         ++dkv;
-        mma_commit(bar(B_KV_EMPTY));
+        mma_commit(bar(B_KV_EMPTY));  // K~_j (read by the last dQ half) and V_j are free
       }
     }
-  } else {
+  } else if (warp >= 4 && warp < 4 + kEWWarps) {
     // ------------------------------------------------- element-wise work
-    const int w = (warp - 2) >> 2;                // column quarter
-    const int row = ((warp & 3) << 5) + lane;     // TMEM lane: key (S^T, dP^T, dV, dK) or query (dQ)
+    const int w = (warp - 4) >> 2;                // column quarter
+    const int row = ((warp & 3) << 5) + lane;     // TMEM lane = key
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tX = tmem + lane_base + 32u * w;
-    const uint32_t tY = tmem + lane_base + 128u + 32u * w;
+    const uint32_t tP = tmem + lane_base + 128u + 16u * w;
     const uint32_t tDV = tmem + lane_base + 256u + 32u * w;
     const uint32_t tDK = tmem + lane_base + 384u + 32u * w;
     // this thread's 64 bytes of the dS tile: key row `row`, query columns
     // 32w..32w+31 = 16-byte chunks 4(w&1)..4(w&1)+3 of box w>>1, swizzled
     const uint32_t sDSrow = base + OFF_DS + (uint32_t)(w >> 1) * kBoxBytes + (uint32_t)row * 128u;
     const uint32_t chunk0 = (uint32_t)(w & 1) * 4u, swz = (uint32_t)row & 7u;
-    uint32_t steps = 0, dkv = 0, dqc = 0, kv_items = 0;
+    uint32_t steps = 0, dkv = 0, kv_items = 0;
     bool ok = true;
     for (uint32_t cons = 0; ok;) {
       const uint32_t sl = cons % kItemSlots;
@@ -420,8 +425,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int64_t key = (int64_t)it.j * 128 + row;
       const bool key_ok = key < p.S;
       const int32_t seg_k = key_ok ? (p.seg ? p.kseg[(size_t)it.b * p.S + key] : 0) : -1;
-      float* acc_bh = p.dq_acc + ((size_t)it.b * p.H + it.h) * (size_t)p.n_tiles * (128 * kD);
-      int n = 0, dq_tile = -1;
+      int n = 0;
       if (p.rot_k && first_rel(p, it) >= 0) {
         // RoPE on this thread's 32 columns of key row `row` of K~_j, in place
         // in shared memory (the producer loaded it un-rotated): pair (2i,
@@ -522,73 +526,62 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
           }
         }
-        // ---- the previous step's dQ partial out of Y (same lanes/columns) ----
-        if (dq_tile >= 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), dqc & 1, ab, 92 + w))) { ok = false; break; }
-          ++dqc;
-          tc_fence_after();
-          drain_dq(tY, acc_bh + (size_t)dq_tile * (128 * kD), row, w);
-          dq_tile = -1;
-        }
-        // ---- P^T (bf16) into the first 16 columns of this quarter of Y ----
+        // ---- P^T (bf16) into this warp's 16 columns of P (dV(i-1), which
+        // read them, completed before S^T(i)) ----
         {
           uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(pr[2 * u], pr[2 * u + 1]);
-          tmem_st16(tY, pk);
+          tmem_st16(tP, pk);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_FULL));
-        // ---- dS^T = P^T o (dP^T - D[q]) ----
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 96 + w))) { ok = false; break; }
+        // ---- dS = P o (dP - D[q]) into the shared tile (the A operand of dK
+        // and of both dQ halves), once dP^T(i) is done and the second dQ half
+        // of the previous step has read the tile ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 96 + w) &&
+                                         (steps == 0 || mbar_wait(bar(B_DQB_FULL), (steps - 1) & 1, ab, 100 + w)))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        uint32_t ds[16];
         {
-          uint32_t r[32];
-          tmem_ld32(tX, r);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_DP_READ));  // S^T(i+1) may overwrite X now
           const float4* d4 = reinterpret_cast<const float4*>(dsum);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 Dv = d4[u];
-            const float* pp = pr + 4 * u;
-            ds[2 * u] = pack_bf16(pp[0] * (__uint_as_float(r[4 * u]) - Dv.x),
-                                  pp[1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
-            ds[2 * u + 1] = pack_bf16(pp[2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
-                                      pp[3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t r[16];
+            tmem_ld16(tX + 16u * hh, r);
+            tmem_wait_ld();
+            if (hh == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(B_DP_READ));  // S^T(i+1) may overwrite X now
+            }
+            uint32_t ds[8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 Dv = d4[4 * hh + u];
+              const float* pp = pr + 16 * hh + 4 * u;
+              ds[2 * u] = pack_bf16(pp[0] * (__uint_as_float(r[4 * u]) - Dv.x),
+                                    pp[1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
+              ds[2 * u + 1] = pack_bf16(pp[2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
+                                        pp[3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              st_shared_v4(sDSrow + (((chunk0 + 2 * hh + c) ^ swz) << 4), ds[4 * c], ds[4 * c + 1],
+                           ds[4 * c + 2], ds[4 * c + 3]);
           }
         }
-        // dS^T into the last 16 columns of this quarter of Y (A of dK), and
-        // dS into the shared tile (A of dQ; the previous dQ, which read the
-        // tile, completed before its partial was drained above)
-        tmem_st16(tY + 16u, ds);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          st_shared_v4(sDSrow + (((chunk0 + c) ^ swz) << 4), ds[4 * c], ds[4 * c + 1], ds[4 * c + 2],
-                       ds[4 * c + 3]);
         fence_proxy_async_smem();
-        tmem_wait_st();
-        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_DS_FULL));
-        dq_tile = i;
         ++steps;
         ++n;
       }
       if (!ok) break;
-      // ---- the item's last dQ partial ----
-      if (dq_tile >= 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DQ_FULL), dqc & 1, ab, 100 + w))) { ok = false; break; }
-        ++dqc;
-        tc_fence_after();
-        drain_dq(tY, acc_bh + (size_t)dq_tile * (128 * kD), row, w);
-        tc_fence_before();
-      }
       // ---- dK, dV epilogue for this key tile (this quarter's 32 columns) ----
       const size_t orow_off = (((size_t)it.b * p.S + (key_ok ? key : 0)) * p.H + it.h) * kD + 32 * w;
       if (n == 0) {
@@ -660,6 +653,59 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           x[2 * u + 1] = b;
         }
         store_row(p.dk + orow_off, p.dk32 ? p.dk32 + orow_off : nullptr, x);
+      }
+    }
+  } else {
+    // ------------------------------------------------------- dQ reducers
+    // One warp per TMEM lane quarter (warps 2, 3, 20, 21).  Each half of a
+    // step's dQ~ partial is read out of R (32 query rows x 64 columns per
+    // warp), R is handed back to the MMA warp, and the half is added into the
+    // accumulator tile with sixteen 512-byte vector reductions per warp while
+    // the other roles go on.
+    const int row = ((warp & 3) << 5) + lane;  // TMEM lane = query row of the tile
+    const uint32_t tR = tmem + ((uint32_t)((warp & 3) * 32) << 16) + 192u;
+    uint32_t steps = 0;
+    bool ok = true;
+    for (uint32_t cons = 0; ok;) {
+      const uint32_t sl = cons % kItemSlots;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 111))) {
+        ok = false;
+        break;
+      }
+      const int idx = item_slot[sl];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + sl));
+      ++cons;
+      if (idx >= n_items) break;
+      const Item it = decode(p, idx);
+      float* acc_bh = p.dq_acc + ((size_t)it.b * p.H + it.h) * (size_t)p.n_tiles * (128 * kD);
+      for (int i = first_rel(p, it); i >= 0 && ok; i = next_rel(p, it, i)) {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(h ? B_DQB_FULL : B_DQA_FULL), steps & 1, ab, 112 + h))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tR, ra);
+          tmem_ld32(tR + 32u, rb);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_R_EMPTY));
+          // columns 64h..64h+63 = column groups 16h..16h+15 of [32][128][4]
+          float* dst = acc_bh + (size_t)i * (128 * kD) + ((size_t)(16 * h) * 128 + row) * 4;
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            red_add_v4(dst + (size_t)g * 512, __uint_as_float(ra[4 * g]), __uint_as_float(ra[4 * g + 1]),
+                       __uint_as_float(ra[4 * g + 2]), __uint_as_float(ra[4 * g + 3]));
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            red_add_v4(dst + (size_t)(8 + g) * 512, __uint_as_float(rb[4 * g]), __uint_as_float(rb[4 * g + 1]),
+                       __uint_as_float(rb[4 * g + 2]), __uint_as_float(rb[4 * g + 3]));
+        }
+        ++steps;
       }
     }
   }
