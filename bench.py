@@ -64,7 +64,7 @@ def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
 # one-pass capture of the full-size 128K launch (profiles/
 # attn_bwd_fused_traffic_long_128k.md).
 FUSED_TRAFFIC = {"bytes": {"long_128k": 14.82e9 + 8.81e9},
-                 "source_sha256": "5fd22d1b8eeecfcaec4ea269951036564e770e4d3f6ec43762440492fae9d706"}
+                 "source_sha256": "3c69b60232b5a26036b8d4255a65005ee322d2cf0da4a7748ed62172daa8cde8"}
 
 
 def split_backward() -> bool:

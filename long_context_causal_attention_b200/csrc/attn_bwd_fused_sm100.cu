@@ -16,9 +16,9 @@
 // tensor memory for the whole walk.  The dQ~_i partial of each step is
 // computed in two 64-column halves; dedicated reducer warps read each half
 // out of tensor memory and add it into an fp32 accumulator in global memory
-// with vector reductions (performed in L2), so the element-wise chain never
-// waits on the L2 reduction path; a short kernel then scales the
-// accumulator, applies the inverse rotation and writes dq.  Roles (704
+// with vector reductions (performed in L2), so the element-wise warps never
+// stall behind the reduction queue themselves; a short kernel then scales
+// the accumulator, applies the inverse rotation and writes dq.  Roles (704
 // threads):
 //   warp 0      TMA producer: K_j (un-rotated: the element-wise warps apply
 //               RoPE to it in shared memory), V_j once per item; per step Q~_i
