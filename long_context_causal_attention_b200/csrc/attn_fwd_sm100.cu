@@ -302,6 +302,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int items = 0;
       bool ok = true;
       const uint32_t sq0 = base + OFF_Q;
+      const uint64_t dQ0 = kmajor_desc(sq0), dQ1 = kmajor_desc(sq0 + kTileBytes);
+      const uint64_t dK0 = kmajor_desc(base + OFF_K), dK1 = kmajor_desc(base + OFF_K + kTileBytes);
+      const uint64_t dV0 = mnmajor_desc(base + OFF_V), dV1 = mnmajor_desc(base + OFF_V + kTileBytes);
       for (uint32_t cons = 0; ok; ++items) {
         const uint32_t sl = cons % kItemSlots;
         if (!mbar_wait(bar(B_ITEM_FULL + sl), (cons / kItemSlots) & 1, ab, 14)) { ok = false; break; }
@@ -325,15 +328,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int jc = (jlo <= jhi && rel_any(p, it, jlo)) ? jlo : next_any(p, it, jlo, jhi);
         bool first_pv[2] = {true, true}, active[2] = {false, false};
 
+        // descriptors precomputed: the issuing thread's work between two
+        // products idles the tensor core, so it is kept to a minimum
         auto issue_s = [&](int t) {
-          mma_kk128(tmem + (uint32_t)(t * 128), kmajor_desc(sq0 + t * kTileBytes),
-                    kmajor_desc(base + OFF_K + (k_it & 1) * kTileBytes), kIdS, 0u);
+          mma_kk128(tmem + (uint32_t)(t * 128), t ? dQ1 : dQ0, (k_it & 1) ? dK1 : dK0, kIdS, 0u);
           mma_commit(bar(B_S_FULL + t));
         };
         auto issue_pv = [&](int t) {
           mma_tm128<false>(tmem + 256u + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128),
-                           mnmajor_desc(base + OFF_V + (v_it & 1) * kTileBytes), kIdPV,
-                           first_pv[t] ? 0u : 1u);
+                           (v_it & 1) ? dV1 : dV0, kIdPV, first_pv[t] ? 0u : 1u);
           first_pv[t] = false;
         };
 
