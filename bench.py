@@ -63,8 +63,8 @@ def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
 # The same for the one-pass backward kernel (attn_bwd_fused_kernel), from a
 # one-pass capture of the full-size 128K launch (profiles/
 # attn_bwd_fused_traffic_long_128k.md).
-FUSED_TRAFFIC = {"bytes": {"long_128k": 14.82e9 + 8.81e9},
-                 "source_sha256": "3c69b60232b5a26036b8d4255a65005ee322d2cf0da4a7748ed62172daa8cde8"}
+FUSED_TRAFFIC = {"bytes": {"long_128k": 14.79e9 + 8.80e9},
+                 "source_sha256": "49af559b0a309977a5905bcc33d642679ab5640e322670bd48e0450c0c425d82"}
 
 
 def split_backward() -> bool:
@@ -489,6 +489,16 @@ def ours(args):
                                   "GB/s": rope_bytes / (rope_ms * 1e-3) / 1e9,
                                   "frac_of_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9
                                   / float(peaks["hbm_gbs"])}}
+    if tensor_cores and not split_fp32 and not split_backward() and dq_k > 0.0:
+        # step B3 of the one-pass backward, timed in the step above: the fp32
+        # dQ~ accumulator read once, dq written once
+        n_tiles = -(-w.seqlen // 128)
+        fin_bytes = (w.batch * w.heads * n_tiles * 128 * w.head_dim * 4
+                     + w.batch * w.seqlen * w.heads * w.head_dim * q.element_size())
+        hbm_kernels["dq_finish"] = {"bytes": fin_bytes, "ms": dq_k,
+                                    "GB/s": fin_bytes / (dq_k * 1e-3) / 1e9,
+                                    "frac_of_hbm": fin_bytes / (dq_k * 1e-3) / 1e9
+                                    / float(peaks["hbm_gbs"])}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

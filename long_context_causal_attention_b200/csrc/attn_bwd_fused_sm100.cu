@@ -740,7 +740,8 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // stores); then each warp writes whole rows, lane l holding columns 4l..4l+3,
 // so a row's 256 (or 512) bytes leave in one contiguous store.
 constexpr int kFinRow = kD + 4;  // padded shared-memory row, floats
-__global__ void __launch_bounds__(128)
+constexpr int kFinThreads = 256;
+__global__ void __launch_bounds__(kFinThreads)
 dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, float* __restrict__ dq32,
                  int64_t S, int H, int n_tiles, float scale, int rotate, double log2_theta) {
   extern __shared__ float tile[];  // [128][kFinRow]
@@ -748,8 +749,8 @@ dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, 
   if (threadIdx.x < kD / 2 && rotate) freq[threadIdx.x] = rope_freq(threadIdx.x, kD, log2_theta);
   const float4* src = reinterpret_cast<const float4*>(acc + (size_t)blockIdx.x * (128 * kD));
 #pragma unroll 8
-  for (int k = 0; k < 32; ++k) {
-    const int i = threadIdx.x + 128 * k;  // float4 index: column group i / 128, row i % 128
+  for (int k = 0; k < 4096 / kFinThreads; ++k) {
+    const int i = threadIdx.x + kFinThreads * k;  // float4 index: column group i / 128, row i % 128
     *reinterpret_cast<float4*>(&tile[(i & 127) * kFinRow + (i >> 7) * 4]) = src[i];
   }
   __syncthreads();
@@ -757,7 +758,7 @@ dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, 
   const int64_t bh = blockIdx.x / n_tiles;
   const int64_t b = bh / H, h = bh % H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < 128; r += 4) {
+  for (int r = warp; r < 128; r += kFinThreads / 32) {
     const int64_t q = (int64_t)tile_i * 128 + r;
     if (q >= S) break;
     const float4 v = *reinterpret_cast<const float4*>(&tile[r * kFinRow + 4 * lane]);
@@ -849,7 +850,7 @@ cudaError_t launch_dq_finish(const Problem& pb, const Workspace& ws, void* dq, c
                                     kFinSmem);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  dq_finish_kernel<<<(unsigned)blocks, 128, kFinSmem, st>>>(
+  dq_finish_kernel<<<(unsigned)blocks, kFinThreads, kFinSmem, st>>>(
       ws.dq_acc, out_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq),
       out_f32 ? static_cast<float*>(dq) : nullptr, pb.S, (int)pb.H, (int)pb.n_tiles, pb.scale,
       rotate, rotate ? log2(pb.theta) : 0.0);
