@@ -348,8 +348,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_commit(bar(B_K_EMPTY + (k_it & 1)));
           ++k_it;
         }
+        bool q_released = false;
         while (jc >= 0 && ok) {
           const int jn = next_any(p, it, jc, jhi);
+          if (jn < 0) {
+            // every S of the item is issued: the Q tiles are free once those
+            // complete, so the producer loads the next item's Q tiles while
+            // this item's last softmax and PV products run
+            mma_commit(bar(B_Q_EMPTY));
+            q_released = true;
+          }
           bool v_ready = false, k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (rel(p, it, t, jc)) {
@@ -391,7 +399,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ++act[t];
           }
         }
-        mma_commit(bar(B_Q_EMPTY));
+        if (!q_released) mma_commit(bar(B_Q_EMPTY));
       }
     }
   } else if (warp >= 4) {
