@@ -176,3 +176,46 @@ def test_python_binding_requires_cuda_tensors(lwm):
     q = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError):
         lwm.lwm_attn_fwd(q, q, q)
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "lwm_attn.h"
+
+int main(void) {
+  lwm_attn_desc d;
+  memset(&d, 0, sizeof d);
+  d.batch = 2; d.seqlen = 300; d.heads = 4; d.head_dim = 128;
+  d.dtype = LWM_DTYPE_BF16; d.causal = 1; d.rope_theta = 1e6; d.softmax_scale = 0.0f;
+  d.segment_ids = NULL;
+  size_t f = lwm_attn_workspace_size(&d, 0), b = lwm_attn_workspace_size(&d, 1);
+  lwm_status s = lwm_attn_fwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL);
+  printf("%zu %zu %d %s %s\n", f, b, (int)s, lwm_status_string(LWM_OK),
+         lwm_status_string(LWM_ERR_INVALID_ARG));
+  return 0;
+}
+"""
+
+
+def test_c_program_compiles_against_the_header_and_links(lwm, tmp_path):
+    """The boundary is plain C: a C11 program includes the header, links the
+    library and gets the same answers as the binding (no GPU touched)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(lwm.LIB_PATH)
+    subprocess.run([cc, "-std=c11", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-llwm_attn", "-Wl,-rpath," + libdir],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    d = _desc(lwm)
+    assert int(out[0]) == lwm.lwm_attn_workspace_size(d, False)
+    assert int(out[1]) == lwm.lwm_attn_workspace_size(d, True)
+    assert int(out[2]) == -1
+    assert out[3] == "LWM_OK" and out[4].startswith("LWM_ERR_INVALID")
