@@ -538,15 +538,16 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_FULL));
-        // ---- dS = P o (dP - D[q]) into the shared tile (the A operand of dK
-        // and of both dQ halves), once dP^T(i) is done and the second dQ half
-        // of the previous step has read the tile ----
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 96 + w) &&
-                                         (steps == 0 || mbar_wait(bar(B_DQB_FULL), (steps - 1) & 1, ab, 100 + w)))) {
+        // ---- dS = P o (dP - D[q]): dP^T(i) read out of X as soon as it is
+        // done (so S^T(i+1) can start), then dS into the shared tile (the A
+        // operand of dK and of both dQ halves) once the second dQ half of the
+        // previous step has read the tile ----
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_DP_FULL), steps & 1, ab, 96 + w))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        uint32_t ds[16];
         {
           const float4* d4 = reinterpret_cast<const float4*>(dsum);
 #pragma unroll
@@ -559,22 +560,26 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
               __syncwarp();
               if (lane == 0) mbar_arrive(bar(B_DP_READ));  // S^T(i+1) may overwrite X now
             }
-            uint32_t ds[8];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const float4 Dv = d4[4 * hh + u];
               const float* pp = pr + 16 * hh + 4 * u;
-              ds[2 * u] = pack_bf16(pp[0] * (__uint_as_float(r[4 * u]) - Dv.x),
-                                    pp[1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
-              ds[2 * u + 1] = pack_bf16(pp[2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
-                                        pp[3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
+              ds[8 * hh + 2 * u] = pack_bf16(pp[0] * (__uint_as_float(r[4 * u]) - Dv.x),
+                                             pp[1] * (__uint_as_float(r[4 * u + 1]) - Dv.y));
+              ds[8 * hh + 2 * u + 1] = pack_bf16(pp[2] * (__uint_as_float(r[4 * u + 2]) - Dv.z),
+                                                 pp[3] * (__uint_as_float(r[4 * u + 3]) - Dv.w));
             }
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              st_shared_v4(sDSrow + (((chunk0 + 2 * hh + c) ^ swz) << 4), ds[4 * c], ds[4 * c + 1],
-                           ds[4 * c + 2], ds[4 * c + 3]);
           }
         }
+        // the shared dS tile is free once the previous step's second dQ half has read it
+        if (!__all_sync(0xffffffffu, steps == 0 || mbar_wait(bar(B_DQB_FULL), (steps - 1) & 1, ab, 100 + w))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(sDSrow + (((chunk0 + c) ^ swz) << 4), ds[4 * c], ds[4 * c + 1], ds[4 * c + 2],
+                       ds[4 * c + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_DS_FULL));
