@@ -457,16 +457,27 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (lane == 0) mbar_arrive(bar(B_K_ROT));
         ++kv_items;
       }
+      // segment bounds of query tile i, loaded one tile ahead so that their
+      // latency stays off the element-wise path
+      const size_t qi0 = (size_t)it.b * p.n_tiles;
+      int32_t nb0 = 0, nb1 = 0;
+      if (p.seg && it.lo <= it.hi) {
+        nb0 = p.tmin[qi0 + it.lo];
+        nb1 = p.tmax[qi0 + it.lo];
+      }
       for (int i = it.lo; i <= it.hi; ++i) {
-        if (!rel(p, it, i)) continue;
+        const int32_t a0 = nb0, a1 = nb1;
+        if (p.seg && i < it.hi) {
+          nb0 = p.tmin[qi0 + i + 1];
+          nb1 = p.tmax[qi0 + i + 1];
+        }
+        // rel(p, it, i) with the bounds already loaded
+        if (p.seg && !meet(it.kmin, it.kmax, a0, a1)) continue;
         const int64_t q0 = (int64_t)i * 128 + 32 * w;  // first query column of this quarter
         bool partial = (p.causal && i == it.j) || ((int64_t)(i + 1) * 128 > p.S) ||
                        ((int64_t)(it.j + 1) * 128 > p.S);
-        if (p.seg) {
-          const size_t qi = (size_t)it.b * p.n_tiles + i;
-          const int32_t a0 = p.tmin[qi], a1 = p.tmax[qi];
+        if (p.seg)
           partial |= !(it.kmin >= 0 && it.kmin == it.kmax && a0 == it.kmin && a1 == it.kmin);
-        }
         uint32_t mw = 0xffffffffu;
         if (partial) {
           // keep query q = q0 + c iff q < S, same segment, and q >= key when causal

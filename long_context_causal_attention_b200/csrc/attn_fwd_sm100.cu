@@ -17,7 +17,9 @@
 //               tiles, online max/sum in log2 units, write P (bf16) back
 //               into the S columns for the PV MMA, rescale O when the
 //               running max grows by more than 2^8, then normalise and
-//               store O and LSE.
+//               store O (bf16 through 2 KB of shared memory per warp, so
+//               that each store instruction writes whole 64-byte row
+//               pieces) and LSE.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
 // P_t is packed bf16 in the first 64 columns of S_t.
 // The MMA issue order ping-pongs the two tiles so one softmax warpgroup
@@ -55,7 +57,9 @@ constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;     // V ring, 2 stages
 constexpr uint32_t OFF_BAR = OFF_V + 2 * kTileBytes;   // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;           // TMEM base, abort flag
 constexpr uint32_t OFF_FREQ = OFF_MISC + 64;          // 64 RoPE frequencies, fp64
-constexpr uint32_t kSmemBytes = OFF_FREQ + 512 + 1024;  // + alignment slack
+constexpr uint32_t OFF_STG = OFF_FREQ + 512;          // O epilogue staging, 2 KB per softmax warp
+constexpr uint32_t kStgWarpBytes = 32 * 64;           // 32 rows x 32 bf16 columns
+constexpr uint32_t kSmemBytes = OFF_STG + 8 * kStgWarpBytes + 1024;  // + alignment slack
 
 // barrier slots (8 bytes each)
 enum : uint32_t {
@@ -148,6 +152,29 @@ __device__ __forceinline__ bool rel_any(const FwdParams& p, const Item& it, int 
 __device__ __forceinline__ int next_any(const FwdParams& p, const Item& it, int j, int jend) {
   for (++j; j <= jend; ++j)
     if (rel_any(p, it, j)) return j;
+  return -1;
+}
+
+// The next key tile after j that either query tile needs, and which of the
+// two need it (rn[t]); the segment bounds of each tile are loaded once.
+__device__ __forceinline__ int next_rel2(const FwdParams& p, const Item& it, int j, int jend,
+                                         bool (&rn)[2]) {
+  for (++j; j <= jend; ++j) {
+    bool r0 = it.qt[0] >= 0 && j >= it.lo[0] && j <= it.hi[0];
+    bool r1 = it.qt[1] >= 0 && j >= it.lo[1] && j <= it.hi[1];
+    if (p.seg && (r0 || r1)) {
+      const size_t kj = (size_t)it.b * p.n_tiles + j;
+      const int32_t a0 = p.ktmin[kj], a1 = p.ktmax[kj];
+      r0 = r0 && meet(it.qmin[0], it.qmax[0], a0, a1);
+      r1 = r1 && meet(it.qmin[1], it.qmax[1], a0, a1);
+    }
+    if (r0 || r1) {
+      rn[0] = r0;
+      rn[1] = r1;
+      return j;
+    }
+  }
+  rn[0] = rn[1] = false;
   return -1;
 }
 
@@ -325,7 +352,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         int jlo, jhi;
         union_range(it, &jlo, &jhi);
-        int jc = (jlo <= jhi && rel_any(p, it, jlo)) ? jlo : next_any(p, it, jlo, jhi);
+        bool rc[2];  // which query tiles need key tile jc
+        const int jc0 = next_rel2(p, it, jlo - 1, jhi, rc);
+        int jc = jlo <= jhi ? jc0 : -1;
         bool first_pv[2] = {true, true}, active[2] = {false, false};
 
         // descriptors precomputed: the issuing thread's work between two
@@ -344,13 +373,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!mbar_wait(bar(B_K_FULL + (k_it & 1)), (k_it >> 1) & 1, ab, 5)) { ok = false; break; }
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
-            if (rel(p, it, t, jc)) issue_s(t);
+            if (rc[t]) issue_s(t);
           mma_commit(bar(B_K_EMPTY + (k_it & 1)));
           ++k_it;
         }
         bool q_released = false;
         while (jc >= 0 && ok) {
-          const int jn = next_any(p, it, jc, jhi);
+          bool rn[2];
+          const int jn = next_rel2(p, it, jc, jhi, rn);
           if (jn < 0) {
             // every S of the item is issued: the Q tiles are free once those
             // complete, so the producer loads the next item's Q tiles while
@@ -360,7 +390,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           bool v_ready = false, k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
-            if (rel(p, it, t, jc)) {
+            if (rc[t]) {
               if (!v_ready) {
                 if (!mbar_wait(bar(B_V_FULL + (v_it & 1)), (v_it >> 1) & 1, ab, 6)) { ok = false; break; }
                 v_ready = true;
@@ -374,7 +404,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               issue_pv(t);
               active[t] = true;
             }
-            if (jn >= 0 && rel(p, it, t, jn)) {
+            if (jn >= 0 && rn[t]) {
               if (!k_ready) {
                 if (!mbar_wait(bar(B_K_FULL + (k_it & 1)), (k_it >> 1) & 1, ab, 9)) { ok = false; break; }
                 tc_fence_after();
@@ -391,6 +421,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_commit(bar(B_V_EMPTY + (v_it & 1)));
           ++v_it;
           jc = jn;
+          rc[0] = rn[0];
+          rc[1] = rn[1];
         }
         if (!ok) break;
         for (int t = 0; t < 2; ++t) {
@@ -424,8 +456,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (idx >= n_items) break;
       const Item it = decode(p, idx);
       const uint32_t q_phase = q_items++ & 1;  // Q_FULL completes once per item
-      if (it.qt[t] < 0) continue;
-      const int64_t row = (int64_t)it.qt[t] * 128 + tid;
+      // this warpgroup's query tile: its fields picked once, kept in registers
+      const int qt_t = t ? it.qt[1] : it.qt[0];
+      const int lo_t = t ? it.lo[1] : it.lo[0], hi_t = t ? it.hi[1] : it.hi[0];
+      const int32_t qmin_t = t ? it.qmin[1] : it.qmin[0], qmax_t = t ? it.qmax[1] : it.qmax[0];
+      if (qt_t < 0) continue;
+      const int64_t row = (int64_t)qt_t * 128 + tid;
       if (p.rotate) {
         // RoPE on this row of the Q tile, in place in shared memory: pair
         // (2i, 2i+1) turns by row * w_i, the angle reduced in fp64 and cos/sin
@@ -461,15 +497,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const size_t tok = (size_t)it.b * p.S + (size_t)(row_ok ? row : 0);
       float m = -INFINITY, l = 0.f;
       int ntiles = 0;
-      for (int j = it.lo[t]; j <= it.hi[t]; ++j) {
-        if (!rel(p, it, t, j)) continue;
+      for (int j = lo_t; j <= hi_t; ++j) {
         // tile needs element masking?
-        bool partial = (p.causal && j == it.qt[t]) || ((int64_t)(j + 1) * 128 > p.S);
+        bool partial = (p.causal && j == qt_t) || ((int64_t)(j + 1) * 128 > p.S);
         if (p.seg) {
           const size_t kj = (size_t)it.b * p.n_tiles + j;
           const int32_t a0 = p.ktmin[kj], a1 = p.ktmax[kj];
-          partial |= !(it.qmin[t] >= 0 && it.qmin[t] == it.qmax[t] && a0 == it.qmin[t] &&
-                       a1 == it.qmin[t]);
+          if (!meet(qmin_t, qmax_t, a0, a1)) continue;  // no query meets a key of tile j
+          partial |= !(qmin_t >= 0 && qmin_t == qmax_t && a0 == qmin_t && a1 == qmin_t);
+        }
+        // packing: lane c's key segment ids (columns 32w + c), loaded before
+        // the wait for S so that their latency overlaps it
+        const int64_t kvalid = p.S - (int64_t)j * 128;
+        int32_t kseg[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
+        if (partial && p.seg) {
+          const int32_t* ks = p.kseg + (size_t)it.b * p.S + (size_t)j * 128;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int64_t kc = 32 * w + lane;
+            if (kc < kvalid) kseg[w] = __ldg(ks + kc);
+          }
         }
         // every thread of the warp must agree before the .sync.aligned TMEM ops
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + t), s_cnt & 1, ab, 10 + t))) {
@@ -487,24 +534,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (partial) {
           // keys c <= lim are inside the row's causal window and the sequence
           const int64_t d = row - (int64_t)j * 128;
-          const int64_t kvalid = p.S - (int64_t)j * 128;
           int lim = p.causal ? (int)(d < -1 ? -1 : (d > 127 ? 127 : d)) : 127;
           if (kvalid - 1 < lim) lim = (int)(kvalid - 1);
           if (seg_row < 0) lim = -1;
           // 128-bit keep mask, built without touching the score registers:
-          // keys 32w + c <= lim, and (packing) the row's segment, one load per
-          // lane per 32 keys
-          const int32_t* ks = p.seg ? p.kseg + (size_t)it.b * p.S + (size_t)j * 128 : nullptr;
+          // keys 32w + c <= lim, and (packing) the row's segment
           uint32_t mw[4];
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             const int n = lim - 32 * w + 1;
             uint32_t bits = bit_range(0, n < 0 ? 0 : (n > 32 ? 32 : n));
-            if (ks) {
-              const int64_t kc = 32 * w + lane;
-              const int32_t kseg = kc < kvalid ? __ldg(ks + kc) : INT_MIN;
-              bits &= warp_segment_bits(kseg, seg_row);
-            }
+            if (p.seg) bits &= warp_segment_bits(kseg[w], seg_row);
             mw[w] = bits;
           }
 #pragma unroll
@@ -580,26 +620,58 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ++o_cnt;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_wait_ld();
-        if (row_ok && p.o32) {
+      if (p.o32) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          tmem_wait_ld();
+          if (!row_ok) continue;
           float4* dst = reinterpret_cast<float4*>(orow32 + c * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             dst[u] = make_float4(__uint_as_float(r[4 * u]) * inv, __uint_as_float(r[4 * u + 1]) * inv,
                                  __uint_as_float(r[4 * u + 2]) * inv, __uint_as_float(r[4 * u + 3]) * inv);
-        } else if (row_ok) {
+        }
+      } else {
+        // bf16 O through this warp's 2 KB of shared memory, 32 columns at a
+        // time: each lane writes its row's four 16-byte chunks, then each
+        // store instruction covers 8 rows x 64 contiguous bytes instead of 32
+        // rows x 16 bytes.  Chunk ch of row r sits at slot ch ^ ((r >> 1) & 3),
+        // which keeps both the row-wise writes and the column-wise reads free
+        // of bank conflicts.
+        const uint32_t stg = base + OFF_STG + (uint32_t)(warp - 4) * kStgWarpBytes;
+        const int rr = lane & 7, cc = lane >> 3;  // read side: rows 8k + rr, chunk cc
+        const int64_t row0 = (int64_t)qt_t * 128 + 32 * (warp & 3);  // this warp's first row
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u)
             pk[u] = pack_bf16(__uint_as_float(r[2 * u]) * inv, __uint_as_float(r[2 * u + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          for (int ch = 0; ch < 4; ++ch)
+            st_shared_v4(stg + (uint32_t)lane * 64u + (uint32_t)((ch ^ ((lane >> 1) & 3)) << 4),
+                         pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rw = 8 * k + rr;  // row within this warp's 32
+            uint32_t v[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                         : "r"(stg + (uint32_t)rw * 64u + (uint32_t)((cc ^ ((rw >> 1) & 3)) << 4)));
+            const int64_t orow_k = row0 + rw;
+            if (orow_k < p.S) {
+              __nv_bfloat16* dst =
+                  p.o + (((size_t)it.b * p.S + (size_t)orow_k) * p.H + it.h) * kD + c * 32 + cc * 8;
+              *reinterpret_cast<uint4*>(dst) = make_uint4(v[0], v[1], v[2], v[3]);
+            }
+          }
+          __syncwarp();
         }
       }
       if (row_ok)
