@@ -63,8 +63,8 @@ def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
 # The same for the one-pass backward kernel (attn_bwd_fused_kernel), from a
 # one-pass capture of the full-size 128K launch (profiles/
 # attn_bwd_fused_traffic_long_128k.md).
-FUSED_TRAFFIC = {"bytes": {"long_128k": 14.88e9 + 8.89e9},
-                 "source_sha256": "57561baea90bf93b06b385a205103922a31c1f7b3e5386c71f12b7e12856dad6"}
+FUSED_TRAFFIC = {"bytes": {"long_128k": 14.88e9 + 8.94e9},
+                 "source_sha256": "0d97416cc08e877d95a6f640a96b38fb57e0c8ddcdbec0d1161744c3439cdc82"}
 
 
 def split_backward() -> bool:

@@ -53,6 +53,8 @@
 namespace lwm {
 
 bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H, int64_t D);
+bool make_bf16_store_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H,
+                         int64_t D);
 int sm_count();
 
 namespace {
@@ -97,7 +99,8 @@ enum : uint32_t {
   B_K_ROT = 28,       // the element-wise warps rotated K~_j in place
   B_DQB_FULL = 29,    // second dQ half done: R holds it, and the dS tile is free
   B_R_EMPTY = 30,     // the reducer warps read R
-  B_COUNT = 31
+  B_STG_FREE = 31,    // every element-wise warp's epilogue stores have read the dS tile
+  B_COUNT = 32
 };
 static_assert(B_COUNT * 8 <= SOFF_MISC, "barrier slots");
 constexpr uint32_t kItemSlots = 4;
@@ -124,6 +127,8 @@ struct FusedParams {
   float scale, scale_log2;
   int causal, rotate;    // rotate: RoPE on (inverse rotation of dK, dQ)
   int rot_k;             // K_j arrives un-rotated: RoPE it in shared memory
+  int out_v8;            // the dK, dV outputs are 32-byte aligned: 256-bit row stores
+  int tma_out;           // bf16 dK, dV leave by tensor stores through the dS tile
   double log2_theta;
 };
 
@@ -184,6 +189,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                       const FusedParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -235,6 +241,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       mbar_init(bar(B_ITEM_EMPTY + sl), 1 + kEWWarps + kReducers);
     }
     mbar_init(bar(B_K_ROT), kEWWarps);
+    mbar_init(bar(B_STG_FREE), kEWWarps);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -426,7 +433,20 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const bool key_ok = key < p.S;
       const int32_t seg_k = key_ok ? (p.seg ? p.kseg[(size_t)it.b * p.S + key] : 0) : -1;
       int n = 0;
-      if (p.rot_k && first_rel(p, it) >= 0) {
+      const bool has_tiles = first_rel(p, it) >= 0;
+      if (p.tma_out && has_tiles && dkv > 0) {
+        // this item writes dS tiles: the dK/dV tensor stores of the previous
+        // item with tiles (dkv - 1), staged all over the tile, must have read
+        // it in every warp
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_STG_FREE));
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_STG_FREE), (dkv - 1) & 1, ab, 116 + w))) {
+          ok = false;
+          break;
+        }
+      }
+      if (p.rot_k && has_tiles) {
         // RoPE on this thread's 32 columns of key row `row` of K~_j, in place
         // in shared memory (the producer loaded it un-rotated): pair (2i,
         // 2i+1) turns by key * w_i, the angle reduced in fp64 and cos/sin from
@@ -625,18 +645,52 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // 32 fp32 values of a row out: bf16 pairs, or fp32 for block partials
       auto store_row = [&](__nv_bfloat16* dst16, float* dst32, const float (&x)[32]) {
         if (!key_ok) return;
+        // Each lane writes its own row: the fewer store instructions, the
+        // fewer passes the L1 makes over 32 rows, so 256-bit stores where the
+        // outputs are 32-byte aligned
         if (dst32) {
+          if (p.out_v8) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            reinterpret_cast<float4*>(dst32)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+            for (int c = 0; c < 4; ++c)
+              st_global_v8(dst32 + 8 * c, __float_as_uint(x[8 * c]), __float_as_uint(x[8 * c + 1]),
+                           __float_as_uint(x[8 * c + 2]), __float_as_uint(x[8 * c + 3]),
+                           __float_as_uint(x[8 * c + 4]), __float_as_uint(x[8 * c + 5]),
+                           __float_as_uint(x[8 * c + 6]), __float_as_uint(x[8 * c + 7]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              reinterpret_cast<float4*>(dst32)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+          }
         } else {
           uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(x[2 * u], x[2 * u + 1]);
+          if (p.out_v8) {
+            st_global_v8(dst16, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+            st_global_v8(dst16 + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
+          } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            reinterpret_cast<uint4*>(dst16)[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            for (int c = 0; c < 4; ++c)
+              reinterpret_cast<uint4*>(dst16)[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
         }
+      };
+      // tensor stores: this warp's 32 keys x 32 columns in bf16 are staged
+      // in its own dense 2 KB of the dS tile (rows of 64 bytes, 16-byte
+      // chunk c of row r at slot c ^ ((r >> 1) & 3): the 64-byte swizzle,
+      // conflict-free) and leave in one box per tensor
+      const uint32_t stg = base + OFF_DS + (uint32_t)(warp - 4) * 2048u;
+      const int krow0 = it.j * 128 + ((warp & 3) << 5);
+      auto stage_row = [&](const float (&x)[32]) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(x[2 * u], x[2 * u + 1]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(stg + (uint32_t)lane * 64u + (uint32_t)((c ^ ((lane >> 1) & 3)) << 4), pk[4 * c],
+                       pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
       };
       {
         uint32_t r[32];
@@ -645,7 +699,15 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float x[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) x[u] = __uint_as_float(r[u]);
-        store_row(p.dv + orow_off, p.dv32 ? p.dv32 + orow_off : nullptr, x);
+        if (p.tma_out) {
+          stage_row(x);
+          if (lane == 0) {
+            tma_store_4d(&tm_dv, stg, 32 * w, it.h, krow0, it.b);
+            bulk_commit();
+          }
+        } else {
+          store_row(p.dv + orow_off, p.dv32 ? p.dv32 + orow_off : nullptr, x);
+        }
       }
       {
         uint32_t r[32];
@@ -668,9 +730,20 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           x[2 * u] = a;
           x[2 * u + 1] = b;
         }
-        store_row(p.dk + orow_off, p.dk32 ? p.dk32 + orow_off : nullptr, x);
+        if (p.tma_out) {
+          if (lane == 0) bulk_wait_read0();  // dV's store has read the staging slots
+          __syncwarp();
+          stage_row(x);
+          if (lane == 0) {
+            tma_store_4d(&tm_dk, stg, 32 * w, it.h, krow0, it.b);
+            bulk_commit();
+          }
+        } else {
+          store_row(p.dk + orow_off, p.dk32 ? p.dk32 + orow_off : nullptr, x);
+        }
       }
     }
+    if (lane == 0) bulk_wait0();  // this warp's tensor stores have completed
   } else {
     // ------------------------------------------------------- dQ reducers
     // One warp per TMEM lane quarter (warps 2, 3, 20, 21).  Each half of a
@@ -806,7 +879,7 @@ size_t fused_dq_acc_bytes(int64_t B, int64_t H, int64_t n_tiles) {
 cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const void* k,
                                    const void* v, const void* d_o, void* dq, void* dk, void* dv,
                                    cudaStream_t st, bool out_f32) {
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if (!make_qkv_map(&tq, ws.q_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tk, rope_on_load_bwd(pb) ? k : ws.k_rot, pb.B, pb.S, pb.H, pb.D) ||
       !make_qkv_map(&tv, v, pb.B, pb.S, pb.H, pb.D) ||
@@ -838,6 +911,15 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.causal = pb.causal;
   p.rotate = pb.theta > 0.0;
+  // a row piece starts at a multiple of 64 bytes from the base (32 bf16 or
+  // fp32 columns), so 32-byte aligned bases make every 256-bit store aligned
+  p.out_v8 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0;
+  // bf16 outputs leave by tensor stores where both maps encode (16-byte
+  // aligned bases), else by the direct row stores
+  memset(&tdk, 0, sizeof(tdk));
+  memset(&tdv, 0, sizeof(tdv));
+  p.tma_out = !out_f32 && make_bf16_store_map(&tdk, dk, pb.B, pb.S, pb.H, pb.D) &&
+              make_bf16_store_map(&tdv, dv, pb.B, pb.S, pb.H, pb.D);
   p.rot_k = rope_on_load_bwd(pb);
   p.log2_theta = p.rotate ? log2(pb.theta) : 0.0;
   static std::once_flag attr_once;
@@ -848,7 +930,7 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int grid = (int)(n_items < sm_count() ? n_items : sm_count());
-  attn_bwd_fused_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, p);
+  attn_bwd_fused_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -745,6 +745,23 @@ bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64
   return make_bf16_map(map, ptr, B, S, H, D, 128);
 }
 
+// [B, S, H, D] bf16 tensor written by 32-row x 32-column boxes (64-byte
+// rows) from shared memory in the 64-byte swizzle: the store map of the
+// one-pass backward's dK / dV epilogue.
+bool make_bf16_store_map(CUtensorMap* map, const void* ptr, int64_t B, int64_t S, int64_t H,
+                         int64_t D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2), (cuuint64_t)(S * H * D * 2)};
+  cuuint32_t box[4] = {32, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);

@@ -58,14 +58,11 @@ struct Workspace {
 enum class Path { kSimt = 0, kSm100 = 1, kSm100X3 = 2 };
 
 // RoPE applied by the tensor-core kernels to their stationary tiles in
-// shared memory instead of a rotated copy in the workspace.  The one-pass
-// backward rotates its K tiles at every length (a work item spans many
-// query tiles, so the rotation is cheaper than the pre-pass it replaces);
-// the forward rotates its Q tiles from 64K tokens on, where the copy is
-// large: below, the copy is small and the rotation before the first MMA of
-// each short work item costs more than the pre-pass.
-constexpr int64_t kRopeOnLoadMinS = 65536;
-inline bool rope_on_load_fwd(const Problem& p) { return p.theta > 0.0 && p.S >= kRopeOnLoadMinS; }
+// shared memory instead of a rotated copy in the workspace, at every
+// length: the one-pass backward rotates its K tiles, the forward its Q
+// tiles.  Each tile is rotated once per work item, which costs less than
+// the pre-pass it replaces, even on the short work items of packed rows.
+inline bool rope_on_load_fwd(const Problem& p) { return p.theta > 0.0; }
 inline bool rope_on_load_bwd(const Problem& p) { return p.theta > 0.0; }
 
 // Which kernels serve the forward / backward of this problem on this device.

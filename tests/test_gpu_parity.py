@@ -250,13 +250,12 @@ def chunked_sum(x, chunk=65536):
 
 def test_workspace_holds_one_rotated_copy_per_pass(lwm):
     """The one-pass backward rotates its K tiles in shared memory and the
-    tensor-core forward its Q tiles from 64K tokens on, so the workspace
+    tensor-core forward its Q tiles, at every length, so the workspace
     holds one rotated copy (Q~ for the backward, K~ for the forward): with
     RoPE it exceeds the one without by one tensor (up to the 1 KB alignment
-    of its region).  Shorter forwards keep both copies (the rotation would
-    lengthen every short work item)."""
+    of its region)."""
     lib = lwm._lib.lib()
-    for S, is_bwd, copies in ((65536, False, 1), (1 << 20, False, 1), (4096, False, 2),
+    for S, is_bwd, copies in ((65536, False, 1), (1 << 20, False, 1), (4096, False, 1),
                               (65536, True, 1), (4096, True, 1)):
         nbytes = S * 32 * 128 * 2
         if True:
