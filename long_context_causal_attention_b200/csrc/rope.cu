@@ -132,40 +132,58 @@ __global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, con
 //   lse2[row] = LSE * log2(e), or +inf when the row has no allowed key or is
 //               past the end (so exp2(s - lse2) is exactly 0 there),
 //   dpad[row] = dot(dO, O), or 0 past the end.
-// A group of D / V lanes per row, V elements (16 bytes) per lane, so each row
-// of O and of dO is one contiguous load per group; 32 / (D / V) rows per warp.
+// One block per batch row and run of `tb` tokens (tb * H rows).  The dot
+// products are taken in memory order, a group of D / V lanes per (token,
+// head) row with V elements (16 bytes) per lane, so a block streams tb * H
+// * D contiguous elements of O and of dO; they go through shared memory so
+// that the outputs, laid out head-major, leave tb consecutive rows per head.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const T* __restrict__ o,
                                                        const T* __restrict__ d_o,
                                                        const float* __restrict__ lse,
                                                        float* __restrict__ lse2,
-                                                       float* __restrict__ dpad, int64_t n_rows,
-                                                       int64_t S, int64_t S_pad, int H, int D) {
+                                                       float* __restrict__ dpad, int64_t S,
+                                                       int64_t S_pad, int H, int D, int tb,
+                                                       int64_t n_chunks) {
+  extern __shared__ float dots[];  // [tb * H], token-major
   constexpr int V = 16 / sizeof(T);
   const int per_row = D / V;              // lanes per row: 4..32, a power of two
-  const int lane = threadIdx.x & 31;
+  const int rows_per_warp = 32 / per_row;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane % per_row;
-  const int64_t r = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (32 / per_row) +
-                    lane / per_row;  // r = (b * H + h) * S_pad + s
-  const int64_t s = r % S_pad, bh = r / S_pad;
-  const int64_t b = bh / H, h = bh % H;
-  const bool live = r < n_rows && s < S;
-  float acc = 0.f, L2 = INFINITY;
-  if (live) {
-    const size_t off = (((size_t)b * S + s) * H + h) * D + (size_t)sub * V;
-    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
-    const uint4 g = *reinterpret_cast<const uint4*>(d_o + off);
-    const T* ea = reinterpret_cast<const T*>(&a);
-    const T* eg = reinterpret_cast<const T*>(&g);
+  const int64_t b = blockIdx.x / n_chunks;
+  const int64_t s0 = (blockIdx.x % n_chunks) * (int64_t)tb;
+  const int n_rows = tb * H;
+  const size_t base = ((size_t)b * S + (size_t)s0) * H * D;  // first element of token s0
+#pragma unroll 4
+  for (int r0 = warp * rows_per_warp; r0 < n_rows; r0 += (blockDim.x >> 5) * rows_per_warp) {
+    const int rr = r0 + lane / per_row;  // row rr = token s0 + rr / H, head rr % H
+    float acc = 0.f;
+    if (rr < n_rows && s0 + rr / H < S) {
+      const size_t off = base + (size_t)rr * D + (size_t)sub * V;
+      const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+      const uint4 g = *reinterpret_cast<const uint4*>(d_o + off);
+      const T* ea = reinterpret_cast<const T*>(&a);
+      const T* eg = reinterpret_cast<const T*>(&g);
 #pragma unroll
-    for (int e = 0; e < V; ++e) acc += to_f32(ea[e]) * to_f32(eg[e]);
-    const float L = lse[(size_t)bh * S + s];
-    L2 = L == -INFINITY ? INFINITY : L * 1.4426950408889634f;
+      for (int e = 0; e < V; ++e) acc += to_f32(ea[e]) * to_f32(eg[e]);
+    }
+    for (int k = per_row >> 1; k > 0; k >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
+    if (rr < n_rows && sub == 0) dots[rr] = acc;
   }
-  for (int k = per_row >> 1; k > 0; k >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
-  if (r < n_rows && sub == 0) {
-    lse2[r] = L2;
-    dpad[r] = acc;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_rows; i += blockDim.x) {
+    const int h = i / tb, t = i % tb;  // head-major: tb consecutive tokens per head
+    const int64_t s = s0 + t;
+    if (s >= S_pad) continue;
+    float L2 = INFINITY;
+    if (s < S) {
+      const float L = lse[((size_t)b * H + h) * S + s];
+      L2 = L == -INFINITY ? INFINITY : L * 1.4426950408889634f;
+    }
+    const size_t out = ((size_t)b * H + h) * S_pad + s;
+    lse2[out] = L2;
+    dpad[out] = s < S ? dots[t * H + h] : 0.f;
   }
 }
 
@@ -235,18 +253,24 @@ cudaError_t launch_delta(const Problem& p, const void* o, const void* d_o, float
 cudaError_t launch_bwd_prep(const Problem& p, const void* o, const void* d_o, const float* lse,
                             const Workspace& ws, cudaStream_t st) {
   const int64_t s_pad = p.n_tiles * kTile;
-  const int64_t rows = p.B * p.H * s_pad;
-  if (rows == 0) return cudaSuccess;
-  const int64_t rows_per_warp = 32 / (p.D / (p.dtype == LWM_DTYPE_BF16 ? 8 : 4));
-  const int64_t grid = (rows + 8 * rows_per_warp - 1) / (8 * rows_per_warp);
+  if (p.B * p.H * s_pad == 0) return cudaSuccess;
+  // tokens per block: about 256 (token, head) rows, a multiple of 8 tokens
+  // where H allows (whole 32-byte sectors of the head-major outputs)
+  int tb = (int)(256 / p.H);
+  if (tb >= 8) tb &= ~7;
+  if (tb < 1) tb = 1;
+  const int64_t n_chunks = (s_pad + tb - 1) / tb;
+  const int64_t grid = p.B * n_chunks;
+  const size_t smem = (size_t)tb * p.H * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;  // H above 12288
   if (p.dtype == LWM_DTYPE_BF16)
-    bwd_prep_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, st>>>(
+    bwd_prep_kernel<__nv_bfloat16><<<(unsigned)grid, 256, smem, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse,
-        ws.lse2_pad, ws.delta_pad, rows, p.S, s_pad, (int)p.H, (int)p.D);
+        ws.lse2_pad, ws.delta_pad, p.S, s_pad, (int)p.H, (int)p.D, tb, n_chunks);
   else
-    bwd_prep_kernel<float><<<(unsigned)grid, 256, 0, st>>>(
+    bwd_prep_kernel<float><<<(unsigned)grid, 256, smem, st>>>(
         static_cast<const float*>(o), static_cast<const float*>(d_o), lse, ws.lse2_pad,
-        ws.delta_pad, rows, p.S, s_pad, (int)p.H, (int)p.D);
+        ws.delta_pad, p.S, s_pad, (int)p.H, (int)p.D, tb, n_chunks);
   note_launches(1);
   return cudaGetLastError();
 }
