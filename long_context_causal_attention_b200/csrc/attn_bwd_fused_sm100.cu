@@ -29,7 +29,8 @@
 //   warps 4-19  element-wise work, four groups of four warps (one per TMEM
 //               lane quarter, warp % 4) on 32 columns each: P^T (bf16) into
 //               tensor memory, dS into a shared-memory tile, then the dK/dV
-//               epilogue.
+//               epilogue (bf16 blocks staged in the then idle dS tile and
+//               sent by tensor stores).
 //   warps 2, 3, 20, 21  dQ reducers, one per TMEM lane quarter.
 // TMEM columns:
 //   X  [0,128)    S^T(i), then dP^T(i) once S^T(i) is in registers
