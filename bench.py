@@ -64,7 +64,7 @@ def kept_pairs(seg: np.ndarray, causal: bool = True) -> int:
 # one-pass capture of the full-size 128K launch (profiles/
 # attn_bwd_fused_traffic_long_128k.md).
 FUSED_TRAFFIC = {"bytes": {"long_128k": 14.88e9 + 8.94e9},
-                 "source_sha256": "5d7ed2116573bc06bebfea82d463419ae582a1180fadd743cb0509b9bf2cf216"}
+                 "source_sha256": "ee25513c06328c0c673b4628fb38bd0933778954cefc51950b25ab4bafbe1d33"}
 
 
 def split_backward() -> bool:

@@ -824,32 +824,38 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 }
 
 // dq = R(p)^T (scale * dQ~) in bf16 (or fp32), from the fp32 accumulator:
-// one CTA per (b, h, query tile).  The 64 KB tile ([32 column groups][128
-// rows][4]) comes in with fully coalesced 16-byte loads and is transposed
-// through shared memory (rows padded by 4 floats: conflict-free 16-byte
-// stores); then each warp writes whole rows, lane l holding columns 4l..4l+3,
-// so a row's 256 (or 512) bytes leave in one contiguous store.
+// one CTA per half (64 rows) of a (b, h, query tile).  The half's 32 KB of
+// the tile ([32 column groups][128 rows][4]: 32 runs of 1 KB) comes in with
+// fully coalesced 16-byte loads and is transposed through shared memory
+// (rows padded by 4 floats: conflict-free 16-byte stores); then each warp
+// writes whole rows, lane l holding columns 4l..4l+3, so a row's 256 (or
+// 512) bytes leave in one contiguous store.  Half tiles keep six CTAs on an
+// SM, so that loads of some overlap the stores of others.
 constexpr int kFinRow = kD + 4;  // padded shared-memory row, floats
+constexpr int kFinRows = 64;     // rows per CTA
 constexpr int kFinThreads = 256;
 __global__ void __launch_bounds__(kFinThreads)
 dq_finish_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, float* __restrict__ dq32,
                  int64_t S, int H, int n_tiles, float scale, int rotate, double log2_theta) {
-  extern __shared__ float tile[];  // [128][kFinRow]
+  extern __shared__ float tile[];  // [kFinRows][kFinRow]
   __shared__ double freq[kD / 2];
   if (threadIdx.x < kD / 2 && rotate) freq[threadIdx.x] = rope_freq(threadIdx.x, kD, log2_theta);
-  const float4* src = reinterpret_cast<const float4*>(acc + (size_t)blockIdx.x * (128 * kD));
+  const int64_t t_all = blockIdx.x >> 1;  // (b, h, query tile)
+  const int half = blockIdx.x & 1;
+  const float4* src = reinterpret_cast<const float4*>(acc + (size_t)t_all * (128 * kD)) + kFinRows * half;
 #pragma unroll 8
-  for (int k = 0; k < 4096 / kFinThreads; ++k) {
-    const int i = threadIdx.x + kFinThreads * k;  // float4 index: column group i / 128, row i % 128
-    *reinterpret_cast<float4*>(&tile[(i & 127) * kFinRow + (i >> 7) * 4]) = src[i];
+  for (int k = 0; k < 32 * kFinRows / kFinThreads; ++k) {
+    const int j = threadIdx.x + kFinThreads * k;  // column group j / 64, row j % 64 of the half
+    *reinterpret_cast<float4*>(&tile[(j & (kFinRows - 1)) * kFinRow + (j / kFinRows) * 4]) =
+        src[(j / kFinRows) * 128 + (j & (kFinRows - 1))];
   }
   __syncthreads();
-  const int tile_i = blockIdx.x % n_tiles;
-  const int64_t bh = blockIdx.x / n_tiles;
+  const int tile_i = (int)(t_all % n_tiles);
+  const int64_t bh = t_all / n_tiles;
   const int64_t b = bh / H, h = bh % H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < 128; r += kFinThreads / 32) {
-    const int64_t q = (int64_t)tile_i * 128 + r;
+  for (int r = warp; r < kFinRows; r += kFinThreads / 32) {
+    const int64_t q = (int64_t)tile_i * 128 + kFinRows * half + r;
     if (q >= S) break;
     const float4 v = *reinterpret_cast<const float4*>(&tile[r * kFinRow + 4 * lane]);
     float x[4] = {v.x * scale, v.y * scale, v.z * scale, v.w * scale};
@@ -938,10 +944,10 @@ cudaError_t launch_sm100_bwd_fused(const Problem& pb, const Workspace& ws, const
 
 cudaError_t launch_dq_finish(const Problem& pb, const Workspace& ws, void* dq, cudaStream_t st,
                              bool out_f32) {
-  const int64_t blocks = pb.B * pb.H * pb.n_tiles;
+  const int64_t blocks = 2 * pb.B * pb.H * pb.n_tiles;  // two half tiles each
   if (blocks == 0) return cudaSuccess;
   const int rotate = pb.theta > 0.0;
-  constexpr int kFinSmem = 128 * kFinRow * (int)sizeof(float);
+  constexpr int kFinSmem = kFinRows * kFinRow * (int)sizeof(float);
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
