@@ -89,10 +89,13 @@ typedef struct {
 } lwm_attn_desc;
 
 /* Bytes of device workspace lwm_attn_fwd (is_bwd = 0) or lwm_attn_bwd
- * (is_bwd != 0) needs for `desc`; 0 if `desc` is invalid.  The workspace
- * holds the status word, per-tile segment bounds, the rotated Q and K and,
- * for the backward, the per-row LSE and dot(dO, O) (fp32, padded to whole
- * tiles for the tensor-core kernels).
+ * (is_bwd != 0) needs for `desc` on the current device; 0 if `desc` is
+ * invalid.  The workspace holds the status word, per-tile segment bounds,
+ * the rotated copies the chosen kernels read (K for the tensor-core forward,
+ * which rotates its Q tiles itself; Q for the one-pass backward, which
+ * rotates its K tiles; both for the other kernels) and, for the backward,
+ * the per-row LSE and dot(dO, O) (fp32, padded to whole tiles for the
+ * tensor-core kernels) and the one-pass backward's fp32 dQ accumulator.
  * The forward's need is never larger than the backward's. */
 size_t lwm_attn_workspace_size(const lwm_attn_desc* desc, int is_bwd);
 
@@ -126,8 +129,10 @@ lwm_status lwm_attn_bwd(const lwm_attn_desc* desc, const void* q, const void* k,
  * after start-up, or a host that must not risk the implicit synchronisation
  * or out-of-memory failure an allocation can bring at that point.  The
  * caller still passes q, k, v, o and lse (same meaning as lwm_attn_fwd).
- *   - Scratch limit: 40 MiB, enough for about 10M bf16 elements per tensor
- *     (e.g. 2,048 tokens x 32 heads x 128).  A problem whose workspace
+ *   - Scratch limit: 40 MiB.  On the tensor-core forward (one rotated
+ *     copy) that is about 20M bf16 elements per tensor (e.g. 4,096 tokens
+ *     x 32 heads x 128); where q and k are both pre-rotated, about 10M.
+ *     A problem whose workspace
  *     (lwm_attn_workspace_size(desc, 0)) is larger returns
  *     LWM_ERR_WORKSPACE and launches nothing.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
